@@ -1,0 +1,414 @@
+"""Benchmark of the paged decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: the paged cache write
+of this step's new K/V (one token per sequence) followed by decode attention of
+every sequence over its paged cache.  The default workload is the LLaMA-2-7B
+layer shape (64 sequences x 2048 tokens, 32 heads MHA, head_dim 128, fp16,
+blocks shuffled across a 12288-block pool).  The KV read of one step (2 GiB) is
+larger than the 126 MB L2, so no flush is needed between steps.
+
+Prints ONE JSON line (rank 0).  `value` is whole-job achieved HBM GB/s: decode
+bytes (sum_s len_s * Hkv * D * 2 * kv_bytes + q + out) of every rank's step
+divided by the max-over-ranks device time of a step.  Multi-GPU runs are
+independent replicas (the path has no exchange step).  `--impl reference`
+times the fp64 CPU oracle on a bounded sample of the same workload instead.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from paged_kv_cache_463_b200 import binding as pab  # noqa: E402
+from paged_kv_cache_463_b200 import workloads as wl  # noqa: E402
+
+METRIC = "paged decode: achieved HBM GB/s (% of B200 peak) and seq-steps/sec"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+DEFAULT_WORKLOAD = "llama2-7b-mha"
+
+
+# ---------------------------------------------------------------- helpers
+def measured_hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_record(kernel_name: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    h = hashlib.sha256()
+    for f in ("decode.cuh", "ptx.cuh", "paged_attn.cu"):
+        with open(os.path.join(ROOT, "paged_kv_cache_463_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    digest = h.hexdigest()[:16]
+    for line in open(path, encoding="utf-8"):
+        parts = line.split()
+        if len(parts) >= 4 and parts[0] == kernel_name and parts[1] == workload and parts[2] == digest:
+            return float(parts[3])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        sms, maxes, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                sms.append(float(p[1]))
+                maxes.append(float(p[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, p[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sms:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sms), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
+                "samples": len(sms)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device(f"cuda:{local}"))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- CPU oracle leg
+def oracle_sample(spec: wl.WorkloadSpec, budget_s: float, max_seqs: int | None = None):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the workload:
+    the first k sequences of a seeded copy of the workload restricted to them.
+    Returns (GB/s under the decode byte formula, seq-steps/s, description, threads)."""
+    import numpy as np
+    from oracle import attention, cache_write  # the oracle: test infrastructure, CPU baseline only
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    k_total, t_total, bytes_total, seqs_done = 0, 0.0, 0, 0
+    k = 1
+    while True:
+        sub = wl.scaled(spec, num_seqs=k, pool_blocks=None,
+                        prefix_groups=min(spec.prefix_groups, 1) if spec.prefix_groups else 0)
+        w = wl.make_workload(sub, "cpu")
+        raw = _raw_numpy(w)
+        t0 = time.perf_counter()
+        kc, vc = raw["kc"].copy(), raw["vc"].copy()
+        cache_write.reshape_and_cache(raw["nk"], raw["nv"], kc, vc, raw["slots"], src_dtype=sub.q_dtype,
+                                      cache_dtype=sub.kv_dtype, k_scale=w.k_scale, v_scale=w.v_scale)
+        attention.decode_attention(raw["q"], kc, vc, raw["bt"], raw["lens"], w.scale, q_dtype=sub.q_dtype,
+                                   kv_dtype=sub.kv_dtype, k_scale=w.k_scale, v_scale=w.v_scale)
+        dt = time.perf_counter() - t0
+        t_total += dt
+        bytes_total += wl.decode_bytes(w)
+        seqs_done += k
+        k_total += 1
+        if t_total >= budget_s or (max_seqs is not None and seqs_done >= max_seqs):
+            break
+        k = min(2 * k, spec.num_seqs)
+    desc = (f"{seqs_done} sequences of {spec.name} ({k_total} oracle call(s); per sequence all "
+            f"{spec.num_heads} heads over its full length), cache write + fp64 decode attention")
+    return bytes_total / t_total / 1e9, seqs_done / t_total, desc, threads, t_total
+
+
+def _raw_numpy(w):
+    import numpy as np
+    def r(t):
+        t = t.cpu()
+        if t.dtype == torch.bfloat16:
+            return t.view(torch.int16).numpy().view(np.uint16)
+        if t.dtype == torch.float8_e4m3fn:
+            return t.view(torch.uint8).numpy()
+        return t.numpy()
+    d = {"q": r(w.query), "nk": r(w.new_key), "nv": r(w.new_value), "slots": r(w.slot_mapping),
+         "bt": r(w.block_tables), "lens": r(w.seq_lens)}
+    if w.spec.kv_dtype == "fp8_e4m3":
+        from oracle import cache_write
+        d["kc"] = cache_write.quantize(r(w.key_src), w.spec.q_dtype, w.k_scale)
+        d["vc"] = cache_write.quantize(r(w.value_src), w.spec.q_dtype, w.v_scale)
+    else:
+        d["kc"], d["vc"] = r(w.key_cache), r(w.value_cache)
+    return d
+
+
+# ---------------------------------------------------------------- arms
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    spec = wl.SPEC_BY_NAME[args.workload]
+    per_step_budget = max(2.0, 60.0 / max(1, args.steps + args.warmup))
+    vals, rates = [], []
+    desc, threads, elapsed = "", 1, 0.0
+    for i in range(args.warmup + args.steps):
+        gbs, sps, desc, threads, el = oracle_sample(spec, per_step_budget, max_seqs=2)
+        if i >= args.warmup:
+            vals.append(gbs)
+            rates.append(sps)
+            elapsed += el
+    value = statistics.median(vals)
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": spec.name, "description": spec.description},
+            "seq_steps_per_s": statistics.median(rates),
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_ours(args, world, rank, local):
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU (the product path has no CPU fallback)")
+    from paged_kv_cache_463_b200 import build
+    build.build()
+    spec = wl.SPEC_BY_NAME[args.workload]
+    dev = f"cuda:{local}"
+    w = wl.make_workload(spec, dev)
+    part = {"auto": pab.PA_PARTITION_AUTO, "none": pab.PA_PARTITION_NONE}.get(args.partition)
+    part = int(args.partition) if part is None else part
+    pa = pab.PagedAttention(spec.num_heads, spec.num_kv_heads, spec.head_dim, w.num_blocks,
+                            block_size=spec.block_size, q_dtype=spec.q_dtype, kv_dtype=spec.kv_dtype,
+                            max_num_seqs=spec.num_seqs, max_blocks_per_seq=w.block_tables.shape[1],
+                            partition_tokens=part, device=local)
+    if spec.kv_dtype == "fp8_e4m3":
+        NB, bs, Hkv, D = w.key_src.shape
+        kc = torch.empty((NB, bs, Hkv, D), dtype=torch.float8_e4m3fn, device=dev)
+        vc = torch.empty_like(kc)
+        pa.reshape_and_cache(w.key_src.view(-1, Hkv, D), w.value_src.view(-1, Hkv, D), kc, vc,
+                             torch.arange(NB * bs, dtype=torch.int64, device=dev), w.k_scale, w.v_scale)
+        w.key_src = w.value_src = None
+    else:
+        kc, vc = w.key_cache, w.value_cache
+    out = torch.empty_like(w.query)
+    stream = torch.cuda.current_stream()
+    max_len = w.max_seq_len
+    chosen_part = pa.partition_tokens(spec.num_seqs, max_len)
+    split = chosen_part > 0 and max_len > chosen_part
+    launches_per_step = 2 + (1 if split else 0)
+
+    def step():
+        pa.reshape_and_cache(w.new_key, w.new_value, kc, vc, w.slot_mapping, w.k_scale, w.v_scale, stream)
+        pa.paged_attention_decode(out, w.query, kc, vc, w.block_tables, w.seq_lens, max_len, w.scale,
+                                  w.k_scale, w.v_scale, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if pa.get_error() != 0:
+        raise SystemExit("device check fired during warm-up")
+
+    # ---- device-timed region: whole steps, plus the decode call inside each
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            a, m, e = ev[i]
+            a.record(stream)
+            pa.reshape_and_cache(w.new_key, w.new_value, kc, vc, w.slot_mapping, w.k_scale, w.v_scale, stream)
+            m.record(stream)
+            pa.paged_attention_decode(out, w.query, kc, vc, w.block_tables, w.seq_lens, max_len, w.scale,
+                                      w.k_scale, w.v_scale, stream)
+            e.record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = t_start.elapsed_time(t_end)
+    decode_ms = [m.elapsed_time(e) for (_, m, e) in ev]
+    write_ms = [a.elapsed_time(m) for (a, m, _) in ev]
+    total_ms = max_over_ranks(total_ms, world)
+    if pa.get_error() != 0:
+        raise SystemExit("device check fired during the timed region")
+
+    dec_bytes = wl.decode_bytes(w)
+    S = spec.num_seqs
+    ms_per_step = total_ms / args.steps
+    value = world * dec_bytes * args.steps / (total_ms * 1e-3) / 1e9
+    seq_steps = world * S * args.steps / (total_ms * 1e-3)
+
+    # ---- end to end through the public API: pinned host inputs -> device, the
+    # two calls, result -> pinned host, every step
+    host = {k: getattr(w, k).cpu().pin_memory() for k in ("new_key", "new_value", "query", "slot_mapping",
+                                                          "block_tables", "seq_lens")}
+    dev_in = {k: torch.empty_like(getattr(w, k)) for k in host}
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+
+    def e2e_step():
+        for k, t in host.items():
+            dev_in[k].copy_(t, non_blocking=True)
+        pa.reshape_and_cache(dev_in["new_key"], dev_in["new_value"], kc, vc, dev_in["slot_mapping"], w.k_scale,
+                             w.v_scale, stream)
+        pa.paged_attention_decode(out, dev_in["query"], kc, vc, dev_in["block_tables"], dev_in["seq_lens"],
+                                  max_len, w.scale, w.k_scale, w.v_scale, stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    barrier(world)
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    s1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1), world)
+    e2e_value = world * dec_bytes * args.steps / (e2e_ms * 1e-3) / 1e9
+
+    peak, peak_kind = measured_hbm_peak()
+    dec_avg_ms = sum(decode_ms) / len(decode_ms)
+    achieved = dec_bytes / (dec_avg_ms * 1e-3) / 1e9
+    traffic = traffic_record("paged_decode_kernel", spec.name)
+    result = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": {"f16": "f16", "bf16": "bf16", "fp8_e4m3": "fp8_e4m3"}[spec.kv_dtype],
+        "data": "synthetic",
+        "config": {"workload": spec.name, "description": spec.description, "num_seqs": S,
+                   "num_heads": spec.num_heads, "num_kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim,
+                   "block_size": spec.block_size, "kv_dtype": spec.kv_dtype, "q_dtype": spec.q_dtype,
+                   "sum_seq_len": int(w.seq_lens.sum().item()), "partition_tokens": chosen_part,
+                   "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "seq_steps_per_s": seq_steps,
+        "pct_of_nominal_8tbs": 100.0 * value / world / NOMINAL_HBM_GBS,
+        "pct_of_measured_copy": 100.0 * value / world / peak,
+        "bytes_per_step": dec_bytes,
+        "decode_ms": dec_avg_ms, "cache_write_ms": sum(write_ms) / len(write_ms),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "kernel": "paged_decode_kernel" + (" + merge" if split else ""),
+                     "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_kind == "measured" else "fallback 6.65 TB/s"},
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms / args.steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, sps, desc, threads, el = oracle_sample(spec, args.cpu_budget)
+        result["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                  "sample": desc, "seq_steps_per_s": sps, "seconds": el}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    pa.close()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(wl.SPEC_BY_NAME))
+    ap.add_argument("--partition", default="auto", help="auto | none | tokens per partition")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    world, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            return run_reference(args, world, rank)
+        return run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,201 @@
+/*
+ * paged_attn.h -- C ABI of a B200 (sm_100a) library for the decode hot path of
+ * PagedAttention: the per-step paged cache write and decode attention over a
+ * block-paged KV cache.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - Pointers named *_cache, key, value, query, out, block_table(s), seq_lens,
+ *   slot_mapping, k_out, v_out are DEVICE pointers into memory the caller owns
+ *   (e.g. torch tensors); the library never frees or keeps them after a call
+ *   returns.  `stream` is a cudaStream_t (NULL = legacy default stream).
+ * - Calls validate their arguments on the host first; an invalid call returns
+ *   a negative status and launches nothing.  Valid calls only enqueue work on
+ *   `stream` and return PA_OK without synchronising.
+ * - Data-dependent problems (a block id outside the pool, a slot outside the
+ *   cache, a sequence longer than its table, a pipeline wait that ran out) are
+ *   caught on the device: the offending access is skipped (or redirected to
+ *   block 0), a bit is or-ed into the context's check word, and
+ *   paged_attn_get_error() reports it.  Nothing traps, asserts or spins
+ *   without bound.
+ * - Layouts (row-major, element = the dtype named):
+ *     query, out           [num_seqs, num_heads, head_dim]
+ *     key_cache/value_cache [num_blocks, block_size, num_kv_heads, head_dim]
+ *     block_tables         int32 [num_seqs, bt_stride]; entry j of row s is the
+ *                          physical block holding tokens [16 j, 16 j + 16) of s;
+ *                          entries past the sequence's last block are never read
+ *                          (page "5.KV Cache 管理 & PagedAttention", Q8.3 uses -1)
+ *     seq_lens             int32 [num_seqs], tokens cached for each sequence
+ *                          (including the one written by this step)
+ *     slot_mapping         int64 [num_tokens], slot = block * block_size + offset
+ *   A context is used from one host thread at a time.
+ */
+#ifndef PAGED_ATTN_H_
+#define PAGED_ATTN_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes */
+#define PA_OK 0
+#define PA_ERR_INVALID_ARG (-1)  /* null pointer, bad shape/stride/alignment, size beyond the context's limits */
+#define PA_ERR_UNSUPPORTED (-2)  /* dtype / head_dim / block_size combination not built */
+#define PA_ERR_CUDA (-3)         /* a CUDA runtime call failed; paged_attn_last_error() has the message */
+#define PA_ERR_DEVICE_CHECK (-4) /* a device-side check fired; paged_attn_last_check_bits() says which */
+#define PA_ERR_NO_MEMORY (-5)    /* workspace allocation failed */
+
+/* ---- device check bits (paged_attn_last_check_bits) */
+#define PA_CHECK_BAD_BLOCK 1    /* block-table entry outside [0, num_blocks): read block 0 instead */
+#define PA_CHECK_BAD_SLOT 2     /* slot >= num_blocks * block_size: write skipped */
+#define PA_CHECK_SEQ_TOO_LONG 4 /* seq_len > bt_stride * block_size, < 0, or beyond max_seq_len: clamped */
+#define PA_CHECK_WAIT_TIMEOUT 8 /* a shared-memory pipeline wait gave up: that CTA's output is invalid */
+
+/* ---- element types */
+typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
+
+/* partition_tokens special values */
+#define PA_PARTITION_NONE 0  /* never split a sequence across CTAs */
+#define PA_PARTITION_AUTO (-1)
+
+/*
+ * Fixed shape of one attention layer's cache and of the batches it serves.
+ *   num_heads, num_kv_heads : query heads and KV heads; num_heads % num_kv_heads == 0.
+ *                             Query head h reads KV head h / (num_heads / num_kv_heads)
+ *                             (grouped-query attention, page "5.KV Cache 管理 &
+ *                             PagedAttention", Q7 repeat_interleave; MHA when equal).
+ *   head_dim                : 64, 128 or 256 for 16-bit caches; 128 or 256 for fp8.
+ *   block_size              : tokens per physical block; 16 (the pages' default,
+ *                             page "KV Cache 优化与内存管理深度解析", BlockSizeSelection).
+ *   num_blocks              : physical blocks in each of key_cache / value_cache.
+ *   q_dtype                 : PA_F16 or PA_BF16 (query, out and the new K/V rows).
+ *   kv_dtype                : PA_F16 / PA_BF16 (must equal q_dtype) or PA_FP8_E4M3
+ *                             (with q_dtype PA_F16); fp8 values carry one scale per
+ *                             cache tensor (value = code * scale).
+ *   max_num_seqs            : largest num_seqs a decode call may pass.
+ *   max_blocks_per_seq      : largest ceil(max_seq_len / block_size) a call may pass.
+ *   partition_tokens        : split-KV partition length (a multiple of block_size),
+ *                             PA_PARTITION_NONE, or PA_PARTITION_AUTO (512-token
+ *                             partitions when a batch would otherwise leave SMs idle).
+ *   device                  : CUDA device ordinal the context and its calls use.
+ *   flags                   : reserved, must be 0.
+ */
+typedef struct pa_config {
+  int num_heads;
+  int num_kv_heads;
+  int head_dim;
+  int block_size;
+  int num_blocks;
+  int q_dtype;
+  int kv_dtype;
+  int max_num_seqs;
+  int max_blocks_per_seq;
+  int partition_tokens;
+  int device;
+  int flags;
+} pa_config;
+
+typedef struct pa_ctx pa_ctx;
+
+/*
+ * Create a context: validates `cfg`, allocates the split-KV workspace
+ * (max_num_seqs * num_heads * max_partitions * (head_dim + 2) floats) and the
+ * device check word on cfg->device.  On success *out owns them.
+ * Returns PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED, PA_ERR_NO_MEMORY or
+ * PA_ERR_CUDA (e.g. no GPU).  *out is NULL on failure.
+ */
+int paged_attn_create(const pa_config* cfg, pa_ctx** out);
+
+/* Free the context's workspace.  Does not synchronise the caller's streams:
+ * the caller must make sure no call on the context is still running. */
+int paged_attn_destroy(pa_ctx* ctx);
+
+/*
+ * Paged cache write (page "5.KV Cache 管理 & PagedAttention", Q12 append_token:
+ * the new token's K/V go to (block_table[len / block_size], len % block_size)).
+ * For every token t in [0, num_tokens) with slot = slot_mapping[t] >= 0:
+ *     key_cache[slot / block_size, slot % block_size, :, :] = key[t, :, :]
+ *     value_cache[...]                                     = value[t, :, :]
+ * key/value: [num_tokens, num_kv_heads, head_dim] of q_dtype, with row strides
+ * key_token_stride / value_token_stride in elements (multiples of 8; pointers
+ * 16-byte aligned).  16-bit caches receive the bytes unchanged.  An fp8 cache
+ * receives E4M3(x / k_scale) (values: v_scale): IEEE fp32 division, round to
+ * nearest even, saturating at +-448.  Slots < 0 are skipped; slots beyond the
+ * cache set PA_CHECK_BAD_SLOT and are skipped.  Two tokens with the same slot
+ * in one call: which one lands is unspecified.
+ */
+int reshape_and_cache(pa_ctx* ctx, const void* key, const void* value, int64_t key_token_stride,
+                      int64_t value_token_stride, void* key_cache, void* value_cache,
+                      const int64_t* slot_mapping, int num_tokens, float k_scale, float v_scale,
+                      void* stream);
+
+/*
+ * Decode attention over the paged cache (page "5.KV Cache 管理 & PagedAttention",
+ * Q4 decode_step step 4 and Q13; listing paged_attention on page
+ * "paged-attention-and-vllm-inference"): for each sequence s < num_seqs and
+ * query head h,
+ *     out[s, h, :] = sum_j softmax_j(scale * q[s,h,:] . K[s,j,:]) V[s,j,:]
+ * over the seq_lens[s] tokens j of s, K[s,j] = key_cache[block_tables[s, j/16],
+ * j%16, h / (num_heads/num_kv_heads)].  fp8 caches are decoded as code*k_scale
+ * and code*v_scale (k_scale, v_scale ignored for 16-bit caches).  Arithmetic is
+ * fp32 (products of 16-bit operands on tensor cores); out is rounded once to
+ * q_dtype.  seq_lens[s] == 0 gives a zero row.
+ * max_seq_len: a host-side upper bound of seq_lens (sizes the partition grid
+ * without a device->host read); 0 <= max_seq_len <= max_blocks_per_seq *
+ * block_size.  Sequences longer than it, or than bt_stride * block_size, are
+ * truncated and flagged (PA_CHECK_SEQ_TOO_LONG).
+ * bt_stride: row stride of block_tables in entries (>= 1).
+ * Pointers: out/query 16-byte aligned, caches 16-byte aligned.
+ * Launches one partition kernel, plus one merge kernel when a sequence spans
+ * several partitions.
+ */
+int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, const void* key_cache,
+                           const void* value_cache, const int32_t* block_tables, int bt_stride,
+                           const int32_t* seq_lens, int num_seqs, int max_seq_len, float scale, float k_scale,
+                           float v_scale, void* stream);
+
+/*
+ * Synchronise `stream`, read and clear the context's device check word.
+ * Returns PA_OK when no check fired since the last call, PA_ERR_DEVICE_CHECK
+ * otherwise (the bits are then in paged_attn_last_check_bits), PA_ERR_CUDA if
+ * the synchronisation failed.
+ */
+int paged_attn_get_error(pa_ctx* ctx, void* stream);
+
+/* Check bits seen by the last paged_attn_get_error (PA_CHECK_*). */
+int paged_attn_last_check_bits(const pa_ctx* ctx);
+
+/* Static description of a status code. */
+const char* paged_attn_status_string(int status);
+
+/* Message of the last PA_ERR_CUDA / validation failure on this context ("" if none). */
+const char* paged_attn_last_error(const pa_ctx* ctx);
+
+/*
+ * Override the split-KV partition length for later decode calls:
+ * PA_PARTITION_NONE, PA_PARTITION_AUTO, or a multiple of block_size no smaller
+ * than the context's workspace allows (cfg.partition_tokens if positive, else 512).
+ */
+int paged_attn_set_partition_tokens(pa_ctx* ctx, int partition_tokens);
+
+/* Partition length (tokens) the next decode call with these sizes would use;
+ * 0 means one partition per sequence.  Negative status on bad arguments. */
+int paged_attn_partition_tokens(const pa_ctx* ctx, int num_seqs, int max_seq_len);
+
+/*
+ * Gather (page "5.KV Cache 管理 & PagedAttention", Q11 read_kv_range): copy
+ * tokens [0, seq_len) of one sequence out of the paged caches into contiguous
+ * k_out / v_out [seq_len, num_kv_heads, head_dim] (cache dtype, bytes
+ * unchanged).  block_table_row: device int32 [>= ceil(seq_len / block_size)].
+ * Entries outside the pool set PA_CHECK_BAD_BLOCK and yield zero rows.
+ */
+int paged_gather_kv(pa_ctx* ctx, void* k_out, void* v_out, const void* key_cache, const void* value_cache,
+                    const int32_t* block_table_row, int seq_len, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGED_ATTN_H_ */

@@ -1,0 +1,182 @@
+"""ctypes binding of ``libpaged_attn.so`` (include/paged_attn.h).
+
+Argument marshalling only: torch tensors are passed as device pointers plus
+sizes, the stream is torch's current stream unless one is given, and every
+step of the computation runs in the library's kernels.  There is no fallback:
+if the library is missing or a call fails, an exception is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+DEFAULT_LIB = os.path.join(_PKG, "lib", "libpaged_attn.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "paged_attn.h")
+
+PA_OK = 0
+PA_ERR_INVALID_ARG = -1
+PA_ERR_UNSUPPORTED = -2
+PA_ERR_CUDA = -3
+PA_ERR_DEVICE_CHECK = -4
+PA_ERR_NO_MEMORY = -5
+PA_CHECK_BAD_BLOCK, PA_CHECK_BAD_SLOT, PA_CHECK_SEQ_TOO_LONG, PA_CHECK_WAIT_TIMEOUT = 1, 2, 4, 8
+PA_PARTITION_NONE, PA_PARTITION_AUTO = 0, -1
+DTYPE_CODES = {"f16": 0, "bf16": 1, "fp8_e4m3": 2}
+TORCH_OF = {"f16": torch.float16, "bf16": torch.bfloat16, "fp8_e4m3": torch.float8_e4m3fn}
+
+
+class PaConfig(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in (
+        "num_heads", "num_kv_heads", "head_dim", "block_size", "num_blocks", "q_dtype", "kv_dtype",
+        "max_num_seqs", "max_blocks_per_seq", "partition_tokens", "device", "flags")]
+
+
+class PagedAttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(what)
+        self.status = status
+
+
+_LIBS: dict[str, ctypes.CDLL] = {}
+_P = ctypes.c_void_p
+
+
+def load_library(path: str | None = None) -> ctypes.CDLL:
+    """Load (once) and type the library; raises if it is not built."""
+    path = os.path.abspath(path or DEFAULT_LIB)
+    if path in _LIBS:
+        return _LIBS[path]
+    if not os.path.exists(path):
+        raise PagedAttnError(PA_ERR_CUDA, f"{path} not built: run `python -m paged_kv_cache_463_b200.build`")
+    lib = ctypes.CDLL(path)
+    i, i64, f = ctypes.c_int, ctypes.c_int64, ctypes.c_float
+    sig = {
+        "paged_attn_create": (i, [ctypes.POINTER(PaConfig), ctypes.POINTER(_P)]),
+        "paged_attn_destroy": (i, [_P]),
+        "reshape_and_cache": (i, [_P, _P, _P, i64, i64, _P, _P, _P, i, f, f, _P]),
+        "paged_attention_decode": (i, [_P, _P, _P, _P, _P, _P, i, _P, i, i, f, f, f, _P]),
+        "paged_attn_get_error": (i, [_P, _P]),
+        "paged_attn_last_check_bits": (i, [_P]),
+        "paged_attn_status_string": (ctypes.c_char_p, [i]),
+        "paged_attn_last_error": (ctypes.c_char_p, [_P]),
+        "paged_attn_set_partition_tokens": (i, [_P, i]),
+        "paged_attn_partition_tokens": (i, [_P, i, i]),
+        "paged_gather_kv": (i, [_P, _P, _P, _P, _P, _P, i, _P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _LIBS[path] = lib
+    return lib
+
+
+def header_functions(header: str = HEADER) -> list[str]:
+    """Names of the functions include/paged_attn.h declares."""
+    text = open(header, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w ]*?\**\s*\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)))
+
+
+def _stream_ptr(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+class PagedAttention:
+    """One attention layer's paged-cache shape bound to a library context."""
+
+    def __init__(self, num_heads: int, num_kv_heads: int, head_dim: int, num_blocks: int, *, block_size: int = 16,
+                 q_dtype: str = "f16", kv_dtype: str = "f16", max_num_seqs: int, max_blocks_per_seq: int,
+                 partition_tokens: int = PA_PARTITION_AUTO, device: int | None = None, lib_path: str | None = None):
+        self.lib = load_library(lib_path)
+        if device is None:
+            device = torch.cuda.current_device() if torch.cuda.is_available() else 0
+        self.cfg = PaConfig(num_heads, num_kv_heads, head_dim, block_size, num_blocks, DTYPE_CODES[q_dtype],
+                            DTYPE_CODES[kv_dtype], max_num_seqs, max_blocks_per_seq, partition_tokens, device, 0)
+        self.q_dtype, self.kv_dtype = q_dtype, kv_dtype
+        self.device = device
+        ctx = _P()
+        st = self.lib.paged_attn_create(ctypes.byref(self.cfg), ctypes.byref(ctx))
+        if st != PA_OK:
+            raise PagedAttnError(st, f"paged_attn_create: {self.lib.paged_attn_status_string(st).decode()}")
+        self.ctx = ctx
+
+    # -- helpers
+    def _check(self, st: int, what: str) -> None:
+        if st != PA_OK:
+            msg = self.lib.paged_attn_last_error(self.ctx).decode()
+            raise PagedAttnError(st, f"{what}: {self.lib.paged_attn_status_string(st).decode()} {msg}".strip())
+
+    def close(self) -> None:
+        if getattr(self, "ctx", None):
+            self.lib.paged_attn_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    # -- the C ABI, one method per entry point
+    def reshape_and_cache(self, key, value, key_cache, value_cache, slot_mapping, k_scale=1.0, v_scale=1.0,
+                          stream=None) -> None:
+        st = self.lib.reshape_and_cache(self.ctx, _ptr(key), _ptr(value), key.stride(0), value.stride(0),
+                                        _ptr(key_cache), _ptr(value_cache), _ptr(slot_mapping), key.shape[0],
+                                        float(k_scale), float(v_scale), _stream_ptr(stream))
+        self._check(st, "reshape_and_cache")
+
+    def paged_attention_decode(self, out, query, key_cache, value_cache, block_tables, seq_lens, max_seq_len: int,
+                               scale: float, k_scale=1.0, v_scale=1.0, stream=None) -> None:
+        st = self.lib.paged_attention_decode(self.ctx, _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+                                             _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens),
+                                             query.shape[0], int(max_seq_len), float(scale), float(k_scale),
+                                             float(v_scale), _stream_ptr(stream))
+        self._check(st, "paged_attention_decode")
+
+    def paged_gather_kv(self, k_out, v_out, key_cache, value_cache, block_table_row, seq_len: int,
+                        stream=None) -> None:
+        st = self.lib.paged_gather_kv(self.ctx, _ptr(k_out), _ptr(v_out), _ptr(key_cache), _ptr(value_cache),
+                                      _ptr(block_table_row), int(seq_len), _stream_ptr(stream))
+        self._check(st, "paged_gather_kv")
+
+    def get_error(self, stream=None) -> int:
+        """Synchronise and return (then clear) the device check bits."""
+        st = self.lib.paged_attn_get_error(self.ctx, _stream_ptr(stream))
+        if st == PA_ERR_DEVICE_CHECK:
+            return self.lib.paged_attn_last_check_bits(self.ctx)
+        self._check(st, "paged_attn_get_error")
+        return 0
+
+    def set_partition_tokens(self, n: int) -> None:
+        self._check(self.lib.paged_attn_set_partition_tokens(self.ctx, int(n)), "paged_attn_set_partition_tokens")
+
+    def partition_tokens(self, num_seqs: int, max_seq_len: int) -> int:
+        r = self.lib.paged_attn_partition_tokens(self.ctx, int(num_seqs), int(max_seq_len))
+        if r < 0:
+            self._check(r, "paged_attn_partition_tokens")
+        return r
+
+    # -- conveniences (allocation of outputs only)
+    def decode(self, query, key_cache, value_cache, block_tables, seq_lens, max_seq_len, scale, k_scale=1.0,
+               v_scale=1.0, stream=None) -> torch.Tensor:
+        out = torch.empty_like(query)
+        self.paged_attention_decode(out, query, key_cache, value_cache, block_tables, seq_lens, max_seq_len, scale,
+                                    k_scale, v_scale, stream)
+        return out
+
+    def new_cache(self) -> torch.Tensor:
+        c = self.cfg
+        return torch.empty((c.num_blocks, c.block_size, c.num_kv_heads, c.head_dim), dtype=TORCH_OF[self.kv_dtype],
+                           device=f"cuda:{self.device}")

@@ -1,0 +1,448 @@
+// Host side of the C ABI declared in include/paged_attn.h: argument
+// validation, the split-KV workspace, TMA tensor maps over the caches, and
+// kernel dispatch.  All compute is in decode.cuh / cache_ops.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <string>
+#include <unordered_map>
+
+#include "../../include/paged_attn.h"
+#include "cache_ops.cuh"
+#include "decode.cuh"
+
+#define PA_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+using pa::DecodeCfg;
+using pa::DecodeParams;
+
+using DecodeFn = void (*)(CUtensorMap, CUtensorMap, DecodeParams);
+using MergeFn = void (*)(DecodeParams);
+
+struct KernelSet {
+  const void* decode = nullptr;
+  const void* merge = nullptr;
+  int threads = 0;
+  int smem = 0;
+};
+
+template <class C>
+KernelSet make_set() {
+  KernelSet k;
+  k.decode = reinterpret_cast<const void*>(&pa::paged_decode_kernel<C>);
+  k.merge = reinterpret_cast<const void*>(&pa::paged_decode_merge_kernel<typename C::Q, C::D, C::kBf16>);
+  k.threads = C::THREADS;
+  k.smem = C::SMEM_BYTES;
+  return k;
+}
+
+// Pipeline shape per (head_dim, cache type): consumer warps, ring stages.
+template <int D, typename KV, typename Q>
+struct Tuned;
+template <> struct Tuned<64, __half, __half> { using C = DecodeCfg<64, __half, __half, 4, 8>; };
+template <> struct Tuned<128, __half, __half> { using C = DecodeCfg<128, __half, __half, 4, 8>; };
+template <> struct Tuned<256, __half, __half> { using C = DecodeCfg<256, __half, __half, 4, 4>; };
+template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<64, __nv_bfloat16, __nv_bfloat16, 4, 8>; };
+template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, 4, 8>; };
+template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, 4, 4>; };
+template <> struct Tuned<128, __nv_fp8_e4m3, __half> { using C = DecodeCfg<128, __nv_fp8_e4m3, __half, 4, 8>; };
+template <> struct Tuned<256, __nv_fp8_e4m3, __half> { using C = DecodeCfg<256, __nv_fp8_e4m3, __half, 4, 8>; };
+
+bool select_kernels(int head_dim, int q_dtype, int kv_dtype, KernelSet* ks) {
+#define PA_CASE(D, KVT, QT) *ks = make_set<typename Tuned<D, KVT, QT>::C>(); return true
+  if (kv_dtype == PA_F16 && q_dtype == PA_F16) {
+    if (head_dim == 64) { PA_CASE(64, __half, __half); }
+    if (head_dim == 128) { PA_CASE(128, __half, __half); }
+    if (head_dim == 256) { PA_CASE(256, __half, __half); }
+  }
+  if (kv_dtype == PA_BF16 && q_dtype == PA_BF16) {
+    if (head_dim == 64) { PA_CASE(64, __nv_bfloat16, __nv_bfloat16); }
+    if (head_dim == 128) { PA_CASE(128, __nv_bfloat16, __nv_bfloat16); }
+    if (head_dim == 256) { PA_CASE(256, __nv_bfloat16, __nv_bfloat16); }
+  }
+  if (kv_dtype == PA_FP8_E4M3 && q_dtype == PA_F16) {
+    if (head_dim == 128) { PA_CASE(128, __nv_fp8_e4m3, __half); }
+    if (head_dim == 256) { PA_CASE(256, __nv_fp8_e4m3, __half); }
+  }
+#undef PA_CASE
+  return false;
+}
+
+int elem_bytes(int dt) { return dt == PA_FP8_E4M3 ? 1 : 2; }
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+}  // namespace
+
+struct pa_ctx {
+  pa_config cfg{};
+  int device = 0;
+  int num_sms = 0;
+  int ctas_per_sm = 1;
+  int max_parts = 0;            // workspace partitions per (seq, head)
+  int min_partition_tokens = 0; // smallest partition the workspace allows
+  int partition_tokens = 0;     // current setting (PA_PARTITION_* or > 0)
+  float* part_o = nullptr;
+  float* part_ml = nullptr;
+  int* err = nullptr;
+  int* err_host = nullptr;      // pinned
+  int last_bits = 0;
+  KernelSet ks;
+  std::unordered_map<const void*, CUtensorMap> maps;
+  std::string msg;
+};
+
+namespace {
+
+int fail(pa_ctx* ctx, int status, const char* what) {
+  if (ctx) ctx->msg = what;
+  return status;
+}
+
+int cuda_fail(pa_ctx* ctx, cudaError_t e, const char* where) {
+  if (ctx) ctx->msg = std::string(where) + ": " + cudaGetErrorString(e);
+  return PA_ERR_CUDA;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// 2-D view of a cache as [num_blocks * block_size rows, num_kv_heads * head_dim
+// elements]; box = one 128-byte-wide, block_size-tall sub-tile, 128-byte swizzle.
+int tensor_map(pa_ctx* ctx, const void* base, CUtensorMap* out) {
+  auto it = ctx->maps.find(base);
+  if (it != ctx->maps.end()) {
+    *out = it->second;
+    return PA_OK;
+  }
+  auto enc = encode_fn();
+  if (!enc) return fail(ctx, PA_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  const pa_config& c = ctx->cfg;
+  const int eb = elem_bytes(c.kv_dtype);
+  CUtensorMap m;
+  cuuint64_t dims[2] = {(cuuint64_t)c.num_kv_heads * c.head_dim, (cuuint64_t)c.num_blocks * c.block_size};
+  cuuint64_t strides[1] = {(cuuint64_t)c.num_kv_heads * c.head_dim * eb};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / eb), (cuuint32_t)c.block_size};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&m, eb == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    char buf[96];
+    snprintf(buf, sizeof buf, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return fail(ctx, PA_ERR_CUDA, buf);
+  }
+  if (ctx->maps.size() >= 512) ctx->maps.clear();
+  ctx->maps.emplace(base, m);
+  *out = m;
+  return PA_OK;
+}
+
+int choose_partition(const pa_ctx* ctx, int num_seqs, int max_seq_len) {
+  const pa_config& c = ctx->cfg;
+  int pt = ctx->partition_tokens;
+  if (pt == PA_PARTITION_AUTO) {
+    const int group = c.num_heads / c.num_kv_heads;
+    const long long units = (long long)num_seqs * c.num_kv_heads * ((group + pa::kNH - 1) / pa::kNH);
+    const long long slots = (long long)ctx->num_sms * ctx->ctas_per_sm;
+    // Split only when whole sequences would not give every SM several CTAs.
+    pt = (units >= 4 * slots || max_seq_len <= ctx->min_partition_tokens) ? PA_PARTITION_NONE
+                                                                         : ctx->min_partition_tokens;
+  }
+  return pt;
+}
+
+}  // namespace
+
+PA_API const char* paged_attn_status_string(int status) {
+  switch (status) {
+    case PA_OK: return "ok";
+    case PA_ERR_INVALID_ARG: return "invalid argument";
+    case PA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case PA_ERR_CUDA: return "CUDA error";
+    case PA_ERR_DEVICE_CHECK: return "device-side check fired";
+    case PA_ERR_NO_MEMORY: return "out of device memory";
+    default: return "unknown status";
+  }
+}
+
+PA_API const char* paged_attn_last_error(const pa_ctx* ctx) { return ctx ? ctx->msg.c_str() : ""; }
+
+PA_API int paged_attn_last_check_bits(const pa_ctx* ctx) { return ctx ? ctx->last_bits : 0; }
+
+PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
+  if (!out) return PA_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (!cfg) return PA_ERR_INVALID_ARG;
+  const pa_config c = *cfg;
+  if (c.num_heads <= 0 || c.num_kv_heads <= 0 || c.num_heads % c.num_kv_heads != 0 || c.num_blocks <= 0 ||
+      c.max_num_seqs <= 0 || c.max_blocks_per_seq <= 0 || c.flags != 0 || c.device < 0)
+    return PA_ERR_INVALID_ARG;
+  if (c.block_size != pa::kBS) return PA_ERR_UNSUPPORTED;
+  if ((long long)c.num_blocks * c.block_size > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
+  if (c.partition_tokens < PA_PARTITION_AUTO || (c.partition_tokens > 0 && c.partition_tokens % c.block_size))
+    return PA_ERR_INVALID_ARG;
+  if (c.q_dtype < PA_F16 || c.q_dtype > PA_BF16 || c.kv_dtype < PA_F16 || c.kv_dtype > PA_FP8_E4M3)
+    return PA_ERR_INVALID_ARG;
+  KernelSet ks;
+  if (!select_kernels(c.head_dim, c.q_dtype, c.kv_dtype, &ks)) return PA_ERR_UNSUPPORTED;
+  if ((long long)c.num_kv_heads * c.head_dim * elem_bytes(c.kv_dtype) % 16 != 0) return PA_ERR_UNSUPPORTED;
+
+  cudaError_t e = cudaSetDevice(c.device);
+  if (e != cudaSuccess) return PA_ERR_CUDA;
+  pa_ctx* ctx = new pa_ctx();
+  ctx->cfg = c;
+  ctx->device = c.device;
+  ctx->ks = ks;
+  ctx->partition_tokens = c.partition_tokens;
+  ctx->min_partition_tokens = c.partition_tokens > 0 ? c.partition_tokens : 512;
+  const int max_tokens = c.max_blocks_per_seq * c.block_size;
+  ctx->max_parts = (max_tokens + ctx->min_partition_tokens - 1) / ctx->min_partition_tokens;
+  if (ctx->max_parts < 1) ctx->max_parts = 1;
+
+  int st = PA_OK;
+  do {
+    if ((e = cudaDeviceGetAttribute(&ctx->num_sms, cudaDevAttrMultiProcessorCount, c.device)) != cudaSuccess) {
+      st = cuda_fail(ctx, e, "cudaDeviceGetAttribute");
+      break;
+    }
+    if ((e = cudaFuncSetAttribute(ks.decode, cudaFuncAttributeMaxDynamicSharedMemorySize, ks.smem)) != cudaSuccess) {
+      st = cuda_fail(ctx, e, "cudaFuncSetAttribute");
+      break;
+    }
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctx->ctas_per_sm, ks.decode, ks.threads, ks.smem)) !=
+        cudaSuccess) {
+      st = cuda_fail(ctx, e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
+      break;
+    }
+    if (ctx->ctas_per_sm < 1) {
+      st = fail(ctx, PA_ERR_UNSUPPORTED, "decode kernel does not fit on an SM");
+      break;
+    }
+    const size_t rows = (size_t)c.max_num_seqs * c.num_heads * ctx->max_parts;
+    if (cudaMalloc(&ctx->part_o, rows * c.head_dim * sizeof(float)) != cudaSuccess ||
+        cudaMalloc(&ctx->part_ml, rows * 2 * sizeof(float)) != cudaSuccess) {
+      cudaGetLastError();
+      st = PA_ERR_NO_MEMORY;
+      break;
+    }
+    if ((e = cudaMalloc(&ctx->err, sizeof(int))) != cudaSuccess || (e = cudaMemset(ctx->err, 0, sizeof(int))) != cudaSuccess) {
+      st = cuda_fail(ctx, e, "cudaMalloc(check word)");
+      break;
+    }
+    if ((e = cudaMallocHost(&ctx->err_host, sizeof(int))) != cudaSuccess) {
+      st = cuda_fail(ctx, e, "cudaMallocHost");
+      break;
+    }
+  } while (false);
+  if (st != PA_OK) {
+    paged_attn_destroy(ctx);
+    return st;
+  }
+  *out = ctx;
+  return PA_OK;
+}
+
+PA_API int paged_attn_destroy(pa_ctx* ctx) {
+  if (!ctx) return PA_ERR_INVALID_ARG;
+  cudaSetDevice(ctx->device);
+  if (ctx->part_o) cudaFree(ctx->part_o);
+  if (ctx->part_ml) cudaFree(ctx->part_ml);
+  if (ctx->err) cudaFree(ctx->err);
+  if (ctx->err_host) cudaFreeHost(ctx->err_host);
+  delete ctx;
+  return PA_OK;
+}
+
+PA_API int paged_attn_set_partition_tokens(pa_ctx* ctx, int partition_tokens) {
+  if (!ctx) return PA_ERR_INVALID_ARG;
+  if (partition_tokens == PA_PARTITION_NONE || partition_tokens == PA_PARTITION_AUTO) {
+    ctx->partition_tokens = partition_tokens;
+    return PA_OK;
+  }
+  if (partition_tokens < ctx->min_partition_tokens || partition_tokens % ctx->cfg.block_size)
+    return fail(ctx, PA_ERR_INVALID_ARG, "partition_tokens below the workspace minimum or not a block multiple");
+  ctx->partition_tokens = partition_tokens;
+  return PA_OK;
+}
+
+PA_API int paged_attn_partition_tokens(const pa_ctx* ctx, int num_seqs, int max_seq_len) {
+  if (!ctx || num_seqs < 0 || max_seq_len < 0) return PA_ERR_INVALID_ARG;
+  return choose_partition(ctx, num_seqs, max_seq_len);
+}
+
+PA_API int reshape_and_cache(pa_ctx* ctx, const void* key, const void* value, int64_t key_token_stride,
+                             int64_t value_token_stride, void* key_cache, void* value_cache,
+                             const int64_t* slot_mapping, int num_tokens, float k_scale, float v_scale,
+                             void* stream) {
+  if (!ctx) return PA_ERR_INVALID_ARG;
+  const pa_config& c = ctx->cfg;
+  if (num_tokens < 0) return fail(ctx, PA_ERR_INVALID_ARG, "num_tokens < 0");
+  if (num_tokens == 0) return PA_OK;
+  if (!key || !value || !key_cache || !value_cache || !slot_mapping)
+    return fail(ctx, PA_ERR_INVALID_ARG, "null pointer");
+  const int row = c.num_kv_heads * c.head_dim;
+  if (key_token_stride < row || value_token_stride < row || key_token_stride % 8 || value_token_stride % 8)
+    return fail(ctx, PA_ERR_INVALID_ARG, "token strides must be >= num_kv_heads*head_dim and multiples of 8");
+  if (!aligned(key, 16) || !aligned(value, 16) || !aligned(key_cache, 16) || !aligned(value_cache, 16) ||
+      !aligned(slot_mapping, 8))
+    return fail(ctx, PA_ERR_INVALID_ARG, "misaligned pointer");
+  const bool fp8 = c.kv_dtype == PA_FP8_E4M3;
+  if (fp8 && !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
+    return fail(ctx, PA_ERR_INVALID_ARG, "fp8 scales must be finite and > 0");
+  cudaSetDevice(ctx->device);
+  pa::CacheWriteParams p;
+  p.key = key;
+  p.value = value;
+  p.key_stride = key_token_stride;
+  p.value_stride = value_token_stride;
+  p.key_cache = key_cache;
+  p.value_cache = value_cache;
+  p.slot_mapping = reinterpret_cast<const long long*>(slot_mapping);
+  p.num_slots = (long long)c.num_blocks * c.block_size;
+  p.num_tokens = num_tokens;
+  p.row_elems = row;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.err = ctx->err;
+  const long long vecs = (long long)num_tokens * (row / 8);
+  const int threads = 256;
+  long long blocks = (vecs + threads - 1) / threads;
+  const long long cap = (long long)ctx->num_sms * 8;
+  if (blocks > cap) blocks = cap;
+  dim3 grid((unsigned)blocks, 2);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!fp8)
+    pa::reshape_and_cache_copy_kernel<<<grid, threads, 0, s>>>(p);
+  else if (c.q_dtype == PA_BF16)
+    pa::reshape_and_cache_fp8_kernel<true><<<grid, threads, 0, s>>>(p);
+  else
+    pa::reshape_and_cache_fp8_kernel<false><<<grid, threads, 0, s>>>(p);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : cuda_fail(ctx, e, "reshape_and_cache launch");
+}
+
+PA_API int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, const void* key_cache,
+                                  const void* value_cache, const int32_t* block_tables, int bt_stride,
+                                  const int32_t* seq_lens, int num_seqs, int max_seq_len, float scale,
+                                  float k_scale, float v_scale, void* stream) {
+  if (!ctx) return PA_ERR_INVALID_ARG;
+  const pa_config& c = ctx->cfg;
+  if (num_seqs < 0 || num_seqs > c.max_num_seqs) return fail(ctx, PA_ERR_INVALID_ARG, "num_seqs out of range");
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens)
+    return fail(ctx, PA_ERR_INVALID_ARG, "null pointer");
+  if (bt_stride < 1) return fail(ctx, PA_ERR_INVALID_ARG, "bt_stride < 1");
+  if (max_seq_len < 0 || max_seq_len > c.max_blocks_per_seq * c.block_size)
+    return fail(ctx, PA_ERR_INVALID_ARG, "max_seq_len outside [0, max_blocks_per_seq*block_size]");
+  if (!aligned(out, 16) || !aligned(query, 16) || !aligned(key_cache, 16) || !aligned(value_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(seq_lens, 4))
+    return fail(ctx, PA_ERR_INVALID_ARG, "misaligned pointer");
+  if (!std::isfinite(scale)) return fail(ctx, PA_ERR_INVALID_ARG, "scale not finite");
+  const bool fp8 = c.kv_dtype == PA_FP8_E4M3;
+  if (fp8 && !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
+    return fail(ctx, PA_ERR_INVALID_ARG, "fp8 scales must be finite and > 0");
+  cudaSetDevice(ctx->device);
+
+  CUtensorMap mk, mv;
+  int st = tensor_map(ctx, key_cache, &mk);
+  if (st != PA_OK) return st;
+  if ((st = tensor_map(ctx, value_cache, &mv)) != PA_OK) return st;
+
+  const int pt = choose_partition(ctx, num_seqs, max_seq_len);
+  const int max_blocks = (max_seq_len + c.block_size - 1) / c.block_size;
+  const int part_blocks = pt > 0 ? pt / c.block_size : (max_blocks > 0 ? max_blocks : 1);
+  int parts = (max_blocks + part_blocks - 1) / part_blocks;
+  if (parts < 1) parts = 1;
+  if (parts > ctx->max_parts) return fail(ctx, PA_ERR_INVALID_ARG, "too many partitions for the workspace");
+
+  DecodeParams p;
+  p.out = out;
+  p.query = query;
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.part_o = ctx->part_o;
+  p.part_ml = ctx->part_ml;
+  p.err = ctx->err;
+  p.num_seqs = num_seqs;
+  p.bt_stride = bt_stride;
+  p.num_heads = c.num_heads;
+  p.group = c.num_heads / c.num_kv_heads;
+  p.head_splits = (p.group + pa::kNH - 1) / pa::kNH;
+  p.num_blocks = c.num_blocks;
+  p.partition_blocks = part_blocks;
+  p.max_parts = parts;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
+  p.v_scale = fp8 ? v_scale : 1.0f;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  dim3 grid(parts, c.num_kv_heads * p.head_splits, num_seqs);
+  void* args[] = {&mk, &mv, &p};
+  cudaError_t e = cudaLaunchKernel(ctx->ks.decode, grid, dim3(ctx->ks.threads), args, ctx->ks.smem, s);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "decode partition launch");
+  if (parts > 1) {
+    const long long warps = (long long)num_seqs * c.num_heads;
+    void* margs[] = {&p};
+    e = cudaLaunchKernel(ctx->ks.merge, dim3((unsigned)((warps + 3) / 4)), dim3(128), margs, 0, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "decode merge launch");
+  }
+  return PA_OK;
+}
+
+PA_API int paged_attn_get_error(pa_ctx* ctx, void* stream) {
+  if (!ctx) return PA_ERR_INVALID_ARG;
+  cudaSetDevice(ctx->device);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(ctx->err_host, ctx->err, sizeof(int), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ctx->err, 0, sizeof(int), s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "paged_attn_get_error");
+  ctx->last_bits = *ctx->err_host;
+  return ctx->last_bits ? PA_ERR_DEVICE_CHECK : PA_OK;
+}
+
+PA_API int paged_gather_kv(pa_ctx* ctx, void* k_out, void* v_out, const void* key_cache, const void* value_cache,
+                           const int32_t* block_table_row, int seq_len, void* stream) {
+  if (!ctx) return PA_ERR_INVALID_ARG;
+  const pa_config& c = ctx->cfg;
+  if (seq_len < 0 || seq_len > c.max_blocks_per_seq * c.block_size)
+    return fail(ctx, PA_ERR_INVALID_ARG, "seq_len out of range");
+  if (seq_len == 0) return PA_OK;
+  if (!k_out || !v_out || !key_cache || !value_cache || !block_table_row)
+    return fail(ctx, PA_ERR_INVALID_ARG, "null pointer");
+  if (!aligned(k_out, 16) || !aligned(v_out, 16) || !aligned(key_cache, 16) || !aligned(value_cache, 16))
+    return fail(ctx, PA_ERR_INVALID_ARG, "misaligned pointer");
+  cudaSetDevice(ctx->device);
+  pa::GatherParams p;
+  p.k_out = k_out;
+  p.v_out = v_out;
+  p.key_cache = key_cache;
+  p.value_cache = value_cache;
+  p.block_table = block_table_row;
+  p.seq_len = seq_len;
+  p.row_bytes = c.num_kv_heads * c.head_dim * elem_bytes(c.kv_dtype);
+  p.num_blocks = c.num_blocks;
+  p.err = ctx->err;
+  const long long vecs = (long long)seq_len * (p.row_bytes / 16);
+  long long blocks = (vecs + 255) / 256;
+  if (blocks > (long long)ctx->num_sms * 8) blocks = (long long)ctx->num_sms * 8;
+  pa::paged_gather_kernel<<<dim3((unsigned)blocks, 2), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : cuda_fail(ctx, e, "paged_gather_kv launch");
+}

@@ -1,0 +1,343 @@
+"""GPU parity: the CUDA path through the C ABI against the fp64 CPU oracle.
+
+Cache writes and gathers must be bit-exact; attention within max abs error
+2e-3 (fp16 out), 8e-3 (bf16 out), 2e-3 for fp8 caches against the oracle run
+on the dequantised cache."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention, cache_write, fp8_e4m3, paging
+from paged_kv_cache_463_b200 import binding as b
+from paged_kv_cache_463_b200 import workloads as wl
+from tests.helpers import TOL, assert_out_close, compact_sequences, raw
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    from paged_kv_cache_463_b200 import build
+    build.build()
+    torch.cuda.init()
+
+
+def _ctx(spec: wl.WorkloadSpec, num_blocks: int, max_blocks: int, num_seqs=None, partition=b.PA_PARTITION_AUTO):
+    return b.PagedAttention(spec.num_heads, spec.num_kv_heads, spec.head_dim, num_blocks,
+                            block_size=spec.block_size, q_dtype=spec.q_dtype, kv_dtype=spec.kv_dtype,
+                            max_num_seqs=num_seqs or spec.num_seqs, max_blocks_per_seq=max_blocks,
+                            partition_tokens=partition)
+
+
+def _fp8_fill(pa, w):
+    """Quantise the 16-bit source pools into fp8 caches with the GPU cache write
+    (every slot of the pool)."""
+    NB, bs, Hkv, D = w.key_src.shape
+    kc = torch.empty((NB, bs, Hkv, D), dtype=torch.float8_e4m3fn, device=DEV)
+    vc = torch.empty_like(kc)
+    slots = torch.arange(NB * bs, dtype=torch.int64, device=DEV)
+    pa.reshape_and_cache(w.key_src.view(NB * bs, Hkv, D), w.value_src.view(NB * bs, Hkv, D), kc, vc, slots,
+                         w.k_scale, w.v_scale)
+    return kc, vc
+
+
+def _run_step(pa, w, kc, vc, partition=None):
+    """One decode step: append this step's token, then attend."""
+    pa.reshape_and_cache(w.new_key, w.new_value, kc, vc, w.slot_mapping, w.k_scale, w.v_scale)
+    if partition is not None:
+        pa.set_partition_tokens(partition)
+    out = pa.decode(w.query, kc, vc, w.block_tables, w.seq_lens, w.max_seq_len, w.scale, w.k_scale, w.v_scale)
+    assert pa.get_error() == 0
+    return out
+
+
+def _oracle_full(w, kc_host, vc_host):
+    """Oracle step on whole (small) host caches: cache write, then attention."""
+    sp = w.spec
+    kh, vh = kc_host.copy(), vc_host.copy()
+    cache_write.reshape_and_cache(raw(w.new_key), raw(w.new_value), kh, vh, raw(w.slot_mapping),
+                                  src_dtype=sp.q_dtype, cache_dtype=sp.kv_dtype, k_scale=w.k_scale,
+                                  v_scale=w.v_scale)
+    ref = attention.decode_attention(raw(w.query), kh, vh, raw(w.block_tables), raw(w.seq_lens), w.scale,
+                                     q_dtype=sp.q_dtype, kv_dtype=sp.kv_dtype, k_scale=w.k_scale,
+                                     v_scale=w.v_scale)
+    return ref, kh, vh
+
+
+def _oracle_fp8_pool(w):
+    """The oracle's own E4M3 encoding of the 16-bit source pools."""
+    sp = w.spec
+    kh = cache_write.quantize(raw(w.key_src), sp.q_dtype, w.k_scale)
+    vh = cache_write.quantize(raw(w.value_src), sp.q_dtype, w.v_scale)
+    return kh, vh
+
+
+SMALL = {
+    "tiny": {},
+    "llama2-7b-mha": dict(num_seqs=3, pool_blocks=None),
+    "gqa-70b-like": dict(num_seqs=5),
+    "long-context-split-kv": dict(num_seqs=1, seq_len_min=20000, seq_len_max=20000),
+    "shared-prefix-fp8": dict(num_seqs=8, prefix_groups=2, prefix_tokens=256),
+}
+
+
+@pytest.mark.parametrize("name", list(SMALL))
+def test_step_parity_small(name):
+    """Each workload's shape at a size the oracle checks in full: the cache
+    write bit-exact everywhere, every output element within tolerance."""
+    spec = wl.scaled(wl.SPEC_BY_NAME[name], **SMALL[name])
+    w = wl.make_workload(spec, DEV)
+    pa = _ctx(spec, w.num_blocks, w.block_tables.shape[1])
+    if spec.kv_dtype == "fp8_e4m3":
+        kh, vh = _oracle_fp8_pool(w)
+        kc = torch.from_numpy(kh).to(DEV).view(torch.float8_e4m3fn)
+        vc = torch.from_numpy(vh).to(DEV).view(torch.float8_e4m3fn)
+    else:
+        kh, vh = raw(w.key_cache), raw(w.value_cache)
+        kc, vc = w.key_cache, w.value_cache
+    out = _run_step(pa, w, kc, vc)
+    ref, kh2, vh2 = _oracle_full(w, kh, vh)
+    np.testing.assert_array_equal(raw(kc), kh2)
+    np.testing.assert_array_equal(raw(vc), vh2)
+    tol = TOL[spec.kv_dtype] if spec.kv_dtype == "fp8_e4m3" else TOL[spec.q_dtype]
+    assert_out_close(out, ref, tol, spec.q_dtype, name)
+
+
+def _sample_pairs(S, H, rng, nseq=6, nh=4):
+    seqs = sorted(set([0, S - 1] + rng.choice(S, size=min(S, nseq), replace=False).tolist()))
+    heads = sorted(set([0, H - 1] + rng.choice(H, size=min(H, nh), replace=False).tolist()))
+    return seqs, heads
+
+
+@pytest.mark.parametrize("name", [s.name for s in wl.SPECS])
+def test_step_parity_full_size_sampled(name):
+    """Full-size workloads in the bench's launch configuration; the oracle
+    checks sampled (sequence, head) rows, and the cache write is checked
+    bit-exact on every written slot."""
+    spec = wl.SPEC_BY_NAME[name]
+    w = wl.make_workload(spec, DEV)
+    pa = _ctx(spec, w.num_blocks, w.block_tables.shape[1])
+    rng = np.random.default_rng(spec.seed)
+    if spec.kv_dtype == "fp8_e4m3":
+        kc, vc = _fp8_fill(pa, w)
+    else:
+        kc, vc = w.key_cache, w.value_cache
+    out = _run_step(pa, w, kc, vc)
+    # cache write: every written slot equals the oracle's value of the new token
+    slots = w.slot_mapping.cpu().numpy()
+    bs = spec.block_size
+    kslot = raw(kc.view(-1, spec.num_kv_heads, spec.head_dim)[w.slot_mapping])
+    vslot = raw(vc.view(-1, spec.num_kv_heads, spec.head_dim)[w.slot_mapping])
+    if spec.kv_dtype == "fp8_e4m3":
+        np.testing.assert_array_equal(kslot, cache_write.quantize(raw(w.new_key), spec.q_dtype, w.k_scale))
+        np.testing.assert_array_equal(vslot, cache_write.quantize(raw(w.new_value), spec.q_dtype, w.v_scale))
+    else:
+        np.testing.assert_array_equal(kslot, raw(w.new_key))
+        np.testing.assert_array_equal(vslot, raw(w.new_value))
+    max_tokens = 200_000  # bound the oracle's work: sample fewer sequences when they are long
+    nseq = max(1, min(6, max_tokens // max(1, w.max_seq_len) - 2))
+    seqs, heads = _sample_pairs(spec.num_seqs, spec.num_heads, rng, nseq=nseq)
+    kh, vh, bt, lens, uniq = compact_sequences(kc, vc, w.block_tables, w.seq_lens, seqs)
+    if spec.kv_dtype == "fp8_e4m3":
+        # the GPU-quantised blocks must equal the oracle's own encoding; the
+        # oracle then reads its own codes
+        idx = uniq.to(DEV)
+        ks = raw(w.key_src.index_select(0, idx))
+        vs = raw(w.value_src.index_select(0, idx))
+        okh = cache_write.quantize(ks, spec.q_dtype, w.k_scale)
+        ovh = cache_write.quantize(vs, spec.q_dtype, w.v_scale)
+        # the appended token's slot holds the new token: patch the oracle copy
+        rows = {int(x): i for i, x in enumerate(uniq.tolist())}
+        for s in range(spec.num_seqs):
+            blk, off = int(slots[s]) // bs, int(slots[s]) % bs
+            if blk in rows:
+                okh[rows[blk], off] = cache_write.quantize(raw(w.new_key[s]), spec.q_dtype, w.k_scale)
+                ovh[rows[blk], off] = cache_write.quantize(raw(w.new_value[s]), spec.q_dtype, w.v_scale)
+        np.testing.assert_array_equal(kh, okh)
+        np.testing.assert_array_equal(vh, ovh)
+        kh, vh = okh, ovh
+    q = raw(w.query)[seqs]
+    pairs = [(i, h) for i in range(len(seqs)) for h in heads]
+    ref = attention.decode_attention(q, kh, vh, bt, lens, w.scale, q_dtype=spec.q_dtype, kv_dtype=spec.kv_dtype,
+                                     k_scale=w.k_scale, v_scale=w.v_scale, pairs=pairs)
+    got = out[seqs]
+    tol = TOL[spec.kv_dtype] if spec.kv_dtype == "fp8_e4m3" else TOL[spec.q_dtype]
+    assert_out_close(got, ref, tol, spec.q_dtype, name)
+
+
+EDGE_LENS = [1, 15, 16, 17, 511, 512, 513, 1000, 0, 33]
+
+
+@pytest.mark.parametrize("q_dtype,kv_dtype", [("f16", "f16"), ("bf16", "bf16"), ("f16", "fp8_e4m3")])
+@pytest.mark.parametrize("group", [1, 2, 4, 8, 16])
+@pytest.mark.parametrize("head_dim", [64, 128, 256])
+def test_edge_sweep(q_dtype, kv_dtype, group, head_dim):
+    if kv_dtype == "fp8_e4m3" and head_dim == 64:
+        pytest.skip("fp8 caches need 128-byte rows (head_dim >= 128)")
+    Hkv = 2
+    spec = wl.WorkloadSpec("edge", len(EDGE_LENS), Hkv * group, Hkv, head_dim, 16, q_dtype, kv_dtype, 1, 1,
+                           seed=77 + group + head_dim)
+    w = wl.make_workload(spec, DEV, seq_lens=EDGE_LENS)
+    pa = _ctx(spec, w.num_blocks, w.block_tables.shape[1])
+    if kv_dtype == "fp8_e4m3":
+        kh, vh = _oracle_fp8_pool(w)
+        kc = torch.from_numpy(kh).to(DEV).view(torch.float8_e4m3fn)
+        vc = torch.from_numpy(vh).to(DEV).view(torch.float8_e4m3fn)
+    else:
+        kh, vh = raw(w.key_cache), raw(w.value_cache)
+        kc, vc = w.key_cache, w.value_cache
+    ref, kh2, vh2 = _oracle_full(w, kh, vh)
+    tol = TOL[kv_dtype] if kv_dtype == "fp8_e4m3" else TOL[q_dtype]
+    for part in (b.PA_PARTITION_NONE, 512):
+        out = _run_step(pa, w, kc, vc, partition=part)
+        np.testing.assert_array_equal(raw(kc), kh2)
+        assert_out_close(out, ref, tol, q_dtype, f"partition={part}")
+        assert torch.all(out[EDGE_LENS.index(0)] == 0)
+
+
+def test_split_matches_unsplit_and_len1_exact():
+    spec = wl.scaled(wl.SPEC_BY_NAME["gqa-70b-like"], num_seqs=4)
+    w = wl.make_workload(spec, DEV, seq_lens=[1, 4096, 2049, 513])
+    pa = _ctx(spec, w.num_blocks, w.block_tables.shape[1])
+    o_none = _run_step(pa, w, w.key_cache, w.value_cache, partition=b.PA_PARTITION_NONE)
+    o_512 = _run_step(pa, w, w.key_cache, w.value_cache, partition=512)
+    o_1024 = _run_step(pa, w, w.key_cache, w.value_cache, partition=1024)
+    assert (o_none.float() - o_512.float()).abs().max().item() <= TOL["bf16"]
+    assert (o_none.float() - o_1024.float()).abs().max().item() <= TOL["bf16"]
+    # one token: softmax weight exactly 1, output = that value row exactly
+    v0 = w.new_value[0]
+    G = spec.group_size
+    for h in range(spec.num_heads):
+        assert torch.equal(o_512[0, h], v0[h // G]), h
+
+
+def test_garbage_in_unused_slots_and_blocks_is_ignored():
+    spec = wl.scaled(wl.SPEC_BY_NAME["gqa-70b-like"], num_seqs=6, seq_len_min=17, seq_len_max=700)
+    w = wl.make_workload(spec, DEV)
+    pa = _ctx(spec, w.num_blocks, w.block_tables.shape[1])
+    base = _run_step(pa, w, w.key_cache, w.value_cache, partition=512)
+    kc, vc = w.key_cache.clone(), w.value_cache.clone()
+    used = torch.zeros(w.num_blocks, dtype=torch.bool)
+    for s, n in enumerate(w.seq_lens.tolist()):
+        nb = -(-n // 16)
+        row = w.block_tables[s, :nb].cpu().long()
+        used[row] = True
+        tail = n - (nb - 1) * 16
+        if tail < 16:
+            kc[row[-1], tail:] = float("nan")
+            vc[row[-1], tail:] = float("inf")
+    kc[~used.to(DEV)] = float("nan")
+    vc[~used.to(DEV)] = float("nan")
+    out = _run_step(pa, w, kc, vc, partition=512)
+    assert torch.equal(out, base)
+
+
+def test_gather_bit_exact():
+    for name in ("tiny", "gqa-70b-like", "shared-prefix-fp8"):
+        spec = wl.scaled(wl.SPEC_BY_NAME[name], num_seqs=3)
+        if spec.prefix_groups:
+            spec = wl.scaled(spec, prefix_groups=1, prefix_tokens=64)
+        w = wl.make_workload(spec, DEV)
+        pa = _ctx(spec, w.num_blocks, w.block_tables.shape[1])
+        if spec.kv_dtype == "fp8_e4m3":
+            kc, vc = _fp8_fill(pa, w)
+        else:
+            kc, vc = w.key_cache, w.value_cache
+        kh, vh = raw(kc), raw(vc)
+        for s, n in enumerate(w.seq_lens.tolist()):
+            ko = torch.empty((n, spec.num_kv_heads, spec.head_dim), dtype=kc.dtype, device=DEV)
+            vo = torch.empty_like(ko)
+            pa.paged_gather_kv(ko, vo, kc, vc, w.block_tables[s].contiguous(), n)
+            assert pa.get_error() == 0
+            row = raw(w.block_tables[s])
+            np.testing.assert_array_equal(raw(ko), paging.gather_sequence(kh, row, n))
+            np.testing.assert_array_equal(raw(vo), paging.gather_sequence(vh, row, n))
+
+
+@pytest.mark.parametrize("src", ["f16", "bf16"])
+def test_cache_write_16bit_bit_exact_and_untouched(src):
+    spec = wl.WorkloadSpec("w", 1, 8, 4, 128, 16, src, src, 1, 1, seed=5)
+    NB, T = 40, 50
+    pa = _ctx(spec, NB, 4, num_seqs=T)
+    dt = wl.TORCH_DTYPES[src]
+    g = torch.Generator(device=DEV).manual_seed(3)
+    kc = torch.randn((NB, 16, 4, 128), generator=g, device=DEV).to(dt)
+    vc = torch.randn((NB, 16, 4, 128), generator=g, device=DEV).to(dt)
+    key = torch.randn((T, 4, 128), generator=g, device=DEV).to(dt)
+    val = torch.randn((T, 4, 128), generator=g, device=DEV).to(dt)
+    slots = torch.randperm(NB * 16, generator=torch.Generator().manual_seed(1))[:T]
+    slots[::7] = -1
+    kh, vh = raw(kc), raw(vc)
+    pa.reshape_and_cache(key, val, kc, vc, slots.to(DEV))
+    assert pa.get_error() == 0
+    cache_write.reshape_and_cache(raw(key), raw(val), kh, vh, slots.numpy(), src_dtype=src, cache_dtype=src)
+    np.testing.assert_array_equal(raw(kc), kh)
+    np.testing.assert_array_equal(raw(vc), vh)
+
+
+def test_cache_write_fp8_bit_exact():
+    """E4M3 quantisation of x / scale: random values, exact midpoints between
+    codes (ties to even), values past +-448*scale (saturation), subnormals."""
+    mids = (fp8_e4m3.VALUES[:0x7E] + fp8_e4m3.VALUES[1:0x7F]) / 2
+    vals = np.concatenate([mids, -mids, fp8_e4m3.VALUES[:0x7F], [449, 500, 1e4, -600, 2 ** -10, 3 * 2 ** -11],
+                           np.random.default_rng(0).standard_normal(4096) * 50])
+    T = -(-len(vals) // 128)
+    x = np.zeros(T * 128)
+    x[:len(vals)] = vals
+    key = torch.from_numpy(x.astype(np.float32)).to(torch.float16).view(T, 1, 128).to(DEV)
+    val = (key.float() * 0.5).to(torch.float16)
+    NB = -(-T // 16) + 1
+    pa = b.PagedAttention(2, 1, 128, NB, q_dtype="f16", kv_dtype="fp8_e4m3", max_num_seqs=1, max_blocks_per_seq=1)
+    kc = torch.zeros((NB, 16, 1, 128), dtype=torch.float8_e4m3fn, device=DEV)
+    vc = torch.zeros_like(kc)
+    slots = torch.arange(T, dtype=torch.int64, device=DEV)
+    for sc in (1.0, 0.0123):
+        pa.reshape_and_cache(key, val, kc, vc, slots, sc, sc * 2)
+        assert pa.get_error() == 0
+        ek = cache_write.quantize(raw(key), "f16", sc)
+        ev = cache_write.quantize(raw(val), "f16", sc * 2)
+        np.testing.assert_array_equal(raw(kc).reshape(-1, 1, 128)[:T], ek)
+        np.testing.assert_array_equal(raw(vc).reshape(-1, 1, 128)[:T], ev)
+
+
+def test_device_checks_flag_and_skip():
+    spec = wl.scaled(wl.SPEC_BY_NAME["tiny"], pool_blocks=None)
+    w = wl.make_workload(spec, DEV)
+    pa = _ctx(spec, w.num_blocks, w.block_tables.shape[1])
+    assert pa.get_error() == 0
+    bad = w.block_tables.clone()
+    bad[0, 0] = w.num_blocks + 5
+    pa.decode(w.query, w.key_cache, w.value_cache, bad, w.seq_lens, w.max_seq_len, w.scale)
+    assert pa.get_error() & b.PA_CHECK_BAD_BLOCK
+    assert pa.get_error() == 0  # cleared
+    slots = w.slot_mapping.clone()
+    slots[1] = w.num_blocks * 16 + 3
+    before = w.key_cache.clone()
+    pa.reshape_and_cache(w.new_key, w.new_value, w.key_cache, w.value_cache, slots)
+    assert pa.get_error() & b.PA_CHECK_BAD_SLOT
+    lens = w.seq_lens.clone()
+    lens[2] = w.block_tables.shape[1] * 16 + 40
+    pa.decode(w.query, w.key_cache, w.value_cache, w.block_tables, lens, w.max_seq_len, w.scale)
+    assert pa.get_error() & b.PA_CHECK_SEQ_TOO_LONG
+    del before
+
+
+def test_host_validation_launches_nothing():
+    spec = wl.SPEC_BY_NAME["tiny"]
+    w = wl.make_workload(spec, DEV)
+    pa = _ctx(spec, w.num_blocks, w.block_tables.shape[1])
+    with pytest.raises(b.PagedAttnError) as e:
+        pa.paged_attention_decode(torch.empty_like(w.query), w.query, w.key_cache, w.value_cache, w.block_tables,
+                                  w.seq_lens, 10 ** 6, w.scale)
+    assert e.value.status == b.PA_ERR_INVALID_ARG
+    with pytest.raises(b.PagedAttnError):
+        pa.paged_attention_decode(torch.empty_like(w.query)[:, :, 1:], w.query, w.key_cache, w.value_cache,
+                                  w.block_tables, w.seq_lens, w.max_seq_len, w.scale)  # misaligned out
+    with pytest.raises(b.PagedAttnError):
+        pa.set_partition_tokens(100)
+    assert pa.get_error() == 0
