@@ -46,6 +46,7 @@ extern "C" {
 #define PA_ERR_CUDA (-3)         /* a CUDA runtime call failed; paged_attn_last_error() has the message */
 #define PA_ERR_DEVICE_CHECK (-4) /* a device-side check fired; paged_attn_last_check_bits() says which */
 #define PA_ERR_NO_MEMORY (-5)    /* workspace allocation failed */
+#define PA_ERR_SCRATCH_TOO_SMALL (-6) /* paged_attention_decode_noalloc: partials exceed PA_NOALLOC_SCRATCH_BYTES */
 
 /* ---- device check bits (paged_attn_last_check_bits) */
 #define PA_CHECK_BAD_BLOCK 1    /* block-table entry outside [0, num_blocks): read block 0 instead */
@@ -193,6 +194,42 @@ int paged_attn_partition_tokens(const pa_ctx* ctx, int num_seqs, int max_seq_len
  */
 int paged_gather_kv(pa_ctx* ctx, void* k_out, void* v_out, const void* key_cache, const void* value_cache,
                     const int32_t* block_table_row, int seq_len, void* stream);
+
+/*
+ * Decode attention that allocates nothing (the pages describe no counterpart:
+ * it exists for callers of this library that cannot allocate device memory,
+ * e.g. code running while its stream is being captured into a CUDA graph, or
+ * hosts that own every device allocation through their own pool).
+ *
+ * Same computation, layouts and argument meanings as paged_attention_decode,
+ * but without a context: the cache shape is passed directly (num_heads,
+ * num_kv_heads, head_dim, block_size == 16, num_blocks, q_dtype, kv_dtype), and
+ * the split-KV partials live in one fixed device array built into the library,
+ * PA_NOALLOC_SCRATCH_BYTES (16 MiB) per GPU, held from the library's first use
+ * on that GPU until the process exits.  The caller passes inputs and outputs.
+ *
+ * partition_tokens: 0 = one partition per sequence (needs no partials), else a
+ * multiple of 16.  A split whose partials (num_seqs * num_heads * partitions *
+ * (head_dim + 2) floats, plus 256 bytes) do not fit the array is refused with
+ * PA_ERR_SCRATCH_TOO_SMALL before anything is launched.
+ * check_bits: optional device int that receives PA_CHECK_* bits (or-ed in;
+ * the caller clears it); NULL sends them to a word inside the array.
+ * Runs on the calling thread's current CUDA device.  The first call on each
+ * device looks up the array's device address and raises the decode kernel's
+ * shared-memory limit; make that first call before any stream capture.
+ * Every call on a device shares the array and finds it as the previous call
+ * left it; calls whose kernels may overlap on the GPU (other streams or host
+ * threads on the same device) race on it and must be serialised by the caller.
+ * Never calls cudaMalloc, cudaFree or any allocating routine.
+ * Returns PA_OK, PA_ERR_INVALID_ARG, PA_ERR_UNSUPPORTED,
+ * PA_ERR_SCRATCH_TOO_SMALL or PA_ERR_CUDA.
+ */
+#define PA_NOALLOC_SCRATCH_BYTES (16u * 1024u * 1024u)
+int paged_attention_decode_noalloc(void* out, const void* query, const void* key_cache, const void* value_cache,
+                                   const int32_t* block_tables, int bt_stride, const int32_t* seq_lens, int num_seqs,
+                                   int max_seq_len, int num_heads, int num_kv_heads, int head_dim, int block_size,
+                                   int num_blocks, int q_dtype, int kv_dtype, int partition_tokens, float scale,
+                                   float k_scale, float v_scale, int* check_bits, void* stream);
 
 #ifdef __cplusplus
 }

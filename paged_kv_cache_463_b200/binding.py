@@ -24,6 +24,8 @@ PA_ERR_UNSUPPORTED = -2
 PA_ERR_CUDA = -3
 PA_ERR_DEVICE_CHECK = -4
 PA_ERR_NO_MEMORY = -5
+PA_ERR_SCRATCH_TOO_SMALL = -6
+PA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 PA_CHECK_BAD_BLOCK, PA_CHECK_BAD_SLOT, PA_CHECK_SEQ_TOO_LONG, PA_CHECK_WAIT_TIMEOUT = 1, 2, 4, 8
 PA_PARTITION_NONE, PA_PARTITION_AUTO = 0, -1
 DTYPE_CODES = {"f16": 0, "bf16": 1, "fp8_e4m3": 2}
@@ -67,6 +69,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "paged_attn_set_partition_tokens": (i, [_P, i]),
         "paged_attn_partition_tokens": (i, [_P, i, i]),
         "paged_gather_kv": (i, [_P, _P, _P, _P, _P, _P, i, _P]),
+        "paged_attention_decode_noalloc": (i, [_P, _P, _P, _P, _P, i, _P, i, i, i, i, i, i, i, i, i, i, f, f, f,
+                                               _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -91,6 +95,29 @@ def _stream_ptr(stream) -> int:
 
 def _ptr(t: torch.Tensor | None) -> int | None:
     return None if t is None else t.data_ptr()
+
+
+def paged_attention_decode_noalloc(out, query, key_cache, value_cache, block_tables, seq_lens, max_seq_len: int,
+                                   scale: float, *, num_kv_heads: int, q_dtype: str, kv_dtype: str,
+                                   partition_tokens: int = 0, k_scale=1.0, v_scale=1.0, check_bits=None,
+                                   stream=None, lib_path: str | None = None) -> None:
+    """Decode without a context and without any device allocation by the
+    library: for callers that cannot allocate (e.g. while capturing a CUDA
+    graph, or under a host-owned memory pool).  Split-KV partials go to the
+    library's fixed 16 MiB per-GPU array; calls that overlap on one GPU race on
+    it.  Arguments as in ``PagedAttention.paged_attention_decode``; the cache
+    shape is taken from the tensors."""
+    lib = load_library(lib_path)
+    num_blocks, block_size, hkv, head_dim = key_cache.shape
+    if hkv != num_kv_heads:
+        raise PagedAttnError(PA_ERR_INVALID_ARG, "key_cache head count differs from num_kv_heads")
+    st = lib.paged_attention_decode_noalloc(
+        _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables), block_tables.stride(0),
+        _ptr(seq_lens), query.shape[0], int(max_seq_len), query.shape[1], num_kv_heads, head_dim, block_size,
+        num_blocks, DTYPE_CODES[q_dtype], DTYPE_CODES[kv_dtype], int(partition_tokens), float(scale),
+        float(k_scale), float(v_scale), _ptr(check_bits), _stream_ptr(stream))
+    if st != PA_OK:
+        raise PagedAttnError(st, f"paged_attention_decode_noalloc: {lib.paged_attn_status_string(st).decode()}")
 
 
 class PagedAttention:

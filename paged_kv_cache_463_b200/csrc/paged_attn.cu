@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
 #include <unordered_map>
 
@@ -178,6 +179,7 @@ PA_API const char* paged_attn_status_string(int status) {
     case PA_ERR_CUDA: return "CUDA error";
     case PA_ERR_DEVICE_CHECK: return "device-side check fired";
     case PA_ERR_NO_MEMORY: return "out of device memory";
+    case PA_ERR_SCRATCH_TOO_SMALL: return "split-KV partials exceed the no-alloc scratch (PA_NOALLOC_SCRATCH_BYTES)";
     default: return "unknown status";
   }
 }
@@ -445,4 +447,161 @@ PA_API int paged_gather_kv(pa_ctx* ctx, void* k_out, void* v_out, const void* ke
   pa::paged_gather_kernel<<<dim3((unsigned)blocks, 2), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
   cudaError_t e = cudaGetLastError();
   return e == cudaSuccess ? PA_OK : cuda_fail(ctx, e, "paged_gather_kv launch");
+}
+
+// ---------------------------------------------------------------------------
+// Decode without any allocation.
+//
+// Some callers cannot call cudaMalloc at all: code that runs while a CUDA
+// graph is being captured on its stream, hosts that hand out device memory
+// from their own pool and forbid outside allocations, or callers that must not
+// risk an allocation failure (or an allocator's implicit synchronisation) in
+// the middle of a serving step.  For them this entry point needs no context:
+// the split-KV partials live in one file-scope device array of fixed size,
+// which every GPU that loads this library holds until the process exits.
+//
+// The array is shared by every call on a device and keeps whatever the last
+// call left in it.  Nothing in it has to start at zero: every partial that the
+// merge reads is written earlier in the same call, and the check word is
+// only ever or-ed into.  Two calls whose kernels overlap on the GPU (different
+// streams, or different host threads, on one device) race on the array.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxNoallocDevices = 64;
+constexpr size_t kNoallocHeader = 256;  // bytes reserved at the front (check word)
+
+struct NoallocDevice {
+  bool ready = false;
+  unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+  const void* kernel_ready[16] = {};  // decode kernels whose shared-memory limit was raised here
+};
+NoallocDevice g_noalloc_dev[kMaxNoallocDevices];
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on `dev` (the current device).  The
+// array's name in host code is only a host-side handle; kernels must be given
+// the address cudaGetSymbolAddress returns with the device current.
+int noalloc_setup(int dev, const void* kernel, int smem, unsigned char** scratch) {
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  NoallocDevice& d = g_noalloc_dev[dev];
+  if (!d.ready) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
+    d.scratch = static_cast<unsigned char*>(p);
+    d.ready = true;
+  }
+  int slot = -1;
+  for (int i = 0; i < 16; ++i) {
+    if (d.kernel_ready[i] == kernel) {
+      slot = i;
+      break;
+    }
+    if (d.kernel_ready[i] == nullptr) {
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return PA_ERR_CUDA;
+      d.kernel_ready[i] = kernel;
+      slot = i;
+      break;
+    }
+  }
+  if (slot < 0) return PA_ERR_CUDA;
+  *scratch = d.scratch;
+  return PA_OK;
+}
+
+// Same 2-D view and box as tensor_map(), encoded on the stack each call.
+int encode_cache_map(const void* base, int kv_dtype, int num_kv_heads, int head_dim, int num_blocks, CUtensorMap* m) {
+  auto enc = encode_fn();
+  if (!enc) return PA_ERR_CUDA;
+  const int eb = elem_bytes(kv_dtype);
+  cuuint64_t dims[2] = {(cuuint64_t)num_kv_heads * head_dim, (cuuint64_t)num_blocks * pa::kBS};
+  cuuint64_t strides[1] = {(cuuint64_t)num_kv_heads * head_dim * eb};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / eb), (cuuint32_t)pa::kBS};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, eb == 1 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_UINT16, 2,
+                   const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? PA_OK : PA_ERR_CUDA;
+}
+
+}  // namespace
+
+PA_API int paged_attention_decode_noalloc(void* out, const void* query, const void* key_cache,
+                                          const void* value_cache, const int32_t* block_tables, int bt_stride,
+                                          const int32_t* seq_lens, int num_seqs, int max_seq_len, int num_heads,
+                                          int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                                          int q_dtype, int kv_dtype, int partition_tokens, float scale,
+                                          float k_scale, float v_scale, int* check_bits, void* stream) {
+  if (num_heads <= 0 || num_kv_heads <= 0 || num_heads % num_kv_heads != 0 || num_blocks <= 0 || num_seqs < 0 ||
+      bt_stride < 1 || max_seq_len < 0 || partition_tokens < 0)
+    return PA_ERR_INVALID_ARG;
+  if (block_size != pa::kBS) return PA_ERR_UNSUPPORTED;
+  if (partition_tokens % block_size) return PA_ERR_INVALID_ARG;
+  if ((long long)num_blocks * block_size > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
+  KernelSet ks;
+  if (!select_kernels(head_dim, q_dtype, kv_dtype, &ks)) return PA_ERR_UNSUPPORTED;
+  if ((long long)num_kv_heads * head_dim * elem_bytes(kv_dtype) % 16 != 0) return PA_ERR_UNSUPPORTED;
+  if (num_seqs == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens) return PA_ERR_INVALID_ARG;
+  if (!aligned(out, 16) || !aligned(query, 16) || !aligned(key_cache, 16) || !aligned(value_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(seq_lens, 4) || (check_bits && !aligned(check_bits, 4)))
+    return PA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return PA_ERR_INVALID_ARG;
+  const bool fp8 = kv_dtype == PA_FP8_E4M3;
+  if (fp8 && !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
+    return PA_ERR_INVALID_ARG;
+
+  // Size the split before touching the device: refuse what the array cannot hold.
+  const int max_blocks = (max_seq_len + block_size - 1) / block_size;
+  const int part_blocks = partition_tokens > 0 ? partition_tokens / block_size : (max_blocks > 0 ? max_blocks : 1);
+  int parts = (max_blocks + part_blocks - 1) / part_blocks;
+  if (parts < 1) parts = 1;
+  const size_t rows = (size_t)num_seqs * num_heads * parts;
+  const size_t ml_bytes = (rows * 2 * sizeof(float) + 255) / 256 * 256;
+  const size_t need = kNoallocHeader + (parts > 1 ? ml_bytes + rows * head_dim * sizeof(float) : 0);
+  if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_SCRATCH_TOO_SMALL;
+
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxNoallocDevices) return PA_ERR_CUDA;
+  unsigned char* scratch = nullptr;
+  int st = noalloc_setup(dev, ks.decode, ks.smem, &scratch);
+  if (st != PA_OK) return st;
+
+  CUtensorMap mk, mv;
+  if ((st = encode_cache_map(key_cache, kv_dtype, num_kv_heads, head_dim, num_blocks, &mk)) != PA_OK) return st;
+  if ((st = encode_cache_map(value_cache, kv_dtype, num_kv_heads, head_dim, num_blocks, &mv)) != PA_OK) return st;
+
+  DecodeParams p;
+  p.out = out;
+  p.query = query;
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.part_ml = reinterpret_cast<float*>(scratch + kNoallocHeader);
+  p.part_o = reinterpret_cast<float*>(scratch + kNoallocHeader + ml_bytes);
+  p.err = check_bits ? check_bits : reinterpret_cast<int*>(scratch);
+  p.num_seqs = num_seqs;
+  p.bt_stride = bt_stride;
+  p.num_heads = num_heads;
+  p.group = num_heads / num_kv_heads;
+  p.head_splits = (p.group + pa::kNH - 1) / pa::kNH;
+  p.num_blocks = num_blocks;
+  p.partition_blocks = part_blocks;
+  p.max_parts = parts;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
+  p.v_scale = fp8 ? v_scale : 1.0f;
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  dim3 grid(parts, num_kv_heads * p.head_splits, num_seqs);
+  void* args[] = {&mk, &mv, &p};
+  if (cudaLaunchKernel(ks.decode, grid, dim3(ks.threads), args, ks.smem, s) != cudaSuccess) return PA_ERR_CUDA;
+  if (parts > 1) {
+    const long long warps = (long long)num_seqs * num_heads;
+    void* margs[] = {&p};
+    if (cudaLaunchKernel(ks.merge, dim3((unsigned)((warps + 3) / 4)), dim3(128), margs, 0, s) != cudaSuccess)
+      return PA_ERR_CUDA;
+  }
+  return PA_OK;
 }
