@@ -274,8 +274,7 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream()
     max_len = w.max_seq_len
     chosen_part = pa.partition_tokens(spec.num_seqs, max_len)
-    split = chosen_part > 0 and max_len > chosen_part
-    launches_per_step = 2 + (1 if split else 0)
+    launches_per_step = 2  # cache write + decode (split partitions are merged inside the decode kernel)
 
     def step():
         pa.reshape_and_cache(w.new_key, w.new_value, kc, vc, w.slot_mapping, w.k_scale, w.v_scale, stream)
@@ -364,7 +363,9 @@ def run_ours(args, world, rank, local):
         "config": {"workload": spec.name, "description": spec.description, "num_seqs": S,
                    "num_heads": spec.num_heads, "num_kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim,
                    "block_size": spec.block_size, "kv_dtype": spec.kv_dtype, "q_dtype": spec.q_dtype,
-                   "sum_seq_len": int(w.seq_lens.sum().item()), "partition_tokens": chosen_part,
+                   "sum_seq_len": int(w.seq_lens.sum().item()),
+                   "partition_tokens": "auto (chosen by the decode kernel from the lengths)" if chosen_part < 0
+                   else chosen_part,
                    "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "seq_steps_per_s": seq_steps,
@@ -373,7 +374,7 @@ def run_ours(args, world, rank, local):
         "bytes_per_step": dec_bytes,
         "decode_ms": dec_avg_ms, "cache_write_ms": sum(write_ms) / len(write_ms),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "kernel": "paged_decode_kernel" + (" + merge" if split else ""),
+                     "traffic": traffic, "kernel": "paged_decode_kernel",
                      "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                      if peak_kind == "measured" else "fallback 6.65 TB/s"},
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,

@@ -78,8 +78,10 @@ typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
  *   max_num_seqs            : largest num_seqs a decode call may pass.
  *   max_blocks_per_seq      : largest ceil(max_seq_len / block_size) a call may pass.
  *   partition_tokens        : split-KV partition length (a multiple of block_size),
- *                             PA_PARTITION_NONE, or PA_PARTITION_AUTO (512-token
- *                             partitions when a batch would otherwise leave SMs idle).
+ *                             PA_PARTITION_NONE, or PA_PARTITION_AUTO: the decode
+ *                             kernel picks, from the actual lengths, a power-of-two
+ *                             multiple of 512 tokens (or no split) that keeps every
+ *                             work item a modest fraction of one CTA's share.
  *   device                  : CUDA device ordinal the context and its calls use.
  *   flags                   : reserved, must be 0.
  */
@@ -181,8 +183,10 @@ const char* paged_attn_last_error(const pa_ctx* ctx);
  */
 int paged_attn_set_partition_tokens(pa_ctx* ctx, int partition_tokens);
 
-/* Partition length (tokens) the next decode call with these sizes would use;
- * 0 means one partition per sequence.  Negative status on bad arguments. */
+/* The context's partition setting for decode calls: a length in tokens,
+ * PA_PARTITION_NONE (0), or PA_PARTITION_AUTO (-1, chosen on the device per
+ * call).  num_seqs and max_seq_len are validated only.  PA_ERR_INVALID_ARG on
+ * bad arguments. */
 int paged_attn_partition_tokens(const pa_ctx* ctx, int num_seqs, int max_seq_len);
 
 /*

@@ -9,24 +9,28 @@
 // with the KV head h / (num_heads / num_kv_heads) (grouped-query attention).
 //
 // Kernel design (B200):
-//  * one CTA per (KV partition, KV head [x query-head chunk of 8], sequence);
-//  * warp NC is the producer: it reads the partition's block-table entries
-//    (one per lane, shuffled out), and lane 0 streams each 16-token block's K
-//    and V tiles into an NS-deep shared-memory ring with 2-D TMA tensor loads
-//    (128-byte swizzle, completion counted on an mbarrier, no multicast);
-//  * warps 0..NC-1 consume whole blocks round-robin, each keeping its own
-//    running max / sum / output (online softmax in the log2 domain):
-//      S^T[16 tok x 8 heads] = K[16 x D] . Q^T[D x 8]     (mma.m16n8k16, K via ldmatrix)
-//      P^T = exp2(S^T - m) packed to 16 bits, moved into the B-operand layout
-//            with movmatrix (an 8x8 transpose in registers)
-//      O^T[D x 8] += V^T[D x 16 tok] . P^T[16 x 8]         (V via ldmatrix.trans)
+//  * work item = (sequence, split-KV partition, KV head [x chunk of 8 query
+//    heads]); items are numbered sequence-major, partition, then KV head, and
+//    handed out by an atomic ticket counter, so every CTA keeps pulling work
+//    until none is left (persistent grid: SMs x CTAs per SM);
+//  * a CTA is two warps.  Warp 1 produces: for each item it bulk-copies the
+//    item's query rows into a 2-slot shared-memory queue and streams each
+//    16-token block's K and V tiles with 2-D TMA tensor loads (128-byte
+//    swizzle, mbarrier byte counts, no multicast) into an NS-stage ring,
+//    with a small metadata record per stage (item, valid tokens, first/last);
+//    it runs ahead into the next item while the consumer finishes this one.
+//    Warp 0 consumes, per block:
+//      S^T[16 tok x 8 heads] = K[16 x D] . Q^T[D x 8]   (mma.m16n8k16, K via ldmatrix)
+//      online softmax in the log2 domain (running max m, sum l)
+//      P^T packed to 16 bits and moved into the B-operand layout with movmatrix
+//      O^T[D x 8] += V^T[D x 16 tok] . P^T[16 x 8]       (V via ldmatrix.trans)
 //    fp8 E4M3 tiles are read with 128-bit shared loads and converted in
-//    registers to f16 pairs (exact); the contraction index order is permuted
-//    so that every lane's operands are contiguous bytes;
-//  * the consumer warps merge their (m, l, O) through shared memory; a
-//    sequence that fits one partition writes its output directly, otherwise
-//    (O / l, m, l) go to the workspace and paged_decode_merge_kernel combines
-//    the partitions with the log-sum-exp rule:
+//    registers to f16 pairs (exact); the contraction order is permuted so
+//    that every lane's operands are contiguous bytes;
+//  * at an item's last block the consumer writes the output (one-partition
+//    sequences) or (O / l, m, l) partials; paged_decode_merge_kernel, launched
+//    as a programmatic dependent of this grid, combines split sequences with
+//    the log-sum-exp rule
 //      M = max_p m_p,  w_p = l_p 2^(m_p - M),  out = sum_p w_p o_p / sum_p w_p.
 #pragma once
 
@@ -39,7 +43,10 @@ namespace pa {
 enum : int { kCheckBadBlock = 1, kCheckBadSlot = 2, kCheckSeqTooLong = 4, kCheckWaitTimeout = 8 };
 
 constexpr int kBS = 16;  // tokens per physical block
-constexpr int kNH = 8;   // query heads per CTA (MMA N)
+constexpr int kNH = 8;   // query heads per item (MMA N)
+
+// stage metadata flags (meta.w)
+enum : int { kFirst = 1, kLast = 2, kEnd = 4 };
 
 struct DecodeParams {
   void* out;                    // [S, Hq, D] query dtype
@@ -49,56 +56,92 @@ struct DecodeParams {
   float* part_o;                // [S, Hq, max_parts, D]
   float* part_ml;               // [S, Hq, max_parts, 2]  (m in log2 units, l)
   int* err;                     // device check bits
+  int* counters;                // [0] ticket, [1] finished CTAs (zero between launches),
+                                // [2] partition size (blocks) the decode kernel used
   int num_seqs;
   int bt_stride;
   int num_heads;
   int group;        // num_heads / num_kv_heads
   int head_splits;  // ceil(group / 8)
+  int kv_units;     // num_kv_heads * head_splits
   int num_blocks;   // physical pool size
-  int partition_blocks;
-  int max_parts;    // grid x of the partition kernel
+  int partition_blocks;  // blocks per partition (the minimum when auto_partition)
+  int auto_partition;    // 1: the kernel picks the partition size from the actual lengths
+  int max_parts;    // partitions a sequence may have (workspace extent)
+  int q_slot_bytes; // min(group, 8) * head_dim * 2: one item's query rows
+  int merge_hpc;    // merge kernel: query heads per CTA
+  int merge_slices; // merge kernel: partition slices per head
   float scale_log2;  // softmax scale * log2(e) (* k_scale for fp8)
   float v_scale;     // 1, or the fp8 value scale
 };
 
-// Partitions a sequence of `len` tokens is split into (after the same clamps
-// the partition kernel applies).
+// Clamp a sequence length to what its table row can address.
 __device__ __forceinline__ int clamp_len(int len, const DecodeParams& p) {
   const int cap = p.bt_stride * kBS;
   return len < 0 ? 0 : (len > cap ? cap : len);
 }
-__device__ __forceinline__ int num_partitions(int len, const DecodeParams& p) {
+// Partitions of a (clamped) length with `pb` blocks per partition; the
+// workspace extent caps it.
+__device__ __forceinline__ int num_partitions(int len, int pb, const DecodeParams& p) {
   const int nblk = (len + kBS - 1) / kBS;
-  const int np = (nblk + p.partition_blocks - 1) / p.partition_blocks;
+  const int np = (nblk + pb - 1) / pb;
   return np < p.max_parts ? np : p.max_parts;
 }
 
-template <int D_, typename KV_, typename Q_, int NC_, int NS_>
+// Partition size (blocks) for this launch.  With auto_partition the size is
+// chosen from the actual lengths: a work item (one partition of one KV unit)
+// should not exceed a fraction of one CTA's average share of the work --
+// 0.6 when all lengths are within 10 % (items finish together), 0.3 when they
+// vary (a long straggler would idle the rest) -- taking the largest power-of-
+// two multiple of the minimum that fits, or no split at all if a whole
+// sequence fits.
+__device__ __forceinline__ int choose_partition_blocks(const DecodeParams& p, long long sum_len, int min_len,
+                                                       int max_len, int ctas) {
+  if (!p.auto_partition || max_len <= 0) return p.partition_blocks;
+  const int max_blk = (max_len + kBS - 1) / kBS;
+  const float per_cta = (float)p.kv_units * (float)sum_len / (float)ctas;  // tokens of work per CTA
+  const float budget = (min_len * 10 >= max_len * 9 ? 0.6f : 0.3f) * per_cta;
+  if ((float)max_len <= budget) return max(max_blk, p.partition_blocks);
+  int pb = p.partition_blocks;
+  while ((float)(2 * pb * kBS) <= budget && 2 * pb < max_blk) pb *= 2;
+  return pb;
+}
+
+// Shared-memory layout of a decode CTA (offsets from a 1024-aligned base):
+// ring[NS stages] | query slots[2] | mbarriers | stage metadata | prefix[S+1], lens[S]
+struct DecodeLayout {
+  int ring, q, bar, meta, prefix;
+  __host__ __device__ DecodeLayout(int ns, int stage_bytes, int q_slot_bytes) {
+    ring = 0;
+    q = ns * stage_bytes;
+    bar = q + 2 * q_slot_bytes;
+    meta = (bar + (2 * ns + 4) * 8 + 15) & ~15;
+    prefix = meta + ns * 16;
+  }
+  // bytes of dynamic shared memory for up to `max_seqs` sequences (+ alignment slack)
+  __host__ __device__ size_t bytes(int max_seqs) const { return 1024 + prefix + 8 * (size_t)(max_seqs + 1); }
+};
+
+template <int D_, typename KV_, typename Q_, int NS_>
 struct DecodeCfg {
   static constexpr int D = D_;
   using KV = KV_;  // __half, __nv_bfloat16 or __nv_fp8_e4m3
   using Q = Q_;    // __half or __nv_bfloat16 (also the MMA operand type)
-  static constexpr int NC = NC_;  // consumer warps
-  static constexpr int NS = NS_;  // ring stages (one block each)
+  static constexpr int NS = NS_;  // ring stages (one 16-token block each)
   static constexpr bool kFp8 = sizeof(KV) == 1;
   static constexpr bool kBf16 = std::is_same<Q, __nv_bfloat16>::value;
   static constexpr int ROW_BYTES = D * (int)sizeof(KV);
   static constexpr int SUBTILES = ROW_BYTES / 128;
   static constexpr int TILE_BYTES = kBS * ROW_BYTES;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int THREADS = (NC + 1) * 32;
-  static constexpr int RED_STRIDE = D + 4;
-  static constexpr int RED_BYTES = NC * kNH * RED_STRIDE * 4;
-  static constexpr int RING_BYTES = NS * STAGE_BYTES > RED_BYTES ? NS * STAGE_BYTES : RED_BYTES;
-  static constexpr int BAR_BYTES = 2 * NS * 8;
-  static constexpr int ML_BYTES = (NC + 1) * kNH * 2 * 4;
-  static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + ML_BYTES;
+  static constexpr int THREADS = 64;
   static constexpr int NKT = D / 16;
   static constexpr int NDT = D / 16;
   static_assert(ROW_BYTES % 128 == 0, "rows must be whole 128-byte swizzle spans");
   static_assert(!kFp8 || std::is_same<Q, __half>::value, "fp8 caches pair with fp16 queries");
   static_assert(!std::is_same<KV, __half>::value || std::is_same<Q, __half>::value, "f16 cache needs f16 query");
   static_assert(!std::is_same<KV, __nv_bfloat16>::value || kBf16, "bf16 cache needs bf16 query");
+  static DecodeLayout layout(int q_slot_bytes) { return DecodeLayout(NS, STAGE_BYTES, q_slot_bytes); }
 };
 
 // Byte offset of (row, byte-in-row) inside a [16 x ROW_BYTES] tile stored as
@@ -110,391 +153,602 @@ __device__ __forceinline__ uint32_t tile_off(int row, int byte) {
   return (uint32_t)(sub * (kBS * 128) + row * 128 + ((((in >> 4) ^ (row & 7)) << 4) | (in & 15)));
 }
 
-__device__ __forceinline__ uint32_t ld_u32(const void* p) { return *reinterpret_cast<const uint32_t*>(p); }
-
 template <class C>
-__global__ void __launch_bounds__(C::THREADS) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
-                                                                  const __grid_constant__ CUtensorMap tmV,
-                                                                  const DecodeParams p) {
+__global__ void __launch_bounds__(64) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                          const __grid_constant__ CUtensorMap tmV,
+                                                          const DecodeParams p) {
   using Q = typename C::Q;
-  constexpr int D = C::D, NC = C::NC, NS = C::NS;
+  constexpr int D = C::D, NS = C::NS;
   extern __shared__ uint8_t smem_dyn[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
-  uint8_t* ring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::RING_BYTES);
-  uint64_t* empty = full + NS;
-  float* red_ml = reinterpret_cast<float*>(empty + NS);  // [NC + 1][kNH][2]
-
-  const int part = blockIdx.x;
-  const int kvh = blockIdx.y / p.head_splits;
-  const int hsplit = blockIdx.y - kvh * p.head_splits;
-  const int s = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int S = p.num_seqs;
+  // the merge kernel (launched as a programmatic dependent) may be scheduled
+  // now; it waits for this grid's completion before reading anything
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
+  const DecodeLayout L(NS, C::STAGE_BYTES, p.q_slot_bytes);
+  const uint32_t base_u32 = smem_u32(smem);
+  const uint32_t full0 = base_u32 + L.bar, empty0 = full0 + NS * 8, qfull0 = full0 + 2 * NS * 8, qempty0 = qfull0 + 16;
+  int4* meta = reinterpret_cast<int4*>(smem + L.meta);
+  int* prefix = reinterpret_cast<int*>(smem + L.prefix);  // [S + 1]
+  int* lens = prefix + (S + 1);                             // [S], clamped
 
-  const int raw_len = p.seq_lens[s];
-  const int len = clamp_len(raw_len, p);
-  const int nblk = (len + kBS - 1) / kBS;
-  const int nparts = num_partitions(len, p);
-  if (threadIdx.x == 0 && part == 0 && blockIdx.y == 0 &&
-      (raw_len != len || (nblk + p.partition_blocks - 1) / p.partition_blocks > p.max_parts))
-    atomicOr(p.err, kCheckSeqTooLong);
 
-  const int head0 = kvh * p.group + hsplit * kNH;
-  const int nheads = min(kNH, p.group - hsplit * kNH);
-  if (part >= nparts) {
-    if (nparts == 0 && part == 0) {  // empty sequence: zero output rows
-      Q* o = reinterpret_cast<Q*>(p.out) + ((size_t)s * p.num_heads + head0) * D;
-      for (int i = threadIdx.x; i < nheads * D; i += blockDim.x) o[i] = Q(0.0f);
+  // clamped lengths and their statistics -> partition size -> items per
+  // sequence -> exclusive prefix (a zero-length sequence is one item with no
+  // blocks, so that its zero output row gets written)
+  int pb = p.partition_blocks;
+  if (warp == 1) {
+    long long sum_len = 0;
+    int min_len = 0x7fffffff, max_len = 0;
+    bool bad = false;
+    for (int b = 0; b < S; b += 32) {
+      const int s = b + lane;
+      if (s < S) {
+        const int raw = p.seq_lens[s];
+        const int len = clamp_len(raw, p);
+        lens[s] = len;
+        bad |= raw != len;
+        sum_len += len;
+        min_len = min(min_len, len);
+        max_len = max(max_len, len);
+      }
     }
-    return;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      sum_len += __shfl_xor_sync(0xffffffffu, sum_len, off);
+      min_len = min(min_len, __shfl_xor_sync(0xffffffffu, min_len, off));
+      max_len = max(max_len, __shfl_xor_sync(0xffffffffu, max_len, off));
+    }
+    pb = choose_partition_blocks(p, sum_len, min_len, max_len, gridDim.x);
+    if (blockIdx.x == 0 && lane == 0) p.counters[2] = pb;
+    __syncwarp();
+    int carry = 0;
+    for (int b = 0; b < S; b += 32) {
+      const int s = b + lane;
+      int n = 0;
+      if (s < S) {
+        const int len = lens[s];
+        const int nblk = (len + kBS - 1) / kBS;
+        bad |= (nblk + pb - 1) / pb > p.max_parts;
+        n = max(1, num_partitions(len, pb, p));
+      }
+      int x = n;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+      }
+      if (s < S) prefix[s + 1] = carry + x;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) prefix[0] = 0;
+    if (blockIdx.x == 0 && __any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, kCheckSeqTooLong);
   }
-  const int b0 = part * p.partition_blocks;
-  const int nb = min(nblk, b0 + p.partition_blocks) - b0;
-
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(smem_u32(&full[i]), 1);
-      mbar_init(smem_u32(&empty[i]), 1);
-    }
+    for (int i = 0; i < 2 * NS + 4; ++i) mbar_init(full0 + 8 * i, 1);
     fence_mbar_init();
   }
   __syncthreads();
+  const int total = prefix[S] * p.kv_units;
 
-  const uint32_t ring_u32 = smem_u32(ring);
-
-  if (warp == NC) {
-    // ------------------------------------------------------------ producer
+  if (warp == 1) {
+    // ---------------------------------------------------------------- producer
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
-    const int32_t* bt = p.block_tables + (size_t)s * p.bt_stride + b0;
-    int stop = 0;
-    for (int i0 = 0; i0 < nb && !stop; i0 += 32) {
-      int my = 0;
-      if (i0 + lane < nb) {
-        my = __ldg(bt + i0 + lane);
-        if (my < 0 || my >= p.num_blocks) {
+    int stage_i = 0, item_i = 0, stop = 0;
+    // Claim stage `stage_i` (lane 0): wait until the consumer released its last use.
+    auto claim = [&](int& st) -> bool {
+      st = stage_i % NS;
+      if (stage_i >= NS && !mbar_wait(empty0 + 8 * st, ((stage_i / NS) - 1) & 1)) {
+        atomicOr(p.err, kCheckWaitTimeout);
+        return false;
+      }
+      return true;
+    };
+    // Item of ticket t (t < total): sequence, partition, KV unit, block range.
+    struct Item {
+      int s, y, part, np, len, b0, nb;
+    };
+    auto decode = [&](int t) -> Item {
+      Item it;
+      const int idx = t / p.kv_units;
+      it.y = t - idx * p.kv_units;
+      int lo = 0, hi = S - 1;  // last s with prefix[s] <= idx
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (prefix[mid] <= idx) lo = mid; else hi = mid - 1;
+      }
+      it.s = lo;
+      it.part = idx - prefix[lo];
+      it.len = lens[lo];
+      it.np = max(1, num_partitions(it.len, pb, p));
+      const int nblk = (it.len + kBS - 1) / kBS;
+      it.b0 = it.part * pb;
+      it.nb = max(0, min(nblk, it.b0 + pb) - it.b0);
+      return it;
+    };
+    // Lane j's block-table entry of chunk c (blocks 32c + j) of an item; out-of-pool ids are flagged.
+    auto load_chunk = [&](const Item& it, int c) -> int {
+      const int i = 32 * c + lane;
+      int b = 0;
+      if (i < it.nb) {
+        b = __ldg(p.block_tables + (size_t)it.s * p.bt_stride + it.b0 + i);
+        if (b < 0 || b >= p.num_blocks) {
           atomicOr(p.err, kCheckBadBlock);
-          my = 0;
+          b = 0;
         }
       }
-      const int cnt = min(32, nb - i0);
-      for (int j = 0; j < cnt; ++j) {
-        const int phys = __shfl_sync(0xffffffffu, my, j);
-        const int i = i0 + j;
-        const int st = i % NS;
+      return b;
+    };
+    // Software pipeline: the next item's ticket is claimed four blocks before
+    // this item's end (late enough to keep the hand-out dynamic, early enough
+    // to hide the atomic's latency) and its first block-table chunk is loaded
+    // one block later.
+    int t_cur = 0, t_next = 0;
+    if (lane == 0) t_cur = atomicAdd(&p.counters[0], 1);
+    t_cur = __shfl_sync(0xffffffffu, t_cur, 0);
+    Item cur = {}, nxt = {};
+    int chunk = 0, nchunk = 0;
+    if (t_cur < total) {
+      cur = decode(t_cur);
+      chunk = load_chunk(cur, 0);
+    }
+    while (t_cur < total && !stop) {
+      const int kvh = cur.y / p.head_splits;
+      const int hs = cur.y - kvh * p.head_splits;
+      const int head0 = kvh * p.group + hs * kNH;
+      const int nheads = min(kNH, p.group - hs * kNH);
+      const int meta_z = cur.part | (cur.np << 16);
+      bool claimed = false, fetched = false;
+      // claim / prefetch at blocks nb-2 / nb-1 (at once for items shorter than that)
+      auto lookahead = [&](int i) {
+        if (!claimed && i >= cur.nb - 4) {
+          if (lane == 0) t_next = atomicAdd(&p.counters[0], 1);
+          claimed = true;
+        }
+        if (!fetched && i >= cur.nb - 3) {
+          t_next = __shfl_sync(0xffffffffu, t_next, 0);
+          if (t_next < total) {
+            nxt = decode(t_next);
+            nchunk = load_chunk(nxt, 0);
+          }
+          fetched = true;
+        }
+      };
+      if (lane == 0) {  // this item's query rows -> q slot
+        const int qs = item_i & 1;
+        if (item_i >= 2 && !mbar_wait(qempty0 + 8 * qs, ((item_i >> 1) - 1) & 1)) {
+          atomicOr(p.err, kCheckWaitTimeout);
+          stop = 1;
+        } else {
+          const uint32_t bytes = nheads * D * 2;
+          mbar_arrive_expect_tx(qfull0 + 8 * qs, bytes);
+          bulk_load(base_u32 + L.q + qs * p.q_slot_bytes,
+                    reinterpret_cast<const uint8_t*>(p.query) + ((size_t)cur.s * p.num_heads + head0) * D * 2, bytes,
+                    qfull0 + 8 * qs);
+        }
+      }
+      stop = __shfl_sync(0xffffffffu, stop, 0);
+      if (stop) break;
+      ++item_i;
+      if (cur.nb == 0) {  // empty sequence: a metadata-only stage
         if (lane == 0) {
-          if (i >= NS && !mbar_wait(smem_u32(&empty[st]), ((i / NS) - 1) & 1)) {
-            atomicOr(p.err, kCheckWaitTimeout);
+          int st;
+          if (!claim(st)) {
             stop = 1;
           } else {
-            const uint32_t fb = smem_u32(&full[st]);
-            mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-            const uint32_t kdst = ring_u32 + st * C::STAGE_BYTES;
-            const uint32_t vdst = kdst + C::TILE_BYTES;
-            const int y = phys * kBS;
-#pragma unroll
-            for (int sub = 0; sub < C::SUBTILES; ++sub) {
-              const int x = kvh * D + sub * (128 / (int)sizeof(typename C::KV));
-              tma_load_2d(kdst + sub * kBS * 128, &tmK, x, y, fb);
-              tma_load_2d(vdst + sub * kBS * 128, &tmV, x, y, fb);
-            }
+            meta[st] = make_int4(cur.s, cur.y, meta_z, kFirst | kLast);
+            mbar_arrive(full0 + 8 * st);
           }
         }
+        ++stage_i;
         stop = __shfl_sync(0xffffffffu, stop, 0);
-        if (stop) break;
+      }
+      const int nchunks = (cur.nb + 31) / 32;
+      for (int c = 0; c < nchunks && !stop; ++c) {
+        const int ahead = (c + 1 < nchunks) ? load_chunk(cur, c + 1) : 0;
+        const int cnt = min(32, cur.nb - 32 * c);
+        for (int j = 0; j < cnt; ++j) {
+          const int phys = __shfl_sync(0xffffffffu, chunk, j);
+          const int i = 32 * c + j;
+          if (lane == 0) {
+            int st;
+            if (!claim(st)) {
+              stop = 1;
+            } else {
+              const int valid = min(kBS, cur.len - (cur.b0 + i) * kBS);
+              const int flags = (i == 0 ? kFirst : 0) | (i == cur.nb - 1 ? kLast : 0) | (valid << 8);
+              meta[st] = make_int4(cur.s, cur.y, meta_z, flags);
+              const uint32_t fb = full0 + 8 * st;
+              mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+              const uint32_t kdst = base_u32 + L.ring + st * C::STAGE_BYTES;
+              const uint32_t vdst = kdst + C::TILE_BYTES;
+              const int yy = phys * kBS;
+#pragma unroll
+              for (int sub = 0; sub < C::SUBTILES; ++sub) {
+                const int x = kvh * D + sub * (128 / (int)sizeof(typename C::KV));
+                tma_load_2d(kdst + sub * kBS * 128, &tmK, x, yy, fb);
+                tma_load_2d(vdst + sub * kBS * 128, &tmV, x, yy, fb);
+              }
+            }
+          }
+          ++stage_i;
+          stop = __shfl_sync(0xffffffffu, stop, 0);
+          if (stop) break;
+          lookahead(i);
+        }
+        chunk = ahead;
+      }
+      lookahead(cur.nb);  // items with no blocks, or a loop cut short
+      t_cur = t_next;
+      cur = nxt;
+      chunk = nchunk;
+    }
+    if (!stop && lane == 0) {  // end marker
+      int st;
+      if (claim(st)) {
+        meta[st] = make_int4(0, 0, 0, kEnd);
+        mbar_arrive(full0 + 8 * st);
       }
     }
-    return;
-  }
+  } else {
+    // ---------------------------------------------------------------- consumer
+    const int gid = lane >> 2, c4 = lane & 3;
+    const int mi = lane >> 3, ri = lane & 7;
+    uint32_t qf[C::NKT][2];
+    float o[C::NDT][4];
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    int stage_i = 0, item_i = 0;
+    int cur_s = 0, cur_head0 = 0, cur_nheads = 0, cur_part = 0, cur_np = 1;
 
-  // -------------------------------------------------------------- consumers
-  const int gid = lane >> 2, c4 = lane & 3;
-  const bool head_ok = gid < nheads;
-  const Q* qrow = reinterpret_cast<const Q*>(p.query) + ((size_t)s * p.num_heads + head0 + (head_ok ? gid : 0)) * D;
-
-  // Q^T as MMA B fragments (k = head_dim, n = query head).
-  uint32_t qf[C::NKT][2];
-#pragma unroll
-  for (int j = 0; j < C::NKT; ++j) {
-    if constexpr (!C::kFp8) {
-      qf[j][0] = head_ok ? ld_u32(qrow + 16 * j + 2 * c4) : 0u;
-      qf[j][1] = head_ok ? ld_u32(qrow + 16 * j + 2 * c4 + 8) : 0u;
-    } else {
-      // permuted contraction order: lane column c4 owns dims [D/4*c4, D/4*c4 + D/4),
-      // k-step j uses 4 consecutive ones of them
-      const uint2 v = head_ok ? *reinterpret_cast<const uint2*>(qrow + (D / 4) * c4 + 4 * j) : make_uint2(0u, 0u);
-      qf[j][0] = v.x;
-      qf[j][1] = v.y;
-    }
-  }
-
-  float o[C::NDT][4];
-#pragma unroll
-  for (int t = 0; t < C::NDT; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-
-  const int mi = lane >> 3, ri = lane & 7;
-  bool dead = false;
-
-  for (int i = warp; i < nb; i += NC) {
-    const int st = i % NS;
-    if (!mbar_wait(smem_u32(&full[st]), (i / NS) & 1)) {
-      atomicOr(p.err, kCheckWaitTimeout);
-      dead = true;
-      break;
-    }
-    const int valid = min(kBS, len - (b0 + i) * kBS);
-    const uint32_t kb = ring_u32 + st * C::STAGE_BYTES;
-    const uint32_t vb = kb + C::TILE_BYTES;
-
-    // ---- S^T = K Q^T
-    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-    if constexpr (!C::kFp8) {
-#pragma unroll
-      for (int j = 0; j < C::NKT; ++j) {
-        const int tok = ri + ((mi & 1) << 3);
-        const int dim = 16 * j + ((mi >> 1) << 3);
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(kb + tile_off(tok, dim * 2), a0, a1, a2, a3);
-        if (j & 1)
-          mma_16816<C::kBf16>(sb, a0, a1, a2, a3, qf[j][0], qf[j][1]);
-        else
-          mma_16816<C::kBf16>(sa, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+    while (true) {
+      const int st = stage_i % NS;
+      if (!mbar_wait(full0 + 8 * st, (stage_i / NS) & 1)) {
+        atomicOr(p.err, kCheckWaitTimeout);
+        break;
       }
-    } else {
-      constexpr int LB = D / 4;        // bytes of a K row owned by one lane
-      constexpr int LC = LB / 16;      // 16-byte chunks of it
-      uint4 kr[2][LC];
+      const int4 md = meta[st];
+      if (md.w & kEnd) break;
+      if (md.w & kFirst) {
+        // new item: its query rows, fresh softmax state
+        cur_s = md.x;
+        const int kvh = md.y / p.head_splits;
+        const int hs = md.y - kvh * p.head_splits;
+        cur_head0 = kvh * p.group + hs * kNH;
+        cur_nheads = min(kNH, p.group - hs * kNH);
+        cur_part = md.z & 0xffff;
+        cur_np = md.z >> 16;
+        const int qs = item_i & 1;
+        if (!mbar_wait(qfull0 + 8 * qs, (item_i >> 1) & 1)) {
+          atomicOr(p.err, kCheckWaitTimeout);
+          break;
+        }
+        const uint8_t* qsm = smem + L.q + qs * p.q_slot_bytes + gid * D * 2;
+        const bool ok = gid < cur_nheads;
 #pragma unroll
-      for (int u = 0; u < LC; ++u) {
-        kr[0][u] = lds128(kb + tile_off(gid, LB * c4 + 16 * u));
-        kr[1][u] = lds128(kb + tile_off(gid + 8, LB * c4 + 16 * u));
+        for (int j = 0; j < C::NKT; ++j) {
+          if constexpr (!C::kFp8) {
+            qf[j][0] = ok ? *reinterpret_cast<const uint32_t*>(qsm + 2 * (16 * j + 2 * c4)) : 0u;
+            qf[j][1] = ok ? *reinterpret_cast<const uint32_t*>(qsm + 2 * (16 * j + 2 * c4 + 8)) : 0u;
+          } else {
+            // permuted contraction order: lane column c4 owns dims [D/4*c4, D/4*c4 + D/4)
+            const uint2 v = ok ? *reinterpret_cast<const uint2*>(qsm + 2 * ((D / 4) * c4 + 4 * j)) : make_uint2(0u, 0u);
+            qf[j][0] = v.x;
+            qf[j][1] = v.y;
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(qempty0 + 8 * qs);
+        ++item_i;
+#pragma unroll
+        for (int t = 0; t < C::NDT; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+        m0 = m1 = -INFINITY;
+        l0 = l1 = 0.f;
       }
+      const int valid = (md.w >> 8) & 0xff;
+      if (valid > 0) {
+        const uint32_t kb = base_u32 + L.ring + st * C::STAGE_BYTES;
+        const uint32_t vb = kb + C::TILE_BYTES;
+        // ---- S^T = K Q^T
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+        if constexpr (!C::kFp8) {
 #pragma unroll
-      for (int j = 0; j < C::NKT; ++j) {
-        const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&kr[0][0]);
-        const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&kr[1][0]);
-        const uint32_t x = w0[j], y = w1[j];
-        const uint32_t a0 = e4m3x2_to_f16x2(x), a2 = e4m3x2_to_f16x2(x >> 16);
-        const uint32_t a1 = e4m3x2_to_f16x2(y), a3 = e4m3x2_to_f16x2(y >> 16);
-        if (j & 1)
-          mma_16816<false>(sb, a0, a1, a2, a3, qf[j][0], qf[j][1]);
-        else
-          mma_16816<false>(sa, a0, a1, a2, a3, qf[j][0], qf[j][1]);
-      }
-    }
-
-    // ---- online softmax (log2 domain); rows of S^T are tokens gid, gid+8
-    const float sl = p.scale_log2;
-    const float x0 = gid < valid ? (sa[0] + sb[0]) * sl : -INFINITY;
-    const float x1 = gid < valid ? (sa[1] + sb[1]) * sl : -INFINITY;
-    const float x2 = gid + 8 < valid ? (sa[2] + sb[2]) * sl : -INFINITY;
-    const float x3 = gid + 8 < valid ? (sa[3] + sb[3]) * sl : -INFINITY;
-    float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
+          for (int j = 0; j < C::NKT; ++j) {
+            const int tok = ri + ((mi & 1) << 3);
+            const int dim = 16 * j + ((mi >> 1) << 3);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(kb + tile_off(tok, dim * 2), a0, a1, a2, a3);
+            if (j & 1)
+              mma_16816<C::kBf16>(sb, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+            else
+              mma_16816<C::kBf16>(sa, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+          }
+        } else {
+          constexpr int LB = D / 4;  // bytes of a K row owned by one lane
+          constexpr int LC = LB / 16;
+          uint4 kr[2][LC];
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
-      bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
-    }
-    const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
-    const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
-    m0 = mn0;
-    m1 = mn1;
-    const float p0 = ex2(x0 - mn0), p1 = ex2(x1 - mn1), p2 = ex2(x2 - mn0), p3 = ex2(x3 - mn1);
-    l0 = fmaf(l0, al0, p0 + p2);
-    l1 = fmaf(l1, al1, p1 + p3);
+          for (int u = 0; u < LC; ++u) {
+            kr[0][u] = lds128(kb + tile_off(gid, LB * c4 + 16 * u));
+            kr[1][u] = lds128(kb + tile_off(gid + 8, LB * c4 + 16 * u));
+          }
+          const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&kr[0][0]);
+          const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&kr[1][0]);
 #pragma unroll
-    for (int t = 0; t < C::NDT; ++t) {
-      o[t][0] *= al0;
-      o[t][1] *= al1;
-      o[t][2] *= al0;
-      o[t][3] *= al1;
-    }
-    const uint32_t pb0 = movmatrix_trans(pack2<C::kBf16>(p0, p1));
-    const uint32_t pb1 = movmatrix_trans(pack2<C::kBf16>(p2, p3));
-
-    // ---- O^T += V^T P^T
-    if constexpr (!C::kFp8) {
-      uint32_t mlo = 0xffffffffu, mhi = 0xffffffffu;
-      if (valid < kBS) {  // zero V of tokens past the end (may hold NaN/Inf)
-        mlo = (2 * c4 < valid ? 0x0000ffffu : 0u) | (2 * c4 + 1 < valid ? 0xffff0000u : 0u);
-        mhi = (2 * c4 + 8 < valid ? 0x0000ffffu : 0u) | (2 * c4 + 9 < valid ? 0xffff0000u : 0u);
-      }
+          for (int j = 0; j < C::NKT; ++j) {
+            uint32_t a0, a1, a2, a3;
+            e4m3x4_to_f16x2x2(w0[j], a0, a2);
+            e4m3x4_to_f16x2x2(w1[j], a1, a3);
+            if (j & 1)
+              mma_16816<false>(sb, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+            else
+              mma_16816<false>(sa, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+          }
+        }
+        // ---- online softmax (log2 domain); rows of S^T are tokens gid, gid+8
+        const float sl = p.scale_log2;
+        const float x0 = gid < valid ? (sa[0] + sb[0]) * sl : -INFINITY;
+        const float x1 = gid < valid ? (sa[1] + sb[1]) * sl : -INFINITY;
+        const float x2 = gid + 8 < valid ? (sa[2] + sb[2]) * sl : -INFINITY;
+        const float x3 = gid + 8 < valid ? (sa[3] + sb[3]) * sl : -INFINITY;
+        float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
 #pragma unroll
-      for (int t = 0; t < C::NDT; ++t) {
-        const int tok = ri + ((mi >> 1) << 3);
-        const int dim = 16 * t + ((mi & 1) << 3);
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4_trans(vb + tile_off(tok, dim * 2), a0, a1, a2, a3);
-        mma_16816<C::kBf16>(o[t], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, pb0, pb1);
-      }
-    } else {
-      // lane row gid owns dims [D/8*gid, D/8*gid + D/8) of tokens 2c4, 2c4+1, 2c4+8, 2c4+9;
-      // output tile t holds dims D/8*gid + 2t (MMA row gid) and +1 (row gid+8)
-      constexpr int LB = D / 8;
-      constexpr int LC = LB / 16;
-      uint4 vr[4][LC];
-      const int rows[4] = {2 * c4, 2 * c4 + 1, 2 * c4 + 8, 2 * c4 + 9};
+        for (int off = 4; off < 32; off <<= 1) {
+          bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
+          bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
+        }
+        // Lazy rescaling: the reference max only moves (and O, l are
+        // rescaled) when some head's block max exceeds it by more than
+        // 2^kLazy; otherwise weights up to 2^kLazy are accumulated as they are
+        // (exact in fp32, and well inside the 16-bit P range).
+        constexpr float kLazy = 8.f;
+        const bool grow = (bm0 > m0 + kLazy) || (bm1 > m1 + kLazy);
+        if (__any_sync(0xffffffffu, grow)) {
+          const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
+          const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
+          m0 = mn0;
+          m1 = mn1;
+          l0 *= al0;
+          l1 *= al1;
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
+          for (int t = 0; t < C::NDT; ++t) {
+            o[t][0] *= al0;
+            o[t][1] *= al1;
+            o[t][2] *= al0;
+            o[t][3] *= al1;
+          }
+        }
+        const float p0 = ex2(x0 - m0), p1 = ex2(x1 - m1), p2 = ex2(x2 - m0), p3 = ex2(x3 - m1);
+        l0 += p0 + p2;
+        l1 += p1 + p3;
+        const uint32_t pb0 = movmatrix_trans(pack2<C::kBf16>(p0, p1));
+        const uint32_t pb1 = movmatrix_trans(pack2<C::kBf16>(p2, p3));
+        // ---- O^T += V^T P^T
+        if constexpr (!C::kFp8) {
+          if (valid == kBS) {
 #pragma unroll
-        for (int u = 0; u < LC; ++u) {
-          uint4 v = lds128(vb + tile_off(rows[r], LB * gid + 16 * u));
-          if (rows[r] >= valid) v = make_uint4(0u, 0u, 0u, 0u);
-          vr[r][u] = v;
+            for (int t = 0; t < C::NDT; ++t) {
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4_trans(vb + tile_off(ri + ((mi >> 1) << 3), (16 * t + ((mi & 1) << 3)) * 2), a0, a1, a2, a3);
+              mma_16816<C::kBf16>(o[t], a0, a1, a2, a3, pb0, pb1);
+            }
+          } else {  // zero V of tokens past the end (they may hold NaN/Inf)
+            const uint32_t mlo = (2 * c4 < valid ? 0x0000ffffu : 0u) | (2 * c4 + 1 < valid ? 0xffff0000u : 0u);
+            const uint32_t mhi = (2 * c4 + 8 < valid ? 0x0000ffffu : 0u) | (2 * c4 + 9 < valid ? 0xffff0000u : 0u);
+#pragma unroll
+            for (int t = 0; t < C::NDT; ++t) {
+              uint32_t a0, a1, a2, a3;
+              ldsm_x4_trans(vb + tile_off(ri + ((mi >> 1) << 3), (16 * t + ((mi & 1) << 3)) * 2), a0, a1, a2, a3);
+              mma_16816<C::kBf16>(o[t], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, pb0, pb1);
+            }
+          }
+        } else {
+          // lane row gid owns dims [D/8*gid, D/8*gid + D/8) of tokens 2c4, 2c4+1, 2c4+8, 2c4+9;
+          // output tile t holds dims D/8*gid + 2t (MMA row gid) and +1 (row gid+8)
+          constexpr int LB = D / 8;
+          constexpr int LC = LB / 16;
+          uint4 vr[4][LC];
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            const int row = 2 * c4 + (r & 1) + ((r >> 1) << 3);
+#pragma unroll
+            for (int u = 0; u < LC; ++u) vr[r][u] = lds128(vb + tile_off(row, LB * gid + 16 * u));
+          }
+          if (valid < kBS) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+              const int row = 2 * c4 + (r & 1) + ((r >> 1) << 3);
+              if (row >= valid) {
+#pragma unroll
+                for (int u = 0; u < LC; ++u) vr[r][u] = make_uint4(0u, 0u, 0u, 0u);
+              }
+            }
+          }
+          const uint32_t* r0 = reinterpret_cast<const uint32_t*>(&vr[0][0]);
+          const uint32_t* r1 = reinterpret_cast<const uint32_t*>(&vr[1][0]);
+          const uint32_t* r2 = reinterpret_cast<const uint32_t*>(&vr[2][0]);
+          const uint32_t* r3 = reinterpret_cast<const uint32_t*>(&vr[3][0]);
+#pragma unroll
+          for (int w = 0; w < C::NDT / 2; ++w) {
+            uint32_t a0, a1, a2, a3;
+            // tile 2w: bytes 0,1 of word w; tile 2w+1: bytes 2,3
+            e4m3x4_to_f16x2x2(prmt(r0[w], r1[w], 0x5140u), a0, a1);
+            e4m3x4_to_f16x2x2(prmt(r2[w], r3[w], 0x5140u), a2, a3);
+            mma_16816<false>(o[2 * w], a0, a1, a2, a3, pb0, pb1);
+            e4m3x4_to_f16x2x2(prmt(r0[w], r1[w], 0x7362u), a0, a1);
+            e4m3x4_to_f16x2x2(prmt(r2[w], r3[w], 0x7362u), a2, a3);
+            mma_16816<false>(o[2 * w + 1], a0, a1, a2, a3, pb0, pb1);
+          }
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * st);
+      ++stage_i;
+
+      if (md.w & kLast) {
+        // ---- finish the item straight from registers: full l over the 16
+        // token rows; lane (gid, c4) holds heads 2c4, 2c4+1 of 2 dims per tile
+        float L0 = l0, L1 = l1;
 #pragma unroll
-      for (int t = 0; t < C::NDT; ++t) {
-        const int w = t >> 1;
-        const uint32_t sel = (t & 1) ? 0x7362u : 0x5140u;
-        const uint32_t xa = reinterpret_cast<const uint32_t*>(&vr[0][0])[w];
-        const uint32_t ya = reinterpret_cast<const uint32_t*>(&vr[1][0])[w];
-        const uint32_t xb = reinterpret_cast<const uint32_t*>(&vr[2][0])[w];
-        const uint32_t yb = reinterpret_cast<const uint32_t*>(&vr[3][0])[w];
-        const uint32_t lo = prmt(xa, ya, sel), hi = prmt(xb, yb, sel);
-        const uint32_t a0 = e4m3x2_to_f16x2(lo), a1 = e4m3x2_to_f16x2(lo >> 16);
-        const uint32_t a2 = e4m3x2_to_f16x2(hi), a3 = e4m3x2_to_f16x2(hi >> 16);
-        mma_16816<false>(o[t], a0, a1, a2, a3, pb0, pb1);
+        for (int off = 4; off < 32; off <<= 1) {
+          L0 += __shfl_xor_sync(0xffffffffu, L0, off);
+          L1 += __shfl_xor_sync(0xffffffffu, L1, off);
+        }
+        const int h0 = 2 * c4, h1 = 2 * c4 + 1;
+        const float i0 = L0 > 0.f ? p.v_scale / L0 : 0.f;
+        const float i1 = L1 > 0.f ? p.v_scale / L1 : 0.f;
+        const bool ok0 = h0 < cur_nheads, ok1 = h1 < cur_nheads;
+        // output dims of (tile t, MMA row r): 16-bit path 16t + r; fp8 path D/8*gid + 2t (+1 for r >= 8)
+        auto dim = [&](int t, int hi) -> int {
+          if constexpr (!C::kFp8) return 16 * t + gid + 8 * hi;
+          else return (D / 8) * gid + 2 * t + hi;
+        };
+        if (cur_np == 1) {
+          Q* d0 = reinterpret_cast<Q*>(p.out) + ((size_t)cur_s * p.num_heads + cur_head0 + h0) * D;
+          Q* d1 = d0 + D;
+#pragma unroll
+          for (int t = 0; t < C::NDT; ++t) {
+            if (ok0) {
+              d0[dim(t, 0)] = Q(o[t][0] * i0);
+              d0[dim(t, 1)] = Q(o[t][2] * i0);
+            }
+            if (ok1) {
+              d1[dim(t, 0)] = Q(o[t][1] * i1);
+              d1[dim(t, 1)] = Q(o[t][3] * i1);
+            }
+          }
+        } else {
+          const size_t row0 = ((size_t)cur_s * p.num_heads + cur_head0 + h0) * p.max_parts + cur_part;
+          const size_t row1 = row0 + p.max_parts;
+          float* d0 = p.part_o + row0 * D;
+          float* d1 = p.part_o + row1 * D;
+#pragma unroll
+          for (int t = 0; t < C::NDT; ++t) {
+            if constexpr (!C::kFp8) {
+              if (ok0) {
+                d0[dim(t, 0)] = o[t][0] * i0;
+                d0[dim(t, 1)] = o[t][2] * i0;
+              }
+              if (ok1) {
+                d1[dim(t, 0)] = o[t][1] * i1;
+                d1[dim(t, 1)] = o[t][3] * i1;
+              }
+            } else {  // adjacent dims: one 8-byte store per head
+              if (ok0) *reinterpret_cast<float2*>(d0 + dim(t, 0)) = make_float2(o[t][0] * i0, o[t][2] * i0);
+              if (ok1) *reinterpret_cast<float2*>(d1 + dim(t, 0)) = make_float2(o[t][1] * i1, o[t][3] * i1);
+            }
+          }
+          if (gid == 0) {
+            if (ok0) *reinterpret_cast<float2*>(p.part_ml + row0 * 2) = make_float2(m0, L0);
+            if (ok1) *reinterpret_cast<float2*>(p.part_ml + row1 * 2) = make_float2(m1, L1);
+          }
+        }
       }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(smem_u32(&empty[st]));
   }
 
-  // ---------------------------------------------------------------- combine
-  // full l over this warp's tokens (rows gid of all lanes with the same c4)
-#pragma unroll
-  for (int off = 4; off < 32; off <<= 1) {
-    l0 += __shfl_xor_sync(0xffffffffu, l0, off);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, off);
-  }
-  if (dead) {  // a timed-out warp contributes nothing
-    m0 = m1 = -INFINITY;
-    l0 = l1 = 0.f;
-  }
-  if (gid == 0) {
-    red_ml[(warp * kNH + 2 * c4) * 2 + 0] = m0;
-    red_ml[(warp * kNH + 2 * c4) * 2 + 1] = l0;
-    red_ml[(warp * kNH + 2 * c4 + 1) * 2 + 0] = m1;
-    red_ml[(warp * kNH + 2 * c4 + 1) * 2 + 1] = l1;
-  }
-  // every consumer is done reading the ring and its m/l are visible
-  if constexpr (NC > 1) named_bar_sync(1, NC * 32); else __syncwarp();
-
-  float M0 = -INFINITY, M1 = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < NC; ++w) {
-    M0 = fmaxf(M0, red_ml[(w * kNH + 2 * c4) * 2]);
-    M1 = fmaxf(M1, red_ml[(w * kNH + 2 * c4 + 1) * 2]);
-  }
-  const float f0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M0);
-  const float f1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M1);
-  if (warp == 0 && gid == 0) {
-    float L0 = 0.f, L1 = 0.f;
-#pragma unroll
-    for (int w = 0; w < NC; ++w) {
-      const float mw0 = red_ml[(w * kNH + 2 * c4) * 2], lw0 = red_ml[(w * kNH + 2 * c4) * 2 + 1];
-      const float mw1 = red_ml[(w * kNH + 2 * c4 + 1) * 2], lw1 = red_ml[(w * kNH + 2 * c4 + 1) * 2 + 1];
-      if (mw0 != -INFINITY) L0 += lw0 * ex2(mw0 - M0);
-      if (mw1 != -INFINITY) L1 += lw1 * ex2(mw1 - M1);
-    }
-    red_ml[(NC * kNH + 2 * c4) * 2 + 0] = M0;
-    red_ml[(NC * kNH + 2 * c4) * 2 + 1] = L0;
-    red_ml[(NC * kNH + 2 * c4 + 1) * 2 + 0] = M1;
-    red_ml[(NC * kNH + 2 * c4 + 1) * 2 + 1] = L1;
-  }
-  float* red = reinterpret_cast<float*>(ring) + warp * kNH * C::RED_STRIDE;
-  float* r0 = red + (2 * c4) * C::RED_STRIDE;
-  float* r1 = red + (2 * c4 + 1) * C::RED_STRIDE;
-#pragma unroll
-  for (int t = 0; t < C::NDT; ++t) {
-    if constexpr (!C::kFp8) {
-      r0[16 * t + gid] = o[t][0] * f0;
-      r1[16 * t + gid] = o[t][1] * f1;
-      r0[16 * t + gid + 8] = o[t][2] * f0;
-      r1[16 * t + gid + 8] = o[t][3] * f1;
-    } else {
-      const int d = (D / 8) * gid + 2 * t;
-      *reinterpret_cast<float2*>(r0 + d) = make_float2(o[t][0] * f0, o[t][2] * f0);
-      *reinterpret_cast<float2*>(r1 + d) = make_float2(o[t][1] * f1, o[t][3] * f1);
-    }
-  }
-  if constexpr (NC > 1) named_bar_sync(1, NC * 32); else __syncwarp();
-
-  // ---------------------------------------------------------------- output
-  const float* all = reinterpret_cast<const float*>(ring);
-  const int tid = threadIdx.x;
-  for (int idx = tid; idx < nheads * (D / 4); idx += NC * 32) {
-    const int n = idx / (D / 4);
-    const int d = 4 * (idx - n * (D / 4));
-    float4 acc = *reinterpret_cast<const float4*>(all + n * C::RED_STRIDE + d);
-#pragma unroll
-    for (int w = 1; w < NC; ++w) {
-      const float4 v = *reinterpret_cast<const float4*>(all + (w * kNH + n) * C::RED_STRIDE + d);
-      acc.x += v.x;
-      acc.y += v.y;
-      acc.z += v.z;
-      acc.w += v.w;
-    }
-    const float Mn = red_ml[(NC * kNH + n) * 2 + 0];
-    const float Ln = red_ml[(NC * kNH + n) * 2 + 1];
-    const float inv = Ln > 0.f ? p.v_scale / Ln : 0.f;
-    const int h = head0 + n;
-    if (nparts == 1) {
-      Q* dst = reinterpret_cast<Q*>(p.out) + ((size_t)s * p.num_heads + h) * D + d;
-      const uint32_t lo = pack2<C::kBf16>(acc.x * inv, acc.y * inv);
-      const uint32_t hi = pack2<C::kBf16>(acc.z * inv, acc.w * inv);
-      *reinterpret_cast<uint2*>(dst) = make_uint2(lo, hi);
-    } else {
-      const size_t row = ((size_t)s * p.num_heads + h) * p.max_parts + part;
-      *reinterpret_cast<float4*>(p.part_o + row * D + d) =
-          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-      if (d == 0) *reinterpret_cast<float2*>(p.part_ml + row * 2) = make_float2(Mn, Ln);
+  // the last CTA to finish resets the counters for the next launch
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const int prev = atomicAdd(&p.counters[1], 1);
+    if (prev == (int)gridDim.x - 1) {
+      atomicExch(&p.counters[0], 0);
+      atomicExch(&p.counters[1], 0);
+      __threadfence();
     }
   }
 }
 
-// Log-sum-exp merge of the partitions of every (sequence, head) that was
-// split; one warp per (sequence, head).
+// Log-sum-exp merge of split sequences.  A CTA of 256 threads covers
+// `merge_hpc` consecutive query heads of one sequence; its threads are
+// (head, partition slice, 4-dim chunk) triples, `merge_slices` slices taking
+// every merge_slices-th partition.  Warp n first finds head n's largest
+// partition max M and weight sum W; each thread then accumulates
+// l_p 2^(m_p - M) o_p over its partitions with 8 partitions' loads in flight,
+// and the slices are summed in shared memory.  Launched as a programmatic
+// dependent of the decode kernel: it may be scheduled early and waits for the
+// decode grid to finish before reading.
 template <typename Q, int D, bool BF16>
-__global__ void __launch_bounds__(128) paged_decode_merge_kernel(const DecodeParams p) {
-  const int wg = blockIdx.x * 4 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (wg >= p.num_seqs * p.num_heads) return;
-  const int s = wg / p.num_heads, h = wg - s * p.num_heads;
-  const int np = num_partitions(clamp_len(p.seq_lens[s], p), p);
+__global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodeParams p) {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  constexpr int CH = D / 4;  // float4 chunks per head
+  __shared__ float hM[kNH], hInvW[kNH];
+  __shared__ float4 red[256];
+  const int hpc = p.merge_hpc, slices = p.merge_slices;
+  const int hblocks = (p.num_heads + hpc - 1) / hpc;
+  const int s = blockIdx.x / hblocks;
+  const int h0 = (blockIdx.x - s * hblocks) * hpc;
+  const int pb = p.auto_partition ? p.counters[2] : p.partition_blocks;  // as the decode grid used
+  const int np = num_partitions(clamp_len(p.seq_lens[s], p), pb, p);
   if (np <= 1) return;
-  const size_t row0 = ((size_t)s * p.num_heads + h) * p.max_parts;
-  const float* ml = p.part_ml + row0 * 2;
-  const float* po = p.part_o + row0 * D;
-  float M = -INFINITY;
-  for (int q = lane; q < np; q += 32) M = fmaxf(M, ml[2 * q]);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp < hpc && h0 + warp < p.num_heads) {
+    const float* ml = p.part_ml + ((size_t)s * p.num_heads + h0 + warp) * p.max_parts * 2;
+    float M = -INFINITY;
+    for (int q = lane; q < np; q += 32) M = fmaxf(M, ml[2 * q]);
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-  constexpr int PER = D / 32;  // dims per lane
-  float acc[PER];
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    float W = 0.f;
+    for (int q = lane; q < np; q += 32) {
+      const float2 v = *reinterpret_cast<const float2*>(ml + 2 * q);
+      if (v.y > 0.f) W += v.y * ex2(v.x - M);
+    }
 #pragma unroll
-  for (int k = 0; k < PER; ++k) acc[k] = 0.f;
-  float W = 0.f;
-  for (int q = 0; q < np; ++q) {
-    const float2 mlq = *reinterpret_cast<const float2*>(ml + 2 * q);
-    const float w = mlq.y > 0.f ? mlq.y * ex2(mlq.x - M) : 0.f;
-    W += w;
-    const float* src = po + (size_t)q * D + lane * PER;
-#pragma unroll
-    for (int k = 0; k < PER; k += 2) {
-      const float2 v = *reinterpret_cast<const float2*>(src + k);
-      acc[k] = fmaf(w, v.x, acc[k]);
-      acc[k + 1] = fmaf(w, v.y, acc[k + 1]);
+    for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
+    if (lane == 0) {
+      hM[warp] = M;
+      hInvW[warp] = W > 0.f ? 1.f / W : 0.f;
     }
   }
-  const float inv = W > 0.f ? 1.f / W : 0.f;
-  Q* dst = reinterpret_cast<Q*>(p.out) + ((size_t)s * p.num_heads + h) * D + lane * PER;
+  __syncthreads();
+  const int c = threadIdx.x % CH;
+  const int rest = threadIdx.x / CH;
+  const int slice = rest % slices, hl = rest / slices;
+  const int h = h0 + hl;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (hl < hpc && h < p.num_heads) {
+    const size_t row0 = ((size_t)s * p.num_heads + h) * p.max_parts;
+    const float* ml = p.part_ml + row0 * 2;
+    const float* po = p.part_o + row0 * D + 4 * c;
+    const float M = hM[hl];
+    for (int q0 = slice; q0 < np; q0 += 8 * slices) {
+      float2 mlq[8];
+      float4 v[8];
 #pragma unroll
-  for (int k = 0; k < PER; k += 2) *reinterpret_cast<uint32_t*>(dst + k) = pack2<BF16>(acc[k] * inv, acc[k + 1] * inv);
+      for (int u = 0; u < 8; ++u) {
+        const int q = q0 + u * slices;
+        const bool ok = q < np;
+        mlq[u] = ok ? *reinterpret_cast<const float2*>(ml + 2 * q) : make_float2(-INFINITY, 0.f);
+        v[u] = ok ? *reinterpret_cast<const float4*>(po + (size_t)q * D) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float w = mlq[u].y > 0.f ? mlq[u].y * ex2(mlq[u].x - M) : 0.f;
+        acc.x = fmaf(w, v[u].x, acc.x);
+        acc.y = fmaf(w, v[u].y, acc.y);
+        acc.z = fmaf(w, v[u].z, acc.z);
+        acc.w = fmaf(w, v[u].w, acc.w);
+      }
+    }
+  }
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  if (slice == 0 && hl < hpc && h < p.num_heads) {
+    for (int k = 1; k < slices; ++k) {
+      const float4 o = red[threadIdx.x + k * CH];
+      acc.x += o.x;
+      acc.y += o.y;
+      acc.z += o.z;
+      acc.w += o.w;
+    }
+    const float inv = hInvW[hl];
+    Q* dst = reinterpret_cast<Q*>(p.out) + ((size_t)s * p.num_heads + h) * D + 4 * c;
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack2<BF16>(acc.x * inv, acc.y * inv), pack2<BF16>(acc.z * inv, acc.w * inv));
+  }
 }
 
 }  // namespace pa

@@ -12,7 +12,7 @@
 #include <string>
 #include <unordered_map>
 
-#include "../../include/paged_attn.h"
+#include "paged_attn.h"
 #include "cache_ops.cuh"
 #include "decode.cuh"
 
@@ -23,14 +23,14 @@ namespace {
 using pa::DecodeCfg;
 using pa::DecodeParams;
 
-using DecodeFn = void (*)(CUtensorMap, CUtensorMap, DecodeParams);
-using MergeFn = void (*)(DecodeParams);
-
 struct KernelSet {
   const void* decode = nullptr;
   const void* merge = nullptr;
   int threads = 0;
-  int smem = 0;
+  int ns = 0, stage_bytes = 0;  // ring shape (the rest of the layout depends on the call)
+  size_t smem(int q_slot_bytes, int max_seqs) const {
+    return pa::DecodeLayout(ns, stage_bytes, q_slot_bytes).bytes(max_seqs);
+  }
 };
 
 template <class C>
@@ -39,21 +39,96 @@ KernelSet make_set() {
   k.decode = reinterpret_cast<const void*>(&pa::paged_decode_kernel<C>);
   k.merge = reinterpret_cast<const void*>(&pa::paged_decode_merge_kernel<typename C::Q, C::D, C::kBf16>);
   k.threads = C::THREADS;
-  k.smem = C::SMEM_BYTES;
+  k.ns = C::NS;
+  k.stage_bytes = C::STAGE_BYTES;
   return k;
 }
 
-// Pipeline shape per (head_dim, cache type): consumer warps, ring stages.
+// Every kernel of the library asks for the same (maximum shared-memory)
+// L1/shared split, so consecutive launches (cache write -> decode -> merge)
+// never make the SMs switch configuration between kernels.
+cudaError_t pin_carveout(const void* fn) {
+  return cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+}
+
+cudaError_t pin_all_carveouts(const KernelSet& ks) {
+  const void* fns[] = {ks.decode, ks.merge, reinterpret_cast<const void*>(&pa::reshape_and_cache_copy_kernel),
+                       reinterpret_cast<const void*>(&pa::reshape_and_cache_fp8_kernel<true>),
+                       reinterpret_cast<const void*>(&pa::reshape_and_cache_fp8_kernel<false>),
+                       reinterpret_cast<const void*>(&pa::paged_gather_kernel)};
+  for (const void* f : fns) {
+    cudaError_t e = pin_carveout(f);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+// The merge kernel as a programmatic dependent of the decode kernel just
+// launched on `s`: its CTAs may be scheduled while the decode grid drains and
+// wait (griddepcontrol.wait) for the decode grid before reading partials.
+// Merge CTA shape: more partitions -> more partition slices per head, fewer
+// heads per CTA (256 threads = heads x slices x head_dim/4 chunks).
+void merge_shape(int head_dim, int parts, int num_heads, int* hpc, int* slices) {
+  const int ch = head_dim / 4;
+  int sl = 1;
+  while (sl < 8 && sl * 16 <= parts) sl *= 2;  // <= 15 partitions: 1 slice, ... , >= 128: 8
+  while (sl > 1 && ch * sl > 256) sl /= 2;
+  int h = 256 / (ch * sl);
+  if (h > pa::kNH) h = pa::kNH;
+  if (h > num_heads) h = num_heads;
+  if (h < 1) h = 1;
+  *hpc = h;
+  *slices = sl;
+}
+
+cudaError_t launch_merge(const KernelSet& ks, const pa::DecodeParams& p, cudaStream_t s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(p.num_seqs * ((p.num_heads + p.merge_hpc - 1) / p.merge_hpc)));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  pa::DecodeParams pp = p;
+  void* args[] = {&pp};
+  return cudaLaunchKernelExC(&cfg, ks.merge, args);
+}
+
+// query rows one item copies: min(group, 8) heads of head_dim 16-bit values
+int q_slot_bytes(int num_heads, int num_kv_heads, int head_dim) {
+  const int g = num_heads / num_kv_heads;
+  return (g < pa::kNH ? g : pa::kNH) * head_dim * 2;
+}
+
+// Ring depth (16-token blocks in flight per CTA) per (head_dim, cache type).
+#ifndef PA_NS_16B_64
+#define PA_NS_16B_64 8
+#endif
+#ifndef PA_NS_16B_128
+#define PA_NS_16B_128 3
+#endif
+#ifndef PA_NS_16B_256
+#define PA_NS_16B_256 3
+#endif
+#ifndef PA_NS_FP8_128
+#define PA_NS_FP8_128 4
+#endif
+#ifndef PA_NS_FP8_256
+#define PA_NS_FP8_256 4
+#endif
 template <int D, typename KV, typename Q>
 struct Tuned;
-template <> struct Tuned<64, __half, __half> { using C = DecodeCfg<64, __half, __half, 4, 8>; };
-template <> struct Tuned<128, __half, __half> { using C = DecodeCfg<128, __half, __half, 4, 8>; };
-template <> struct Tuned<256, __half, __half> { using C = DecodeCfg<256, __half, __half, 4, 4>; };
-template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<64, __nv_bfloat16, __nv_bfloat16, 4, 8>; };
-template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, 4, 8>; };
-template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, 4, 4>; };
-template <> struct Tuned<128, __nv_fp8_e4m3, __half> { using C = DecodeCfg<128, __nv_fp8_e4m3, __half, 4, 8>; };
-template <> struct Tuned<256, __nv_fp8_e4m3, __half> { using C = DecodeCfg<256, __nv_fp8_e4m3, __half, 4, 8>; };
+template <> struct Tuned<64, __half, __half> { using C = DecodeCfg<64, __half, __half, PA_NS_16B_64>; };
+template <> struct Tuned<128, __half, __half> { using C = DecodeCfg<128, __half, __half, PA_NS_16B_128>; };
+template <> struct Tuned<256, __half, __half> { using C = DecodeCfg<256, __half, __half, PA_NS_16B_256>; };
+template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<64, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_64>; };
+template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128>; };
+template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_256>; };
+template <> struct Tuned<128, __nv_fp8_e4m3, __half> { using C = DecodeCfg<128, __nv_fp8_e4m3, __half, PA_NS_FP8_128>; };
+template <> struct Tuned<256, __nv_fp8_e4m3, __half> { using C = DecodeCfg<256, __nv_fp8_e4m3, __half, PA_NS_FP8_256>; };
 
 bool select_kernels(int head_dim, int q_dtype, int kv_dtype, KernelSet* ks) {
 #define PA_CASE(D, KVT, QT) *ks = make_set<typename Tuned<D, KVT, QT>::C>(); return true
@@ -101,8 +176,9 @@ struct pa_ctx {
   int partition_tokens = 0;     // current setting (PA_PARTITION_* or > 0)
   float* part_o = nullptr;
   float* part_ml = nullptr;
-  int* err = nullptr;
+  int* err = nullptr;           // [0] check word, [1..2] ticket / finished-CTA counters
   int* err_host = nullptr;      // pinned
+  int grid = 0;                 // persistent grid: SMs x resident CTAs
   int last_bits = 0;
   KernelSet ks;
   std::unordered_map<const void*, CUtensorMap> maps;
@@ -155,18 +231,11 @@ int tensor_map(pa_ctx* ctx, const void* base, CUtensorMap* out) {
   return PA_OK;
 }
 
-int choose_partition(const pa_ctx* ctx, int num_seqs, int max_seq_len) {
-  const pa_config& c = ctx->cfg;
-  int pt = ctx->partition_tokens;
-  if (pt == PA_PARTITION_AUTO) {
-    const int group = c.num_heads / c.num_kv_heads;
-    const long long units = (long long)num_seqs * c.num_kv_heads * ((group + pa::kNH - 1) / pa::kNH);
-    const long long slots = (long long)ctx->num_sms * ctx->ctas_per_sm;
-    // Split only when whole sequences would not give every SM several CTAs.
-    pt = (units >= 4 * slots || max_seq_len <= ctx->min_partition_tokens) ? PA_PARTITION_NONE
-                                                                         : ctx->min_partition_tokens;
-  }
-  return pt;
+// Partition length for the host-side sizing of a launch: the configured one,
+// or for PA_PARTITION_AUTO the smallest the device may choose (the decode
+// kernel then picks the actual size from the lengths).
+int min_partition(const pa_ctx* ctx) {
+  return ctx->partition_tokens == PA_PARTITION_AUTO ? ctx->min_partition_tokens : ctx->partition_tokens;
 }
 
 }  // namespace
@@ -224,12 +293,22 @@ PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
       st = cuda_fail(ctx, e, "cudaDeviceGetAttribute");
       break;
     }
-    if ((e = cudaFuncSetAttribute(ks.decode, cudaFuncAttributeMaxDynamicSharedMemorySize, ks.smem)) != cudaSuccess) {
+    int optin = 0;
+    if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, c.device)) != cudaSuccess) {
+      st = cuda_fail(ctx, e, "cudaDeviceGetAttribute");
+      break;
+    }
+    if (ks.smem(q_slot_bytes(c.num_heads, c.num_kv_heads, c.head_dim), c.max_num_seqs) > (size_t)optin) {
+      st = fail(ctx, PA_ERR_UNSUPPORTED, "max_num_seqs too large for the decode kernel's shared memory");
+      break;
+    }
+    if ((e = cudaFuncSetAttribute(ks.decode, cudaFuncAttributeMaxDynamicSharedMemorySize, optin)) != cudaSuccess ||
+        (e = pin_all_carveouts(ks)) != cudaSuccess) {
       st = cuda_fail(ctx, e, "cudaFuncSetAttribute");
       break;
     }
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctx->ctas_per_sm, ks.decode, ks.threads, ks.smem)) !=
-        cudaSuccess) {
+    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctx->ctas_per_sm, ks.decode, ks.threads,
+                                                           ks.smem(q_slot_bytes(c.num_heads, c.num_kv_heads, c.head_dim), c.max_num_seqs))) != cudaSuccess) {
       st = cuda_fail(ctx, e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
       break;
     }
@@ -244,7 +323,10 @@ PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
       st = PA_ERR_NO_MEMORY;
       break;
     }
-    if ((e = cudaMalloc(&ctx->err, sizeof(int))) != cudaSuccess || (e = cudaMemset(ctx->err, 0, sizeof(int))) != cudaSuccess) {
+    ctx->grid = ctx->num_sms * ctx->ctas_per_sm;
+
+    if ((e = cudaMalloc(&ctx->err, 4 * sizeof(int))) != cudaSuccess ||
+        (e = cudaMemset(ctx->err, 0, 4 * sizeof(int))) != cudaSuccess) {
       st = cuda_fail(ctx, e, "cudaMalloc(check word)");
       break;
     }
@@ -286,7 +368,7 @@ PA_API int paged_attn_set_partition_tokens(pa_ctx* ctx, int partition_tokens) {
 
 PA_API int paged_attn_partition_tokens(const pa_ctx* ctx, int num_seqs, int max_seq_len) {
   if (!ctx || num_seqs < 0 || max_seq_len < 0) return PA_ERR_INVALID_ARG;
-  return choose_partition(ctx, num_seqs, max_seq_len);
+  return ctx->partition_tokens;
 }
 
 PA_API int reshape_and_cache(pa_ctx* ctx, const void* key, const void* value, int64_t key_token_stride,
@@ -367,7 +449,7 @@ PA_API int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, con
   if (st != PA_OK) return st;
   if ((st = tensor_map(ctx, value_cache, &mv)) != PA_OK) return st;
 
-  const int pt = choose_partition(ctx, num_seqs, max_seq_len);
+  const int pt = min_partition(ctx);
   const int max_blocks = (max_seq_len + c.block_size - 1) / c.block_size;
   const int part_blocks = pt > 0 ? pt / c.block_size : (max_blocks > 0 ? max_blocks : 1);
   int parts = (max_blocks + part_blocks - 1) / part_blocks;
@@ -382,28 +464,28 @@ PA_API int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, con
   p.part_o = ctx->part_o;
   p.part_ml = ctx->part_ml;
   p.err = ctx->err;
+  p.counters = ctx->err + 1;
   p.num_seqs = num_seqs;
   p.bt_stride = bt_stride;
   p.num_heads = c.num_heads;
   p.group = c.num_heads / c.num_kv_heads;
   p.head_splits = (p.group + pa::kNH - 1) / pa::kNH;
+  p.kv_units = c.num_kv_heads * p.head_splits;
+  p.q_slot_bytes = q_slot_bytes(c.num_heads, c.num_kv_heads, c.head_dim);
   p.num_blocks = c.num_blocks;
   p.partition_blocks = part_blocks;
+  p.auto_partition = (ctx->partition_tokens == PA_PARTITION_AUTO && pt > 0) ? 1 : 0;
   p.max_parts = parts;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
   p.v_scale = fp8 ? v_scale : 1.0f;
 
+  merge_shape(c.head_dim, parts, c.num_heads, &p.merge_hpc, &p.merge_slices);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  dim3 grid(parts, c.num_kv_heads * p.head_splits, num_seqs);
   void* args[] = {&mk, &mv, &p};
-  cudaError_t e = cudaLaunchKernel(ctx->ks.decode, grid, dim3(ctx->ks.threads), args, ctx->ks.smem, s);
-  if (e != cudaSuccess) return cuda_fail(ctx, e, "decode partition launch");
-  if (parts > 1) {
-    const long long warps = (long long)num_seqs * c.num_heads;
-    void* margs[] = {&p};
-    e = cudaLaunchKernel(ctx->ks.merge, dim3((unsigned)((warps + 3) / 4)), dim3(128), margs, 0, s);
-    if (e != cudaSuccess) return cuda_fail(ctx, e, "decode merge launch");
-  }
+  cudaError_t e = cudaLaunchKernel(ctx->ks.decode, dim3(ctx->grid), dim3(ctx->ks.threads), args,
+                                   ctx->ks.smem(q_slot_bytes(c.num_heads, c.num_kv_heads, c.head_dim), c.max_num_seqs), s);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "decode launch");
+  if (parts > 1 && (e = launch_merge(ctx->ks, p, s)) != cudaSuccess) return cuda_fail(ctx, e, "merge launch");
   return PA_OK;
 }
 
@@ -416,6 +498,12 @@ PA_API int paged_attn_get_error(pa_ctx* ctx, void* stream) {
   if (e == cudaSuccess) e = cudaStreamSynchronize(s);
   if (e != cudaSuccess) return cuda_fail(ctx, e, "paged_attn_get_error");
   ctx->last_bits = *ctx->err_host;
+  if (ctx->last_bits & PA_CHECK_WAIT_TIMEOUT) {
+    // a launch that gave up may have left its work counters non-zero
+    if ((e = cudaMemsetAsync(ctx->err + 1, 0, 3 * sizeof(int), s)) != cudaSuccess ||
+        (e = cudaStreamSynchronize(s)) != cudaSuccess)
+      return cuda_fail(ctx, e, "paged_attn_get_error(counter reset)");
+  }
   return ctx->last_bits ? PA_ERR_DEVICE_CHECK : PA_OK;
 }
 
@@ -461,9 +549,10 @@ PA_API int paged_gather_kv(pa_ctx* ctx, void* k_out, void* v_out, const void* ke
 // which every GPU that loads this library holds until the process exits.
 //
 // The array is shared by every call on a device and keeps whatever the last
-// call left in it.  Nothing in it has to start at zero: every partial that the
-// merge reads is written earlier in the same call, and the check word is
-// only ever or-ed into.  Two calls whose kernels overlap on the GPU (different
+// call left in it.  Only the decode kernel's two work-ticket counters must
+// start at zero: the first call on a device clears the whole array, and every
+// launch leaves them at zero again.  Every partial that the merge reads is
+// written earlier in the same call; the check word is only ever or-ed into.  Two calls whose kernels overlap on the GPU (different
 // streams, or different host threads, on one device) race on the array.
 // ---------------------------------------------------------------------------
 namespace {
@@ -476,6 +565,8 @@ constexpr size_t kNoallocHeader = 256;  // bytes reserved at the front (check wo
 struct NoallocDevice {
   bool ready = false;
   unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch on this device
+  int num_sms = 0;
+  int smem_optin = 0;
   const void* kernel_ready[16] = {};  // decode kernels whose shared-memory limit was raised here
 };
 NoallocDevice g_noalloc_dev[kMaxNoallocDevices];
@@ -484,12 +575,19 @@ std::mutex g_noalloc_mu;
 // Device address of the scratch array on `dev` (the current device).  The
 // array's name in host code is only a host-side handle; kernels must be given
 // the address cudaGetSymbolAddress returns with the device current.
-int noalloc_setup(int dev, const void* kernel, int smem, unsigned char** scratch) {
+int noalloc_setup(int dev, const void* kernel, const void* merge, unsigned char** scratch, int* num_sms,
+                  int* smem_optin) {
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   NoallocDevice& d = g_noalloc_dev[dev];
   if (!d.ready) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
+    // the decode kernel's work counters must start at zero (each launch
+    // leaves the ones it used at zero again); clear the whole array once
+    if (cudaMemset(p, 0, PA_NOALLOC_SCRATCH_BYTES) != cudaSuccess) return PA_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+      return PA_ERR_CUDA;
     d.scratch = static_cast<unsigned char*>(p);
     d.ready = true;
   }
@@ -500,7 +598,8 @@ int noalloc_setup(int dev, const void* kernel, int smem, unsigned char** scratch
       break;
     }
     if (d.kernel_ready[i] == nullptr) {
-      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) != cudaSuccess ||
+          pin_carveout(kernel) != cudaSuccess || pin_carveout(merge) != cudaSuccess)
         return PA_ERR_CUDA;
       d.kernel_ready[i] = kernel;
       slot = i;
@@ -509,6 +608,8 @@ int noalloc_setup(int dev, const void* kernel, int smem, unsigned char** scratch
   }
   if (slot < 0) return PA_ERR_CUDA;
   *scratch = d.scratch;
+  *num_sms = d.num_sms;
+  *smem_optin = d.smem_optin;
   return PA_OK;
 }
 
@@ -567,8 +668,15 @@ PA_API int paged_attention_decode_noalloc(void* out, const void* query, const vo
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxNoallocDevices) return PA_ERR_CUDA;
   unsigned char* scratch = nullptr;
-  int st = noalloc_setup(dev, ks.decode, ks.smem, &scratch);
+  int num_sms = 0, smem_optin = 0;
+  int st = noalloc_setup(dev, ks.decode, ks.merge, &scratch, &num_sms, &smem_optin);
   if (st != PA_OK) return st;
+  const size_t smem = ks.smem(q_slot_bytes(num_heads, num_kv_heads, head_dim), num_seqs);
+  if (smem > (size_t)smem_optin) return PA_ERR_UNSUPPORTED;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ks.decode, ks.threads, smem) != cudaSuccess ||
+      per_sm < 1)
+    return PA_ERR_CUDA;
 
   CUtensorMap mk, mv;
   if ((st = encode_cache_map(key_cache, kv_dtype, num_kv_heads, head_dim, num_blocks, &mk)) != PA_OK) return st;
@@ -582,26 +690,26 @@ PA_API int paged_attention_decode_noalloc(void* out, const void* query, const vo
   p.part_ml = reinterpret_cast<float*>(scratch + kNoallocHeader);
   p.part_o = reinterpret_cast<float*>(scratch + kNoallocHeader + ml_bytes);
   p.err = check_bits ? check_bits : reinterpret_cast<int*>(scratch);
+  p.counters = reinterpret_cast<int*>(scratch) + 4;
   p.num_seqs = num_seqs;
   p.bt_stride = bt_stride;
   p.num_heads = num_heads;
   p.group = num_heads / num_kv_heads;
   p.head_splits = (p.group + pa::kNH - 1) / pa::kNH;
+  p.kv_units = num_kv_heads * p.head_splits;
+  p.q_slot_bytes = q_slot_bytes(num_heads, num_kv_heads, head_dim);
   p.num_blocks = num_blocks;
   p.partition_blocks = part_blocks;
+  p.auto_partition = 0;
   p.max_parts = parts;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
   p.v_scale = fp8 ? v_scale : 1.0f;
 
+  merge_shape(head_dim, parts, num_heads, &p.merge_hpc, &p.merge_slices);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  dim3 grid(parts, num_kv_heads * p.head_splits, num_seqs);
   void* args[] = {&mk, &mv, &p};
-  if (cudaLaunchKernel(ks.decode, grid, dim3(ks.threads), args, ks.smem, s) != cudaSuccess) return PA_ERR_CUDA;
-  if (parts > 1) {
-    const long long warps = (long long)num_seqs * num_heads;
-    void* margs[] = {&p};
-    if (cudaLaunchKernel(ks.merge, dim3((unsigned)((warps + 3) / 4)), dim3(128), margs, 0, s) != cudaSuccess)
-      return PA_ERR_CUDA;
-  }
+  if (cudaLaunchKernel(ks.decode, dim3(num_sms * per_sm), dim3(ks.threads), args, smem, s) != cudaSuccess)
+    return PA_ERR_CUDA;
+  if (parts > 1 && launch_merge(ks, p, s) != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
 }
