@@ -273,7 +273,7 @@ def run_ours(args, world, rank, local):
     out = torch.empty_like(w.query)
     stream = torch.cuda.current_stream()
     max_len = w.max_seq_len
-    chosen_part = pa.partition_tokens(spec.num_seqs, max_len)
+    chosen_part = pa.get_partition_tokens()
     launches_per_step = 2  # cache write + decode (split partitions are merged inside the decode kernel)
 
     def step():

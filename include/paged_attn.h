@@ -183,11 +183,11 @@ const char* paged_attn_last_error(const pa_ctx* ctx);
  */
 int paged_attn_set_partition_tokens(pa_ctx* ctx, int partition_tokens);
 
-/* The context's partition setting for decode calls: a length in tokens,
- * PA_PARTITION_NONE (0), or PA_PARTITION_AUTO (-1, chosen on the device per
- * call).  num_seqs and max_seq_len are validated only.  PA_ERR_INVALID_ARG on
- * bad arguments. */
-int paged_attn_partition_tokens(const pa_ctx* ctx, int num_seqs, int max_seq_len);
+/* Read the context's partition setting for decode calls into
+ * *partition_tokens: a length in tokens, PA_PARTITION_NONE (0), or
+ * PA_PARTITION_AUTO (-1, chosen on the device per call from the lengths).
+ * Returns PA_OK, or PA_ERR_INVALID_ARG for a null pointer. */
+int paged_attn_get_partition_tokens(const pa_ctx* ctx, int* partition_tokens);
 
 /*
  * Gather (page "5.KV Cache 管理 & PagedAttention", Q11 read_kv_range): copy

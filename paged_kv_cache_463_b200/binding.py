@@ -67,7 +67,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "paged_attn_status_string": (ctypes.c_char_p, [i]),
         "paged_attn_last_error": (ctypes.c_char_p, [_P]),
         "paged_attn_set_partition_tokens": (i, [_P, i]),
-        "paged_attn_partition_tokens": (i, [_P, i, i]),
+        "paged_attn_get_partition_tokens": (i, [_P, ctypes.POINTER(i)]),
         "paged_gather_kv": (i, [_P, _P, _P, _P, _P, _P, i, _P]),
         "paged_attention_decode_noalloc": (i, [_P, _P, _P, _P, _P, i, _P, i, i, i, i, i, i, i, i, i, i, f, f, f,
                                                _P, _P]),
@@ -189,11 +189,12 @@ class PagedAttention:
     def set_partition_tokens(self, n: int) -> None:
         self._check(self.lib.paged_attn_set_partition_tokens(self.ctx, int(n)), "paged_attn_set_partition_tokens")
 
-    def partition_tokens(self, num_seqs: int, max_seq_len: int) -> int:
-        r = self.lib.paged_attn_partition_tokens(self.ctx, int(num_seqs), int(max_seq_len))
-        if r < 0:
-            self._check(r, "paged_attn_partition_tokens")
-        return r
+    def get_partition_tokens(self) -> int:
+        """The partition setting: tokens, PA_PARTITION_NONE or PA_PARTITION_AUTO."""
+        v = ctypes.c_int(0)
+        self._check(self.lib.paged_attn_get_partition_tokens(self.ctx, ctypes.byref(v)),
+                    "paged_attn_get_partition_tokens")
+        return v.value
 
     # -- conveniences (allocation of outputs only)
     def decode(self, query, key_cache, value_cache, block_tables, seq_lens, max_seq_len, scale, k_scale=1.0,

@@ -122,7 +122,7 @@ struct DecodeLayout {
   __host__ __device__ size_t bytes(int max_seqs) const { return 1024 + prefix + 8 * (size_t)(max_seqs + 1); }
 };
 
-template <int D_, typename KV_, typename Q_, int NS_>
+template <int D_, typename KV_, typename Q_, int NS_, int MIN_CTAS_ = 1>
 struct DecodeCfg {
   static constexpr int D = D_;
   using KV = KV_;  // __half, __nv_bfloat16 or __nv_fp8_e4m3
@@ -135,6 +135,7 @@ struct DecodeCfg {
   static constexpr int TILE_BYTES = kBS * ROW_BYTES;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
   static constexpr int THREADS = 64;
+  static constexpr int MIN_CTAS = MIN_CTAS_;  // register budget hint: CTAs that must fit on one SM
   static constexpr int NKT = D / 16;
   static constexpr int NDT = D / 16;
   static_assert(ROW_BYTES % 128 == 0, "rows must be whole 128-byte swizzle spans");
@@ -154,7 +155,7 @@ __device__ __forceinline__ uint32_t tile_off(int row, int byte) {
 }
 
 template <class C>
-__global__ void __launch_bounds__(64) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                           const __grid_constant__ CUtensorMap tmV,
                                                           const DecodeParams p) {
   using Q = typename C::Q;

@@ -121,14 +121,19 @@ int q_slot_bytes(int num_heads, int num_kv_heads, int head_dim) {
 #endif
 template <int D, typename KV, typename Q>
 struct Tuned;
-template <> struct Tuned<64, __half, __half> { using C = DecodeCfg<64, __half, __half, PA_NS_16B_64>; };
-template <> struct Tuned<128, __half, __half> { using C = DecodeCfg<128, __half, __half, PA_NS_16B_128>; };
-template <> struct Tuned<256, __half, __half> { using C = DecodeCfg<256, __half, __half, PA_NS_16B_256>; };
-template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<64, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_64>; };
-template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128>; };
-template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_256>; };
-template <> struct Tuned<128, __nv_fp8_e4m3, __half> { using C = DecodeCfg<128, __nv_fp8_e4m3, __half, PA_NS_FP8_128>; };
-template <> struct Tuned<256, __nv_fp8_e4m3, __half> { using C = DecodeCfg<256, __nv_fp8_e4m3, __half, PA_NS_FP8_256>; };
+// (head_dim, cache type) -> ring depth, and the CTAs per SM the register
+// budget must allow (matching what shared memory allows).
+#ifndef PA_MIN_CTAS_FP8_128
+#define PA_MIN_CTAS_FP8_128 8
+#endif
+template <> struct Tuned<64, __half, __half> { using C = DecodeCfg<64, __half, __half, PA_NS_16B_64, 8>; };
+template <> struct Tuned<128, __half, __half> { using C = DecodeCfg<128, __half, __half, PA_NS_16B_128, 8>; };
+template <> struct Tuned<256, __half, __half> { using C = DecodeCfg<256, __half, __half, PA_NS_16B_256, 3>; };
+template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<64, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_64, 8>; };
+template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128, 8>; };
+template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_256, 3>; };
+template <> struct Tuned<128, __nv_fp8_e4m3, __half> { using C = DecodeCfg<128, __nv_fp8_e4m3, __half, PA_NS_FP8_128, PA_MIN_CTAS_FP8_128>; };
+template <> struct Tuned<256, __nv_fp8_e4m3, __half> { using C = DecodeCfg<256, __nv_fp8_e4m3, __half, PA_NS_FP8_256, 4>; };
 
 bool select_kernels(int head_dim, int q_dtype, int kv_dtype, KernelSet* ks) {
 #define PA_CASE(D, KVT, QT) *ks = make_set<typename Tuned<D, KVT, QT>::C>(); return true
@@ -366,9 +371,10 @@ PA_API int paged_attn_set_partition_tokens(pa_ctx* ctx, int partition_tokens) {
   return PA_OK;
 }
 
-PA_API int paged_attn_partition_tokens(const pa_ctx* ctx, int num_seqs, int max_seq_len) {
-  if (!ctx || num_seqs < 0 || max_seq_len < 0) return PA_ERR_INVALID_ARG;
-  return ctx->partition_tokens;
+PA_API int paged_attn_get_partition_tokens(const pa_ctx* ctx, int* partition_tokens) {
+  if (!ctx || !partition_tokens) return PA_ERR_INVALID_ARG;
+  *partition_tokens = ctx->partition_tokens;
+  return PA_OK;
 }
 
 PA_API int reshape_and_cache(pa_ctx* ctx, const void* key, const void* value, int64_t key_token_stride,

@@ -327,6 +327,15 @@ def test_device_checks_flag_and_skip():
     del before
 
 
+def test_partition_setting_round_trip():
+    spec = wl.SPEC_BY_NAME["tiny"]
+    pa = _ctx(spec, 64, 8)
+    assert pa.get_partition_tokens() == b.PA_PARTITION_AUTO
+    for v in (b.PA_PARTITION_NONE, 512, 1024, b.PA_PARTITION_AUTO):
+        pa.set_partition_tokens(v)
+        assert pa.get_partition_tokens() == v
+
+
 def test_host_validation_launches_nothing():
     spec = wl.SPEC_BY_NAME["tiny"]
     w = wl.make_workload(spec, DEV)
