@@ -9,10 +9,17 @@
 // with the KV head h / (num_heads / num_kv_heads) (grouped-query attention).
 //
 // Kernel design (B200):
-//  * work item = (sequence, split-KV partition, KV head [x chunk of 8 query
-//    heads]); items are numbered sequence-major, partition, then KV head, and
-//    handed out by an atomic ticket counter, so every CTA keeps pulling work
-//    until none is left (persistent grid: SMs x CTAs per SM);
+//  * persistent grid (SMs x CTAs per SM).  Work is (sequence, KV unit =
+//    KV head [x chunk of 8 query heads], range of 16-token blocks).  Two
+//    ways of handing it out:
+//      - stream-K (the default): CTAs form groups of kv_units, one CTA per
+//        KV unit; the flattened (sequence, block) space is cut into equal
+//        contiguous ranges, one per group, so every CTA has the same work and
+//        the CTAs of a group read the same blocks (all KV heads of a token are
+//        one contiguous row) at about the same time; a sequence cut by a
+//        range boundary becomes several pieces, merged afterwards;
+//      - tickets (an explicit partition length): items (sequence, partition,
+//        KV unit) numbered in that order, handed out by an atomic counter;
 //  * a CTA is two warps.  Warp 1 produces: for each item it bulk-copies the
 //    item's query rows into a 2-slot shared-memory queue and streams each
 //    16-token block's K and V tiles with 2-D TMA tensor loads (128-byte
@@ -57,7 +64,8 @@ struct DecodeParams {
   float* part_ml;               // [S, Hq, max_parts, 2]  (m in log2 units, l)
   int* err;                     // device check bits
   int* counters;                // [0] ticket, [1] finished CTAs (zero between launches),
-                                // [2] partition size (blocks) the decode kernel used
+                                // [2] partition blocks or stream-K blocks per group, [3] 1 if stream-K
+                                // (both: what the last launch used, for the merge kernel)
   int num_seqs;
   int bt_stride;
   int num_heads;
@@ -65,8 +73,11 @@ struct DecodeParams {
   int head_splits;  // ceil(group / 8)
   int kv_units;     // num_kv_heads * head_splits
   int num_blocks;   // physical pool size
-  int partition_blocks;  // blocks per partition (the minimum when auto_partition)
-  int auto_partition;    // 1: the kernel picks the partition size from the actual lengths
+  int max_blocks;        // ceil(max_seq_len / 16) of the call: lengths are clamped to it
+  int partition_blocks;  // ticket mode: blocks per partition
+  int auto_mode;         // 1: the kernel chooses tickets or stream-K (and the partition) from the lengths
+  int min_piece_blocks;  // stream-K mode: shortest range a CTA group is given
+  int* seq_prefix;       // stream-K mode: [S + 1] block offsets of the sequences, for the merge
   int max_parts;    // partitions a sequence may have (workspace extent)
   int q_slot_bytes; // min(group, 8) * head_dim * 2: one item's query rows
   int merge_hpc;    // merge kernel: query heads per CTA
@@ -75,9 +86,10 @@ struct DecodeParams {
   float v_scale;     // 1, or the fp8 value scale
 };
 
-// Clamp a sequence length to what its table row can address.
+// Clamp a sequence length to what its table row can address and to the
+// call's max_seq_len bound (which sizes the partial workspace).
 __device__ __forceinline__ int clamp_len(int len, const DecodeParams& p) {
-  const int cap = p.bt_stride * kBS;
+  const int cap = min(p.bt_stride, p.max_blocks) * kBS;
   return len < 0 ? 0 : (len > cap ? cap : len);
 }
 // Partitions of a (clamped) length with `pb` blocks per partition; the
@@ -88,23 +100,32 @@ __device__ __forceinline__ int num_partitions(int len, int pb, const DecodeParam
   return np < p.max_parts ? np : p.max_parts;
 }
 
-// Partition size (blocks) for this launch.  With auto_partition the size is
-// chosen from the actual lengths: a work item (one partition of one KV unit)
-// should not exceed a fraction of one CTA's average share of the work --
-// 0.6 when all lengths are within 10 % (items finish together), 0.3 when they
-// vary (a long straggler would idle the rest) -- taking the largest power-of-
-// two multiple of the minimum that fits, or no split at all if a whole
-// sequence fits.
-__device__ __forceinline__ int choose_partition_blocks(const DecodeParams& p, long long sum_len, int min_len,
-                                                       int max_len, int ctas) {
-  if (!p.auto_partition || max_len <= 0) return p.partition_blocks;
+// Partition size (blocks) for near-uniform lengths in auto mode: the largest
+// power-of-two multiple of the minimum such that one work item stays under
+// 0.6 of one CTA's average share of the work (items then finish together), or
+// no split at all if a whole sequence fits.
+__device__ __forceinline__ int uniform_partition_blocks(const DecodeParams& p, long long sum_len, int max_len,
+                                                        int ctas) {
   const int max_blk = (max_len + kBS - 1) / kBS;
-  const float per_cta = (float)p.kv_units * (float)sum_len / (float)ctas;  // tokens of work per CTA
-  const float budget = (min_len * 10 >= max_len * 9 ? 0.6f : 0.3f) * per_cta;
+  if (max_blk <= 0) return p.partition_blocks;
+  const float budget = 0.6f * (float)p.kv_units * (float)sum_len / (float)ctas;  // tokens
   if ((float)max_len <= budget) return max(max_blk, p.partition_blocks);
   int pb = p.partition_blocks;
   while ((float)(2 * pb * kBS) <= budget && 2 * pb < max_blk) pb *= 2;
   return pb;
+}
+
+// Stream-K split of one sequence: its blocks occupy the global range
+// [a, a + nblk) of the flattened (sequence, block) space, which is cut into
+// equal ranges of `per_group` blocks, one per group of kv_units CTAs; the
+// sequence's pieces are the groups g0..g1 that overlap it (the same pieces for
+// every KV unit).
+struct Pieces {
+  int c0, count;
+};
+__device__ __forceinline__ Pieces unit_pieces(int a, int nblk, int per_group) {
+  const int c0 = a / per_group;
+  return {c0, (a + nblk - 1) / per_group - c0 + 1};
 }
 
 // Shared-memory layout of a decode CTA (offsets from a 1024-aligned base):
@@ -175,14 +196,21 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
   int* lens = prefix + (S + 1);                             // [S], clamped
 
 
-  // clamped lengths and their statistics -> partition size -> items per
-  // sequence -> exclusive prefix (a zero-length sequence is one item with no
-  // blocks, so that its zero output row gets written)
-  int pb = p.partition_blocks;
+  // Clamped lengths and their statistics; in auto mode the work hand-out is
+  // chosen from them: near-uniform lengths (all within 10 %) -> tickets with
+  // large partitions (items finish together; the memory system stays
+  // saturated), varying lengths -> stream-K ranges (no stragglers).  Then an
+  // exclusive prefix over the sequences of
+  //  ticket mode:    items (partitions x KV units; a zero-length sequence is
+  //                  one item with no blocks, so its zero output gets written)
+  //  stream-K mode:  blocks (a zero-length sequence has none; the merge
+  //                  kernel writes its zero output)
+  int pb = p.partition_blocks, per_cta = 0;
+  bool sk = false;
   if (warp == 1) {
+    bool bad = false;
     long long sum_len = 0;
     int min_len = 0x7fffffff, max_len = 0;
-    bool bad = false;
     for (int b = 0; b < S; b += 32) {
       const int s = b + lane;
       if (s < S) {
@@ -201,8 +229,11 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
       min_len = min(min_len, __shfl_xor_sync(0xffffffffu, min_len, off));
       max_len = max(max_len, __shfl_xor_sync(0xffffffffu, max_len, off));
     }
-    pb = choose_partition_blocks(p, sum_len, min_len, max_len, gridDim.x);
-    if (blockIdx.x == 0 && lane == 0) p.counters[2] = pb;
+    if (p.auto_mode) {
+      const bool uniform = (long long)min_len * 10 >= (long long)max_len * 9;
+      sk = !uniform && (int)gridDim.x >= p.kv_units;
+      if (!sk) pb = uniform_partition_blocks(p, sum_len, max_len, gridDim.x);
+    }
     __syncwarp();
     int carry = 0;
     for (int b = 0; b < S; b += 32) {
@@ -211,8 +242,12 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
       if (s < S) {
         const int len = lens[s];
         const int nblk = (len + kBS - 1) / kBS;
-        bad |= (nblk + pb - 1) / pb > p.max_parts;
-        n = max(1, num_partitions(len, pb, p));
+        if (sk) {
+          n = nblk;
+        } else {
+          bad |= (nblk + pb - 1) / pb > p.max_parts;
+          n = max(1, num_partitions(len, pb, p)) * p.kv_units;
+        }
       }
       int x = n;
 #pragma unroll
@@ -225,13 +260,26 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
     }
     if (lane == 0) prefix[0] = 0;
     if (blockIdx.x == 0 && __any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, kCheckSeqTooLong);
+    if (sk) {
+      const int groups = max(1, (int)gridDim.x / p.kv_units);
+      per_cta = max(p.min_piece_blocks, (carry + groups - 1) / groups);  // blocks per CTA group
+    }
+    if (blockIdx.x == 0) {  // what this launch used, for the merge kernel
+      __syncwarp();
+      if (sk)
+        for (int i = lane; i <= S; i += 32) p.seq_prefix[i] = prefix[i];
+      if (lane == 0) {
+        p.counters[2] = sk ? per_cta : pb;
+        p.counters[3] = sk ? 1 : 0;
+      }
+    }
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2 * NS + 4; ++i) mbar_init(full0 + 8 * i, 1);
     fence_mbar_init();
   }
   __syncthreads();
-  const int total = prefix[S] * p.kv_units;
+  const int total = prefix[S];  // items (ticket mode) or blocks (stream-K mode)
 
   if (warp == 1) {
     // ---------------------------------------------------------------- producer
@@ -249,26 +297,45 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
       }
       return true;
     };
-    // Item of ticket t (t < total): sequence, partition, KV unit, block range.
+    // A work item: sequence, partition (piece) index and count, KV unit, block range.
     struct Item {
       int s, y, part, np, len, b0, nb;
     };
-    auto decode = [&](int t) -> Item {
-      Item it;
-      const int idx = t / p.kv_units;
-      it.y = t - idx * p.kv_units;
-      int lo = 0, hi = S - 1;  // last s with prefix[s] <= idx
+    auto last_seq_at = [&](int v) {  // last s with prefix[s] <= v (skips empty sequences)
+      int lo = 0, hi = S - 1;
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
-        if (prefix[mid] <= idx) lo = mid; else hi = mid - 1;
+        if (prefix[mid] <= v) lo = mid; else hi = mid - 1;
       }
-      it.s = lo;
-      it.part = idx - prefix[lo];
-      it.len = lens[lo];
+      return lo;
+    };
+    // ticket mode: item t of the (sequence, partition, KV unit) enumeration
+    auto decode = [&](int t) -> Item {
+      Item it;
+      it.s = last_seq_at(t);
+      const int r = t - prefix[it.s];
+      it.part = r / p.kv_units;
+      it.y = r - it.part * p.kv_units;
+      it.len = lens[it.s];
       it.np = max(1, num_partitions(it.len, pb, p));
       const int nblk = (it.len + kBS - 1) / kBS;
       it.b0 = it.part * pb;
       it.nb = max(0, min(nblk, it.b0 + pb) - it.b0);
+      return it;
+    };
+    // stream-K mode: this CTA's KV unit of the sequence under global block g, up to `end`
+    const int sk_group = (int)blockIdx.x / p.kv_units;
+    auto decode_sk = [&](int g, int end) -> Item {
+      Item it;
+      it.s = last_seq_at(g);
+      it.len = lens[it.s];
+      const int nblk = (it.len + kBS - 1) / kBS;
+      it.y = (int)blockIdx.x - sk_group * p.kv_units;
+      it.b0 = g - prefix[it.s];
+      it.nb = min(nblk - it.b0, end - g);
+      const Pieces pc = unit_pieces(prefix[it.s], nblk, per_cta);
+      it.part = sk_group - pc.c0;
+      it.np = pc.count;
       return it;
     };
     // Lane j's block-table entry of chunk c (blocks 32c + j) of an item; out-of-pool ids are flagged.
@@ -284,36 +351,48 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
       }
       return b;
     };
+    // Work cursor: a ticket (ticket mode) or a global block index (stream-K
+    // mode, over this CTA's range [blockIdx.x * per_cta, g_end)).
     // Software pipeline: the next item's ticket is claimed four blocks before
     // this item's end (late enough to keep the hand-out dynamic, early enough
     // to hide the atomic's latency) and its first block-table chunk is loaded
     // one block later.
+    // Stream-K: group g = blockIdx / kv_units covers [g * per_cta, (g + 1) * per_cta)
+    // of the (sequence, block) space, each CTA of the group for its own KV unit
+    // (CTAs beyond the last whole group get no work).
+    const bool sk_idle = sk && sk_group >= max(1, (int)gridDim.x / p.kv_units);
+    const int g_end = sk ? (int)min((long long)total, ((long long)sk_group + 1) * per_cta) : 0;
+    auto has = [&](int t) { return sk ? (!sk_idle && t < g_end) : t < total; };
     int t_cur = 0, t_next = 0;
-    if (lane == 0) t_cur = atomicAdd(&p.counters[0], 1);
-    t_cur = __shfl_sync(0xffffffffu, t_cur, 0);
+    if (sk) {
+      t_cur = (int)min((long long)sk_group * per_cta, (long long)total);
+    } else {
+      if (lane == 0) t_cur = atomicAdd(&p.counters[0], 1);
+      t_cur = __shfl_sync(0xffffffffu, t_cur, 0);
+    }
     Item cur = {}, nxt = {};
     int chunk = 0, nchunk = 0;
-    if (t_cur < total) {
-      cur = decode(t_cur);
+    if (has(t_cur)) {
+      cur = sk ? decode_sk(t_cur, g_end) : decode(t_cur);
       chunk = load_chunk(cur, 0);
     }
-    while (t_cur < total && !stop) {
+    while (has(t_cur) && !stop) {
       const int kvh = cur.y / p.head_splits;
       const int hs = cur.y - kvh * p.head_splits;
       const int head0 = kvh * p.group + hs * kNH;
       const int nheads = min(kNH, p.group - hs * kNH);
       const int meta_z = cur.part | (cur.np << 16);
       bool claimed = false, fetched = false;
-      // claim / prefetch at blocks nb-2 / nb-1 (at once for items shorter than that)
+      // claim / prefetch near the item's end (at once for items shorter than that)
       auto lookahead = [&](int i) {
         if (!claimed && i >= cur.nb - 4) {
-          if (lane == 0) t_next = atomicAdd(&p.counters[0], 1);
+          if (!sk && lane == 0) t_next = atomicAdd(&p.counters[0], 1);
           claimed = true;
         }
         if (!fetched && i >= cur.nb - 3) {
-          t_next = __shfl_sync(0xffffffffu, t_next, 0);
-          if (t_next < total) {
-            nxt = decode(t_next);
+          t_next = sk ? t_cur + cur.nb : __shfl_sync(0xffffffffu, t_next, 0);
+          if (has(t_next)) {
+            nxt = sk ? decode_sk(t_next, g_end) : decode(t_next);
             nchunk = load_chunk(nxt, 0);
           }
           fetched = true;
@@ -678,31 +757,52 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
   asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int CH = D / 4;  // float4 chunks per head
   __shared__ float hM[kNH], hInvW[kNH];
+  __shared__ int hNp[kNH];
   __shared__ float4 red[256];
   const int hpc = p.merge_hpc, slices = p.merge_slices;
   const int hblocks = (p.num_heads + hpc - 1) / hpc;
   const int s = blockIdx.x / hblocks;
   const int h0 = (blockIdx.x - s * hblocks) * hpc;
-  const int pb = p.auto_partition ? p.counters[2] : p.partition_blocks;  // as the decode grid used
-  const int np = num_partitions(clamp_len(p.seq_lens[s], p), pb, p);
-  if (np <= 1) return;
+  const int len = clamp_len(p.seq_lens[s], p);
+  const int nblk = (len + kBS - 1) / kBS;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp < hpc && h0 + warp < p.num_heads) {
-    const float* ml = p.part_ml + ((size_t)s * p.num_heads + h0 + warp) * p.max_parts * 2;
-    float M = -INFINITY;
-    for (int q = lane; q < np; q += 32) M = fmaxf(M, ml[2 * q]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    float W = 0.f;
-    for (int q = lane; q < np; q += 32) {
-      const float2 v = *reinterpret_cast<const float2*>(ml + 2 * q);
-      if (v.y > 0.f) W += v.y * ex2(v.x - M);
+  // the decode launch's hand-out: stream-K or tickets with pb blocks per partition
+  const bool sk = p.auto_mode && p.counters[3] != 0;
+  const int param = p.auto_mode ? p.counters[2] : p.partition_blocks;
+  // partitions of head h (the same for every head of a sequence)
+  auto parts_of = [&](int h) -> int {
+    (void)h;
+    if (!sk) return num_partitions(len, param, p);
+    if (nblk == 0) return 0;
+    return unit_pieces(p.seq_prefix[s], nblk, param).count;
+  };
+  if (sk && nblk == 0) {  // empty sequence: zero rows (no decode item covered it)
+    for (int i = threadIdx.x; i < hpc * D; i += blockDim.x) {
+      const int h = h0 + i / D;
+      if (h < p.num_heads) reinterpret_cast<Q*>(p.out)[((size_t)s * p.num_heads + h) * D + i % D] = Q(0.0f);
     }
+    return;
+  }
+  if (warp < hpc) {
+    const int h = h0 + warp;
+    const int np = h < p.num_heads ? parts_of(h) : 0;
+    float M = -INFINITY, W = 0.f;
+    if (np > 1) {
+      const float* ml = p.part_ml + ((size_t)s * p.num_heads + h) * p.max_parts * 2;
+      for (int q = lane; q < np; q += 32) M = fmaxf(M, ml[2 * q]);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
+      for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+      for (int q = lane; q < np; q += 32) {
+        const float2 v = *reinterpret_cast<const float2*>(ml + 2 * q);
+        if (v.y > 0.f) W += v.y * ex2(v.x - M);
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
+    }
     if (lane == 0) {
       hM[warp] = M;
       hInvW[warp] = W > 0.f ? 1.f / W : 0.f;
+      hNp[warp] = np;
     }
   }
   __syncthreads();
@@ -710,8 +810,9 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
   const int rest = threadIdx.x / CH;
   const int slice = rest % slices, hl = rest / slices;
   const int h = h0 + hl;
+  const int np = hl < hpc ? hNp[hl] : 0;  // <= 1: written by the decode kernel
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (hl < hpc && h < p.num_heads) {
+  if (np > 1) {
     const size_t row0 = ((size_t)s * p.num_heads + h) * p.max_parts;
     const float* ml = p.part_ml + row0 * 2;
     const float* po = p.part_o + row0 * D + 4 * c;
@@ -738,7 +839,7 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
   }
   red[threadIdx.x] = acc;
   __syncthreads();
-  if (slice == 0 && hl < hpc && h < p.num_heads) {
+  if (slice == 0 && np > 1) {
     for (int k = 1; k < slices; ++k) {
       const float4 o = red[threadIdx.x + k * CH];
       acc.x += o.x;

@@ -97,6 +97,10 @@ cudaError_t launch_merge(const KernelSet& ks, const pa::DecodeParams& p, cudaStr
   return cudaLaunchKernelExC(&cfg, ks.merge, args);
 }
 
+// Shortest block range a CTA is given in stream-K mode (256 tokens), which
+// bounds the pieces a sequence can be cut into.
+constexpr int kMinPieceBlocks = 16;
+
 // query rows one item copies: min(group, 8) heads of head_dim 16-bit values
 int q_slot_bytes(int num_heads, int num_kv_heads, int head_dim) {
   const int g = num_heads / num_kv_heads;
@@ -181,7 +185,8 @@ struct pa_ctx {
   int partition_tokens = 0;     // current setting (PA_PARTITION_* or > 0)
   float* part_o = nullptr;
   float* part_ml = nullptr;
-  int* err = nullptr;           // [0] check word, [1..2] ticket / finished-CTA counters
+  int* err = nullptr;           // [0] check word, [1..4] decode kernel counters (DecodeParams::counters)
+  int* seq_prefix = nullptr;    // [max_num_seqs + 1] stream-K block offsets (decode -> merge)
   int* err_host = nullptr;      // pinned
   int grid = 0;                 // persistent grid: SMs x resident CTAs
   int last_bits = 0;
@@ -236,12 +241,7 @@ int tensor_map(pa_ctx* ctx, const void* base, CUtensorMap* out) {
   return PA_OK;
 }
 
-// Partition length for the host-side sizing of a launch: the configured one,
-// or for PA_PARTITION_AUTO the smallest the device may choose (the decode
-// kernel then picks the actual size from the lengths).
-int min_partition(const pa_ctx* ctx) {
-  return ctx->partition_tokens == PA_PARTITION_AUTO ? ctx->min_partition_tokens : ctx->partition_tokens;
-}
+
 
 }  // namespace
 
@@ -289,8 +289,11 @@ PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
   ctx->partition_tokens = c.partition_tokens;
   ctx->min_partition_tokens = c.partition_tokens > 0 ? c.partition_tokens : 512;
   const int max_tokens = c.max_blocks_per_seq * c.block_size;
-  ctx->max_parts = (max_tokens + ctx->min_partition_tokens - 1) / ctx->min_partition_tokens;
-  if (ctx->max_parts < 1) ctx->max_parts = 1;
+  // partials per (sequence, head): fixed partitions of >= min_partition_tokens,
+  // or stream-K pieces of >= kMinPieceBlocks blocks (+1 for a range boundary)
+  const int ticket_parts = (max_tokens + ctx->min_partition_tokens - 1) / ctx->min_partition_tokens;
+  const int sk_parts = (c.max_blocks_per_seq + kMinPieceBlocks - 1) / kMinPieceBlocks + 1;
+  ctx->max_parts = ticket_parts > sk_parts ? ticket_parts : sk_parts;
 
   int st = PA_OK;
   do {
@@ -329,9 +332,14 @@ PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
       break;
     }
     ctx->grid = ctx->num_sms * ctx->ctas_per_sm;
+    if ((e = cudaMalloc(&ctx->seq_prefix, (c.max_num_seqs + 1) * sizeof(int))) != cudaSuccess) {
+      cudaGetLastError();
+      st = PA_ERR_NO_MEMORY;
+      break;
+    }
 
-    if ((e = cudaMalloc(&ctx->err, 4 * sizeof(int))) != cudaSuccess ||
-        (e = cudaMemset(ctx->err, 0, 4 * sizeof(int))) != cudaSuccess) {
+    if ((e = cudaMalloc(&ctx->err, 8 * sizeof(int))) != cudaSuccess ||
+        (e = cudaMemset(ctx->err, 0, 8 * sizeof(int))) != cudaSuccess) {
       st = cuda_fail(ctx, e, "cudaMalloc(check word)");
       break;
     }
@@ -354,6 +362,7 @@ PA_API int paged_attn_destroy(pa_ctx* ctx) {
   if (ctx->part_o) cudaFree(ctx->part_o);
   if (ctx->part_ml) cudaFree(ctx->part_ml);
   if (ctx->err) cudaFree(ctx->err);
+  if (ctx->seq_prefix) cudaFree(ctx->seq_prefix);
   if (ctx->err_host) cudaFreeHost(ctx->err_host);
   delete ctx;
   return PA_OK;
@@ -455,12 +464,27 @@ PA_API int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, con
   if (st != PA_OK) return st;
   if ((st = tensor_map(ctx, value_cache, &mv)) != PA_OK) return st;
 
-  const int pt = min_partition(ctx);
+  // PA_PARTITION_AUTO: stream-K ranges (the split follows from the balance);
+  // otherwise fixed partitions handed out by tickets
+  const int group = c.num_heads / c.num_kv_heads;
+  const int kv_units = c.num_kv_heads * ((group + pa::kNH - 1) / pa::kNH);
+  const bool is_auto = ctx->partition_tokens == PA_PARTITION_AUTO;
   const int max_blocks = (max_seq_len + c.block_size - 1) / c.block_size;
+  // auto: the device picks tickets (partitions >= min_partition_tokens) or
+  // stream-K ranges (pieces >= kMinPieceBlocks) per call; the workspace holds
+  // either.  `parts` only shapes the merge kernel.
+  const int pt = is_auto ? ctx->min_partition_tokens : ctx->partition_tokens;
   const int part_blocks = pt > 0 ? pt / c.block_size : (max_blocks > 0 ? max_blocks : 1);
   int parts = (max_blocks + part_blocks - 1) / part_blocks;
   if (parts < 1) parts = 1;
   if (parts > ctx->max_parts) return fail(ctx, PA_ERR_INVALID_ARG, "too many partitions for the workspace");
+  if (is_auto && ctx->grid >= kv_units) {
+    const long long groups = ctx->grid / kv_units;
+    long long per_group = ((long long)num_seqs * (max_blocks > 0 ? max_blocks : 1) + groups - 1) / groups;
+    if (per_group < kMinPieceBlocks) per_group = kMinPieceBlocks;
+    const int sk_parts = (int)((max_blocks + per_group - 1) / per_group) + 1;
+    if (sk_parts > parts) parts = sk_parts < ctx->max_parts ? sk_parts : ctx->max_parts;
+  }
 
   DecodeParams p;
   p.out = out;
@@ -479,9 +503,12 @@ PA_API int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, con
   p.kv_units = c.num_kv_heads * p.head_splits;
   p.q_slot_bytes = q_slot_bytes(c.num_heads, c.num_kv_heads, c.head_dim);
   p.num_blocks = c.num_blocks;
+  p.max_blocks = max_blocks > 0 ? max_blocks : 1;
   p.partition_blocks = part_blocks;
-  p.auto_partition = (ctx->partition_tokens == PA_PARTITION_AUTO && pt > 0) ? 1 : 0;
-  p.max_parts = parts;
+  p.auto_mode = is_auto ? 1 : 0;
+  p.min_piece_blocks = kMinPieceBlocks;
+  p.seq_prefix = ctx->seq_prefix;
+  p.max_parts = ctx->max_parts;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
   p.v_scale = fp8 ? v_scale : 1.0f;
 
@@ -491,7 +518,8 @@ PA_API int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, con
   cudaError_t e = cudaLaunchKernel(ctx->ks.decode, dim3(ctx->grid), dim3(ctx->ks.threads), args,
                                    ctx->ks.smem(q_slot_bytes(c.num_heads, c.num_kv_heads, c.head_dim), c.max_num_seqs), s);
   if (e != cudaSuccess) return cuda_fail(ctx, e, "decode launch");
-  if (parts > 1 && (e = launch_merge(ctx->ks, p, s)) != cudaSuccess) return cuda_fail(ctx, e, "merge launch");
+  if ((is_auto || parts > 1) && (e = launch_merge(ctx->ks, p, s)) != cudaSuccess)
+    return cuda_fail(ctx, e, "merge launch");
   return PA_OK;
 }
 
@@ -705,8 +733,11 @@ PA_API int paged_attention_decode_noalloc(void* out, const void* query, const vo
   p.kv_units = num_kv_heads * p.head_splits;
   p.q_slot_bytes = q_slot_bytes(num_heads, num_kv_heads, head_dim);
   p.num_blocks = num_blocks;
+  p.max_blocks = max_blocks > 0 ? max_blocks : 1;
   p.partition_blocks = part_blocks;
-  p.auto_partition = 0;
+  p.auto_mode = 0;
+  p.min_piece_blocks = kMinPieceBlocks;
+  p.seq_prefix = nullptr;
   p.max_parts = parts;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
   p.v_scale = fp8 ? v_scale : 1.0f;
