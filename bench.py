@@ -392,12 +392,74 @@ def run_ours(args, world, rank, local):
     return 0
 
 
+def run_copy_blocks(args, world, rank, local):
+    """Block copies (copy-on-write / swap) on the 7B layer's block shape
+    (16 tokens x 32 heads x 128 dims fp16 = 128 KiB per tensor): device ->
+    device pairs, then a swap out to pinned host memory and back in.  GB/s
+    count bytes read + written on the device side (2 x K and V per block)."""
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    from paged_kv_cache_463_b200 import build
+    build.build()
+    spec = wl.SPEC_BY_NAME["llama2-7b-mha"]
+    nb = 12288
+    pa = pab.PagedAttention(spec.num_heads, spec.num_kv_heads, spec.head_dim, nb, max_num_seqs=1,
+                            max_blocks_per_seq=128, device=local)
+    dev = f"cuda:{local}"
+    kc = torch.randn((nb, 16, spec.num_kv_heads, spec.head_dim), device=dev).half()
+    vc = torch.randn_like(kc)
+    block_bytes = kc[0].numel() * kc.element_size()
+    perm = torch.randperm(nb, generator=torch.Generator().manual_seed(0))
+    n = 4096
+    pairs = torch.stack([perm[:n], perm[n:2 * n]], 1).to(torch.int64).to(dev)
+    hn = 1024
+    hk = torch.empty((hn, 16, spec.num_kv_heads, spec.head_dim), dtype=torch.float16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    out_pairs = torch.stack([perm[:hn], torch.arange(hn)], 1).to(torch.int64).to(dev)
+    in_pairs = torch.stack([torch.arange(hn), perm[2 * n:2 * n + hn]], 1).to(torch.int64).to(dev)
+    stream = torch.cuda.current_stream()
+
+    def timed(fn, steps):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / steps
+
+    d2d_ms = timed(lambda: pa.paged_copy_blocks(kc, vc, kc, vc, pairs, stream=stream), args.steps)
+    out_ms = timed(lambda: pa.paged_copy_blocks(hk, hv, kc, vc, out_pairs, stream=stream), max(3, args.steps // 10))
+    in_ms = timed(lambda: pa.paged_copy_blocks(kc, vc, hk, hv, in_pairs, stream=stream), max(3, args.steps // 10))
+    if pa.get_error() != 0:
+        raise SystemExit("device check fired")
+    d2d = 2 * 2 * n * block_bytes / (d2d_ms * 1e-3) / 1e9
+    line = {"metric": "paged block copy (copy-on-write, swap): GB/s read+written", "value": d2d, "unit": "GB/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": d2d_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic",
+            "config": {"workload": "block copy, 7B layer block shape (128 KiB per tensor per block)",
+                       "pairs": n, "swap_blocks": hn},
+            "swap_out_to_pinned_host_gbs": 2 * hn * block_bytes / (out_ms * 1e-3) / 1e9,
+            "swap_in_from_pinned_host_gbs": 2 * hn * block_bytes / (in_ms * 1e-3) / 1e9,
+            "roofline": {"bound": "hbm", "achieved": d2d, "peak": measured_hbm_peak()[0], "unit": "GB/s",
+                         "frac": d2d / measured_hbm_peak()[0]}}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    pa.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--op", choices=["decode-step", "copy-blocks"], default="decode-step",
+                    help="decode-step: the hot path (default); copy-blocks: block copies for COW / swap")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(wl.SPEC_BY_NAME))
     ap.add_argument("--partition", default="auto", help="auto | none | tokens per partition")
     ap.add_argument("--num-seqs", type=int, default=0, help="smaller batch of the same workload (profiling)")
@@ -410,6 +472,8 @@ def main():
     try:
         if args.impl == "reference":
             return run_reference(args, world, rank)
+        if args.op == "copy-blocks":
+            return run_copy_blocks(args, world, rank, local)
         return run_ours(args, world, rank, local)
     finally:
         if world > 1:

@@ -200,6 +200,28 @@ int paged_gather_kv(pa_ctx* ctx, void* k_out, void* v_out, const void* key_cache
                     const int32_t* block_table_row, int seq_len, void* stream);
 
 /*
+ * Whole-block copies between paged caches, for copy-on-write and swap.
+ * Copy-on-write (page "5.KV Cache 管理 & PagedAttention", Q18
+ * COWBlockManager.write_token): before a sequence writes into a block other
+ * sequences still share, the block is copied to a fresh one.  Swap (page "KV
+ * Cache 优化与内存管理深度解析", CPUSwap): blocks move from GPU to CPU memory
+ * and back into newly allocated GPU blocks.
+ * For each pair i: dst_cache[pairs[i][1]] = src_cache[pairs[i][0]] for both K
+ * and V (every token slot and KV head of the block; bytes unchanged).
+ * Caches: [*_num_blocks, block_size, num_kv_heads, head_dim] of the context's
+ * kv dtype, in any memory the device can address: device memory, or host
+ * memory allocated pinned (cudaMallocHost / cudaHostAlloc), which the kernel
+ * reads or writes directly over the host link.  block_pairs: int64
+ * [num_pairs][2] (src, dst), device or pinned host memory.  A pair naming a
+ * block outside its cache sets PA_CHECK_BAD_BLOCK and is skipped.  Pairs whose
+ * blocks overlap (a block written by one pair and read or written by another)
+ * give an unspecified result.  Pointers 16-byte aligned (pairs 8-byte).
+ */
+int paged_copy_blocks(pa_ctx* ctx, void* dst_key_cache, void* dst_value_cache, int64_t dst_num_blocks,
+                      const void* src_key_cache, const void* src_value_cache, int64_t src_num_blocks,
+                      const int64_t* block_pairs, int num_pairs, void* stream);
+
+/*
  * Decode attention that allocates nothing (the pages describe no counterpart:
  * it exists for callers of this library that cannot allocate device memory,
  * e.g. code running while its stream is being captured into a CUDA graph, or

@@ -69,6 +69,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "paged_attn_set_partition_tokens": (i, [_P, i]),
         "paged_attn_get_partition_tokens": (i, [_P, ctypes.POINTER(i)]),
         "paged_gather_kv": (i, [_P, _P, _P, _P, _P, _P, i, _P]),
+        "paged_copy_blocks": (i, [_P, _P, _P, i64, _P, _P, i64, _P, i, _P]),
         "paged_attention_decode_noalloc": (i, [_P, _P, _P, _P, _P, i, _P, i, i, i, i, i, i, i, i, i, i, f, f, f,
                                                _P, _P]),
     }
@@ -177,6 +178,16 @@ class PagedAttention:
         st = self.lib.paged_gather_kv(self.ctx, _ptr(k_out), _ptr(v_out), _ptr(key_cache), _ptr(value_cache),
                                       _ptr(block_table_row), int(seq_len), _stream_ptr(stream))
         self._check(st, "paged_gather_kv")
+
+    def paged_copy_blocks(self, dst_key_cache, dst_value_cache, src_key_cache, src_value_cache, block_pairs,
+                          stream=None) -> None:
+        """dst[pairs[i, 1]] = src[pairs[i, 0]] for whole blocks (copy-on-write, swap).
+        The caches may be device tensors or pinned host tensors."""
+        st = self.lib.paged_copy_blocks(self.ctx, _ptr(dst_key_cache), _ptr(dst_value_cache),
+                                        dst_key_cache.shape[0], _ptr(src_key_cache), _ptr(src_value_cache),
+                                        src_key_cache.shape[0], _ptr(block_pairs), block_pairs.shape[0],
+                                        _stream_ptr(stream))
+        self._check(st, "paged_copy_blocks")
 
     def get_error(self, stream=None) -> int:
         """Synchronise and return (then clear) the device check bits."""

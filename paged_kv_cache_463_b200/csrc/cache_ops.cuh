@@ -9,7 +9,14 @@
 // Gather (Q11 read_kv_range): tokens [0, seq_len) of one sequence copied out
 // of paged storage into a contiguous [seq_len, Hkv, D] buffer, bytes unchanged.
 //
-// Both are pure data movement: one thread moves one 16-byte source vector.
+// Block copy (page "5.KV Cache 管理 & PagedAttention", Q18 copy-on-write: a
+// shared block is copied before a sequence writes into it; page "KV Cache
+// 优化与内存管理深度解析", CPUSwap: blocks move between GPU and CPU memory):
+// dst_cache[dst] = src_cache[src] for each (src, dst) pair, whole blocks (all
+// token slots and KV heads, K and V).  Either cache may be pinned host memory,
+// which the kernel reaches directly over the host link.
+//
+// All are pure data movement: one thread moves 16-byte vectors.
 #pragma once
 
 #include "decode.cuh"
@@ -131,6 +138,49 @@ __global__ void __launch_bounds__(256) paged_gather_kernel(const GatherParams p)
       x = *reinterpret_cast<const uint4*>(src + row * p.row_bytes + v * 16);
     }
     *reinterpret_cast<uint4*>(dst + (long long)pos * p.row_bytes + v * 16) = x;
+  }
+}
+
+struct CopyBlocksParams {
+  void* dst_key;
+  void* dst_value;
+  const void* src_key;
+  const void* src_value;
+  const long long* pairs;  // [num_pairs, 2]: (src block, dst block)
+  int num_pairs;
+  int block_vecs;          // 16-byte vectors per block and tensor
+  long long src_blocks, dst_blocks;
+  int* err;
+};
+
+// CTAs stride over the pairs; the threads of a CTA copy one block's 16-byte
+// vectors, four independent copies in flight per thread.  blockIdx.y selects
+// K (0) or V (1).
+__global__ void __launch_bounds__(256) paged_copy_blocks_kernel(const CopyBlocksParams p) {
+  const bool is_v = blockIdx.y == 1;
+  const uint4* src = reinterpret_cast<const uint4*>(is_v ? p.src_value : p.src_key);
+  uint4* dst = reinterpret_cast<uint4*>(is_v ? p.dst_value : p.dst_key);
+  for (int pair = blockIdx.x; pair < p.num_pairs; pair += gridDim.x) {
+    const long long sb = p.pairs[2 * pair], db = p.pairs[2 * pair + 1];
+    if (sb < 0 || sb >= p.src_blocks || db < 0 || db >= p.dst_blocks) {
+      if (threadIdx.x == 0) atomicOr(p.err, kCheckBadBlock);
+      continue;
+    }
+    const uint4* s = src + sb * p.block_vecs;
+    uint4* d = dst + db * p.block_vecs;
+    for (int w0 = threadIdx.x; w0 < p.block_vecs; w0 += 4 * blockDim.x) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int w = w0 + u * blockDim.x;
+        if (w < p.block_vecs) v[u] = s[w];
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int w = w0 + u * blockDim.x;
+        if (w < p.block_vecs) d[w] = v[u];
+      }
+    }
   }
 }
 

@@ -55,7 +55,8 @@ cudaError_t pin_all_carveouts(const KernelSet& ks) {
   const void* fns[] = {ks.decode, ks.merge, reinterpret_cast<const void*>(&pa::reshape_and_cache_copy_kernel),
                        reinterpret_cast<const void*>(&pa::reshape_and_cache_fp8_kernel<true>),
                        reinterpret_cast<const void*>(&pa::reshape_and_cache_fp8_kernel<false>),
-                       reinterpret_cast<const void*>(&pa::paged_gather_kernel)};
+                       reinterpret_cast<const void*>(&pa::paged_gather_kernel),
+                       reinterpret_cast<const void*>(&pa::paged_copy_blocks_kernel)};
   for (const void* f : fns) {
     cudaError_t e = pin_carveout(f);
     if (e != cudaSuccess) return e;
@@ -749,4 +750,37 @@ PA_API int paged_attention_decode_noalloc(void* out, const void* query, const vo
     return PA_ERR_CUDA;
   if (parts > 1 && launch_merge(ks, p, s) != cudaSuccess) return PA_ERR_CUDA;
   return PA_OK;
+}
+
+PA_API int paged_copy_blocks(pa_ctx* ctx, void* dst_key_cache, void* dst_value_cache, int64_t dst_num_blocks,
+                             const void* src_key_cache, const void* src_value_cache, int64_t src_num_blocks,
+                             const int64_t* block_pairs, int num_pairs, void* stream) {
+  if (!ctx) return PA_ERR_INVALID_ARG;
+  const pa_config& c = ctx->cfg;
+  if (num_pairs < 0) return fail(ctx, PA_ERR_INVALID_ARG, "num_pairs < 0");
+  if (num_pairs == 0) return PA_OK;
+  if (!dst_key_cache || !dst_value_cache || !src_key_cache || !src_value_cache || !block_pairs)
+    return fail(ctx, PA_ERR_INVALID_ARG, "null pointer");
+  if (dst_num_blocks <= 0 || src_num_blocks <= 0) return fail(ctx, PA_ERR_INVALID_ARG, "block counts must be > 0");
+  if (!aligned(dst_key_cache, 16) || !aligned(dst_value_cache, 16) || !aligned(src_key_cache, 16) ||
+      !aligned(src_value_cache, 16) || !aligned(block_pairs, 8))
+    return fail(ctx, PA_ERR_INVALID_ARG, "misaligned pointer");
+  cudaSetDevice(ctx->device);
+  pa::CopyBlocksParams p;
+  p.dst_key = dst_key_cache;
+  p.dst_value = dst_value_cache;
+  p.src_key = src_key_cache;
+  p.src_value = src_value_cache;
+  p.pairs = reinterpret_cast<const long long*>(block_pairs);
+  p.num_pairs = num_pairs;
+  p.block_vecs = c.block_size * c.num_kv_heads * c.head_dim * elem_bytes(c.kv_dtype) / 16;
+  p.src_blocks = src_num_blocks;
+  p.dst_blocks = dst_num_blocks;
+  p.err = ctx->err;
+  long long blocks = num_pairs;
+  const long long cap = (long long)ctx->num_sms * 16;
+  if (blocks > cap) blocks = cap;
+  pa::paged_copy_blocks_kernel<<<dim3((unsigned)blocks, 2), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? PA_OK : cuda_fail(ctx, e, "paged_copy_blocks launch");
 }
