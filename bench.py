@@ -257,10 +257,13 @@ def run_ours(args, world, rank, local):
     w = wl.make_workload(spec, dev)
     part = {"auto": pab.PA_PARTITION_AUTO, "none": pab.PA_PARTITION_NONE}.get(args.partition)
     part = int(args.partition) if part is None else part
+    shared = w.group_start is not None and args.shared_prefix != "off"
+    if args.shared_prefix == "on" and not shared:
+        raise SystemExit(f"workload {spec.name} has no shared-prefix groups")
     pa = pab.PagedAttention(spec.num_heads, spec.num_kv_heads, spec.head_dim, w.num_blocks,
                             block_size=spec.block_size, q_dtype=spec.q_dtype, kv_dtype=spec.kv_dtype,
                             max_num_seqs=spec.num_seqs, max_blocks_per_seq=w.block_tables.shape[1],
-                            partition_tokens=part, device=local)
+                            partition_tokens=part, device=local, shared_prefix=shared)
     if spec.kv_dtype == "fp8_e4m3":
         NB, bs, Hkv, D = w.key_src.shape
         kc = torch.empty((NB, bs, Hkv, D), dtype=torch.float8_e4m3fn, device=dev)
@@ -274,12 +277,26 @@ def run_ours(args, world, rank, local):
     stream = torch.cuda.current_stream()
     max_len = w.max_seq_len
     chosen_part = pa.get_partition_tokens()
-    launches_per_step = 2  # cache write + decode (split partitions are merged inside the decode kernel)
+    # cache write + decode, + the merge kernel (auto partitioning or a split),
+    # + the prefix pass (shared-prefix decode)
+    launches_per_step = 2 + (1 if (chosen_part < 0 or shared or 0 < chosen_part < max_len) else 0) + \
+        (1 if shared else 0)
+    if shared:
+        gsizes = (w.group_start[1:] - w.group_start[:-1]).cpu()
+        max_group = int(gsizes.max().item())
+        max_prefix = int(w.group_prefix_len.max().item())
+
+    def attend(q, bt, lens):
+        if shared:
+            pa.paged_attention_decode_shared_prefix(out, q, kc, vc, bt, lens, max_len, w.group_start,
+                                                    w.group_prefix_len, max_group, max_prefix, w.scale,
+                                                    w.k_scale, w.v_scale, stream)
+        else:
+            pa.paged_attention_decode(out, q, kc, vc, bt, lens, max_len, w.scale, w.k_scale, w.v_scale, stream)
 
     def step():
         pa.reshape_and_cache(w.new_key, w.new_value, kc, vc, w.slot_mapping, w.k_scale, w.v_scale, stream)
-        pa.paged_attention_decode(out, w.query, kc, vc, w.block_tables, w.seq_lens, max_len, w.scale,
-                                  w.k_scale, w.v_scale, stream)
+        attend(w.query, w.block_tables, w.seq_lens)
 
     for _ in range(args.warmup):
         step()
@@ -301,8 +318,7 @@ def run_ours(args, world, rank, local):
             a.record(stream)
             pa.reshape_and_cache(w.new_key, w.new_value, kc, vc, w.slot_mapping, w.k_scale, w.v_scale, stream)
             m.record(stream)
-            pa.paged_attention_decode(out, w.query, kc, vc, w.block_tables, w.seq_lens, max_len, w.scale,
-                                      w.k_scale, w.v_scale, stream)
+            attend(w.query, w.block_tables, w.seq_lens)
             e.record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -334,8 +350,7 @@ def run_ours(args, world, rank, local):
             dev_in[k].copy_(t, non_blocking=True)
         pa.reshape_and_cache(dev_in["new_key"], dev_in["new_value"], kc, vc, dev_in["slot_mapping"], w.k_scale,
                              w.v_scale, stream)
-        pa.paged_attention_decode(out, dev_in["query"], kc, vc, dev_in["block_tables"], dev_in["seq_lens"],
-                                  max_len, w.scale, w.k_scale, w.v_scale, stream)
+        attend(dev_in["query"], dev_in["block_tables"], dev_in["seq_lens"])
         out_host.copy_(out, non_blocking=True)
 
     for _ in range(args.warmup):
@@ -353,8 +368,10 @@ def run_ours(args, world, rank, local):
 
     peak, peak_kind = measured_hbm_peak()
     dec_avg_ms = sum(decode_ms) / len(decode_ms)
-    achieved = dec_bytes / (dec_avg_ms * 1e-3) / 1e9
-    traffic = traffic_record("paged_decode_kernel", spec.name)
+    # bytes the call must move: with shared prefixes, each group's prefix once
+    alg_bytes = wl.shared_decode_bytes(w) if shared else dec_bytes
+    achieved = alg_bytes / (dec_avg_ms * 1e-3) / 1e9
+    traffic = None if shared else traffic_record("paged_decode_kernel", spec.name)
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -367,14 +384,20 @@ def run_ours(args, world, rank, local):
                    "partition_tokens": "auto (chosen by the decode kernel from the lengths)" if chosen_part < 0
                    else chosen_part,
                    "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
+                   "shared_prefix": bool(shared),
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "seq_steps_per_s": seq_steps,
         "pct_of_nominal_8tbs": 100.0 * value / world / NOMINAL_HBM_GBS,
         "pct_of_measured_copy": 100.0 * value / world / peak,
         "bytes_per_step": dec_bytes,
+        "bytes_note": ("value counts every sequence's prefix (the metric's byte formula); the roofline counts "
+                       "each group's shared prefix once (the bytes the call must read)") if shared else None,
         "decode_ms": dec_avg_ms, "cache_write_ms": sum(write_ms) / len(write_ms),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "kernel": "paged_decode_kernel",
+                     "traffic": traffic,
+                     "kernel": ("paged_prefix_kernel + paged_decode_kernel + merge (the whole call)" if shared
+                                else "paged_decode_kernel"),
+                     "algorithmic_bytes": alg_bytes,
                      "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
                      if peak_kind == "measured" else "fallback 6.65 TB/s"},
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
@@ -463,6 +486,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(wl.SPEC_BY_NAME))
     ap.add_argument("--partition", default="auto", help="auto | none | tokens per partition")
     ap.add_argument("--num-seqs", type=int, default=0, help="smaller batch of the same workload (profiling)")
+    ap.add_argument("--shared-prefix", choices=["auto", "on", "off"], default="auto",
+                    help="shared-prefix decode for workloads with prefix groups (auto: when the workload has them)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
     args = ap.parse_args()

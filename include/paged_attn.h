@@ -53,6 +53,8 @@ extern "C" {
 #define PA_CHECK_BAD_SLOT 2     /* slot >= num_blocks * block_size: write skipped */
 #define PA_CHECK_SEQ_TOO_LONG 4 /* seq_len > bt_stride * block_size, < 0, or beyond max_seq_len: clamped */
 #define PA_CHECK_WAIT_TIMEOUT 8 /* a shared-memory pipeline wait gave up: that CTA's output is invalid */
+#define PA_CHECK_BAD_PREFIX 16  /* shared-prefix decode: a group's description was unusable (see
+                                   paged_attention_decode_shared_prefix) */
 
 /* ---- element types */
 typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
@@ -83,8 +85,13 @@ typedef enum pa_dtype { PA_F16 = 0, PA_BF16 = 1, PA_FP8_E4M3 = 2 } pa_dtype;
  *                             multiple of 512 tokens (or no split) that keeps every
  *                             work item a modest fraction of one CTA's share.
  *   device                  : CUDA device ordinal the context and its calls use.
- *   flags                   : reserved, must be 0.
+ *   flags                   : 0, or PA_FLAG_SHARED_PREFIX: also allocate the
+ *                             shared-prefix workspace (max_num_seqs * num_heads *
+ *                             ceil(max_blocks_per_seq / 32) * (head_dim + 2) floats,
+ *                             plus max_num_seqs ints) that
+ *                             paged_attention_decode_shared_prefix needs.
  */
+#define PA_FLAG_SHARED_PREFIX 1
 typedef struct pa_config {
   int num_heads;
   int num_kv_heads;
@@ -158,6 +165,49 @@ int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, const void
                            const void* value_cache, const int32_t* block_tables, int bt_stride,
                            const int32_t* seq_lens, int num_seqs, int max_seq_len, float scale, float k_scale,
                            float v_scale, void* stream);
+
+/*
+ * Decode attention for batches in which groups of sequences share the physical
+ * blocks of a common prefix: sequences forked from one prompt (page "5.KV Cache
+ * 管理 & PagedAttention", Q18: the fork copies the parent's block table and
+ * raises the shared blocks' reference counts), or requests that reuse cached
+ * prefix blocks (page "paged-attention-and-vllm-inference", prefix caching).
+ * The result is the same as paged_attention_decode's on the same arguments
+ * (rounding aside); only the order of work differs.  Each shared block is read
+ * once per group and scored against the queries of all its members (one pass
+ * over the prefixes); each sequence's private suffix is then decoded as usual,
+ * and the two sets of partial results are combined by log-sum-exp.
+ *
+ * Groups (device int32 arrays):
+ *   group_start[num_groups + 1]  : group g is sequences [group_start[g],
+ *                                  group_start[g + 1]); non-decreasing, within
+ *                                  [0, num_seqs].  Sequences before
+ *                                  group_start[0] or from group_start[num_groups]
+ *                                  on share nothing.
+ *   group_prefix_len[num_groups] : tokens that group g's members share: a
+ *                                  multiple of block_size (whole blocks), at most
+ *                                  every member's seq_lens, at most
+ *                                  max_prefix_len, and the members' block tables
+ *                                  name the same physical blocks for it.  0: no
+ *                                  shared prefix.
+ * Host bounds: 1 <= num_groups <= num_seqs; 1 <= max_group_size <= num_seqs
+ * (largest group); 0 <= max_prefix_len <= max_seq_len (largest prefix).
+ * A group that breaks one of these rules (too many members, a prefix length
+ * that is not a block multiple, longer than a member or than max_prefix_len,
+ * or tables that differ over the prefix) sets PA_CHECK_BAD_PREFIX and its
+ * members are decoded in full, without sharing (the output stays correct).  A
+ * group_start that is decreasing or leaves [0, num_seqs] sets the same bit and
+ * the affected sequences' outputs are unspecified.
+ * The context must have been created with PA_FLAG_SHARED_PREFIX
+ * (PA_ERR_UNSUPPORTED otherwise).  Launches the prefix pass, the decode pass
+ * over the suffixes and the merge kernel, in stream order.
+ */
+int paged_attention_decode_shared_prefix(pa_ctx* ctx, void* out, const void* query, const void* key_cache,
+                                         const void* value_cache, const int32_t* block_tables, int bt_stride,
+                                         const int32_t* seq_lens, int num_seqs, int max_seq_len,
+                                         const int32_t* group_start, const int32_t* group_prefix_len,
+                                         int num_groups, int max_group_size, int max_prefix_len, float scale,
+                                         float k_scale, float v_scale, void* stream);
 
 /*
  * Synchronise `stream`, read and clear the context's device check word.

@@ -22,6 +22,7 @@ pages it cites:
                      recurrence that the GPU path uses.
 * ``cache_write`` -- the per-token slot write (reshape_and_cache).
 * ``block_copy``  -- whole-block copies (copy-on-write fork, CPU swap).
+* ``prefix_sharing`` -- the whole blocks a group of forked sequences shares.
 * ``fp8_e4m3``    -- an OCP FP8 E4M3 codec written from the format definition.
 * ``dtypes``      -- raw 16-bit / 8-bit storage -> fp64 values.
 * ``kv_size``     -- the pages' closed-form KV-cache size.
@@ -32,4 +33,4 @@ than itself: the pages' worked values, closed forms, invariants, and library
 routines (torch SDPA, torch's fp8/bf16 casts) on special cases.
 """
 
-from . import attention, block_copy, cache_write, dtypes, fp8_e4m3, kv_size, paging  # noqa: F401
+from . import attention, block_copy, cache_write, dtypes, fp8_e4m3, kv_size, paging, prefix_sharing  # noqa: F401

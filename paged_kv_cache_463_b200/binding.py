@@ -27,6 +27,8 @@ PA_ERR_NO_MEMORY = -5
 PA_ERR_SCRATCH_TOO_SMALL = -6
 PA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 PA_CHECK_BAD_BLOCK, PA_CHECK_BAD_SLOT, PA_CHECK_SEQ_TOO_LONG, PA_CHECK_WAIT_TIMEOUT = 1, 2, 4, 8
+PA_CHECK_BAD_PREFIX = 16
+PA_FLAG_SHARED_PREFIX = 1
 PA_PARTITION_NONE, PA_PARTITION_AUTO = 0, -1
 DTYPE_CODES = {"f16": 0, "bf16": 1, "fp8_e4m3": 2}
 TORCH_OF = {"f16": torch.float16, "bf16": torch.bfloat16, "fp8_e4m3": torch.float8_e4m3fn}
@@ -62,6 +64,8 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "paged_attn_destroy": (i, [_P]),
         "reshape_and_cache": (i, [_P, _P, _P, i64, i64, _P, _P, _P, i, f, f, _P]),
         "paged_attention_decode": (i, [_P, _P, _P, _P, _P, _P, i, _P, i, i, f, f, f, _P]),
+        "paged_attention_decode_shared_prefix": (i, [_P, _P, _P, _P, _P, _P, i, _P, i, i, _P, _P, i, i, i, f, f, f,
+                                                     _P]),
         "paged_attn_get_error": (i, [_P, _P]),
         "paged_attn_last_check_bits": (i, [_P]),
         "paged_attn_status_string": (ctypes.c_char_p, [i]),
@@ -126,12 +130,14 @@ class PagedAttention:
 
     def __init__(self, num_heads: int, num_kv_heads: int, head_dim: int, num_blocks: int, *, block_size: int = 16,
                  q_dtype: str = "f16", kv_dtype: str = "f16", max_num_seqs: int, max_blocks_per_seq: int,
-                 partition_tokens: int = PA_PARTITION_AUTO, device: int | None = None, lib_path: str | None = None):
+                 partition_tokens: int = PA_PARTITION_AUTO, device: int | None = None, lib_path: str | None = None,
+                 shared_prefix: bool = False):
         self.lib = load_library(lib_path)
         if device is None:
             device = torch.cuda.current_device() if torch.cuda.is_available() else 0
         self.cfg = PaConfig(num_heads, num_kv_heads, head_dim, block_size, num_blocks, DTYPE_CODES[q_dtype],
-                            DTYPE_CODES[kv_dtype], max_num_seqs, max_blocks_per_seq, partition_tokens, device, 0)
+                            DTYPE_CODES[kv_dtype], max_num_seqs, max_blocks_per_seq, partition_tokens, device,
+                            PA_FLAG_SHARED_PREFIX if shared_prefix else 0)
         self.q_dtype, self.kv_dtype = q_dtype, kv_dtype
         self.device = device
         ctx = _P()
@@ -172,6 +178,20 @@ class PagedAttention:
                                              query.shape[0], int(max_seq_len), float(scale), float(k_scale),
                                              float(v_scale), _stream_ptr(stream))
         self._check(st, "paged_attention_decode")
+
+    def paged_attention_decode_shared_prefix(self, out, query, key_cache, value_cache, block_tables, seq_lens,
+                                             max_seq_len: int, group_start, group_prefix_len, max_group_size: int,
+                                             max_prefix_len: int, scale: float, k_scale=1.0, v_scale=1.0,
+                                             stream=None) -> None:
+        """Decode with groups of sequences sharing prefix blocks: group g is
+        sequences [group_start[g], group_start[g+1]) sharing group_prefix_len[g]
+        tokens (device int32 tensors).  Needs ``shared_prefix=True`` at construction."""
+        st = self.lib.paged_attention_decode_shared_prefix(
+            self.ctx, _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache), _ptr(block_tables),
+            block_tables.stride(0), _ptr(seq_lens), query.shape[0], int(max_seq_len), _ptr(group_start),
+            _ptr(group_prefix_len), group_prefix_len.shape[0], int(max_group_size), int(max_prefix_len),
+            float(scale), float(k_scale), float(v_scale), _stream_ptr(stream))
+        self._check(st, "paged_attention_decode_shared_prefix")
 
     def paged_gather_kv(self, k_out, v_out, key_cache, value_cache, block_table_row, seq_len: int,
                         stream=None) -> None:

@@ -74,6 +74,7 @@ struct DecodeParams {
   int kv_units;     // num_kv_heads * head_splits
   int num_blocks;   // physical pool size
   int max_blocks;        // ceil(max_seq_len / 16) of the call: lengths are clamped to it
+  int force_partials;    // 1: one-partition sequences also write partials (a prefix pass adds terms)
   int partition_blocks;  // ticket mode: blocks per partition
   int auto_mode;         // 1: the kernel chooses tickets or stream-K (and the partition) from the lengths
   int min_piece_blocks;  // stream-K mode: shortest range a CTA group is given
@@ -84,7 +85,16 @@ struct DecodeParams {
   int merge_slices; // merge kernel: partition slices per head
   float scale_log2;  // softmax scale * log2(e) (* k_scale for fp8)
   float v_scale;     // 1, or the fp8 value scale
+  // shared-prefix decode (all null / 0 otherwise): the prefix pass covered the
+  // first seq_skip[s] blocks of sequence s; this pass covers the rest, and the
+  // merge adds the prefix pass's ceil(seq_skip[s] / 32) partials per head
+  const int* seq_skip = nullptr;  // [S]
+  const float* pre_o = nullptr;   // [S, Hq, max_chunks, D]
+  const float* pre_ml = nullptr;  // [S, Hq, max_chunks, 2]
+  int max_chunks = 0;
 };
+
+constexpr int kPrefixChunkBlocks = 32;  // blocks per partial of the prefix pass
 
 // Clamp a sequence length to what its table row can address and to the
 // call's max_seq_len bound (which sizes the partial workspace).
@@ -175,6 +185,236 @@ __device__ __forceinline__ uint32_t tile_off(int row, int byte) {
   return (uint32_t)(sub * (kBS * 128) + row * 128 + ((((in >> 4) ^ (row & 7)) << 4) | (in & 15)));
 }
 
+// Store a warp's normalised partial rows (o / l as fp32, plus (m, l)) for
+// output columns 2*c4 (row0) and 2*c4 + 1 (row1), straight from registers.
+template <int D, bool FP8>
+__device__ __forceinline__ void store_partial(const float (&o)[D / 16][4], float m0, float L0, float i0, bool ok0,
+                                              float m1, float L1, float i1, bool ok1, float* part_o, float* part_ml,
+                                              size_t row0, size_t row1, int lane) {
+  const int gid = lane >> 2;
+  float* d0 = part_o + row0 * D;
+  float* d1 = part_o + row1 * D;
+#pragma unroll
+  for (int t = 0; t < D / 16; ++t) {
+    if constexpr (!FP8) {
+      if (ok0) {
+        d0[16 * t + gid] = o[t][0] * i0;
+        d0[16 * t + gid + 8] = o[t][2] * i0;
+      }
+      if (ok1) {
+        d1[16 * t + gid] = o[t][1] * i1;
+        d1[16 * t + gid + 8] = o[t][3] * i1;
+      }
+    } else {  // adjacent dims: one 8-byte store per column
+      const int d = (D / 8) * gid + 2 * t;
+      if (ok0) *reinterpret_cast<float2*>(d0 + d) = make_float2(o[t][0] * i0, o[t][2] * i0);
+      if (ok1) *reinterpret_cast<float2*>(d1 + d) = make_float2(o[t][1] * i1, o[t][3] * i1);
+    }
+  }
+  if (gid == 0) {
+    if (ok0) *reinterpret_cast<float2*>(part_ml + row0 * 2) = make_float2(m0, L0);
+    if (ok1) *reinterpret_cast<float2*>(part_ml + row1 * 2) = make_float2(m1, L1);
+  }
+}
+
+// One warp's attention state for 8 query columns (MMA N) over a stream of
+// 16-token K/V tiles in shared memory, and the per-tile math:
+//   S^T[16 tok x 8] = K[16 x D] . Q^T[D x 8]          (mma.m16n8k16)
+//   online softmax in the log2 domain with lazy rescaling
+//   O^T[D x 8] += V^T[D x 16 tok] . P^T[16 x 8]        (P^T via movmatrix)
+// Lane (gid = lane / 4, c4 = lane % 4) holds query column gid's fragments and
+// the output columns 2*c4, 2*c4 + 1.  FP8 tiles (E4M3) are converted to f16 in
+// registers, with the contraction order permuted so that a lane's operand
+// bytes are contiguous.
+template <int D, bool FP8, bool BF16>
+struct WarpAttn {
+  static constexpr int NKT = D / 16;
+  static constexpr int NDT = D / 16;
+  uint32_t qf[NKT][2];
+  float o[NDT][4];
+  float m0, m1, l0, l1;
+
+  __device__ __forceinline__ void reset() {
+#pragma unroll
+    for (int t = 0; t < NDT; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
+    m0 = m1 = -INFINITY;
+    l0 = l1 = 0.f;
+  }
+
+  // Q^T as MMA B fragments from this lane's query column (row gid of the
+  // warp's 8); `row` == nullptr gives a zero column.  16-bit elements.
+  __device__ __forceinline__ void load_q(const void* row, int c4) {
+    const uint8_t* q = reinterpret_cast<const uint8_t*>(row);
+#pragma unroll
+    for (int j = 0; j < NKT; ++j) {
+      if constexpr (!FP8) {
+        qf[j][0] = q ? *reinterpret_cast<const uint32_t*>(q + 2 * (16 * j + 2 * c4)) : 0u;
+        qf[j][1] = q ? *reinterpret_cast<const uint32_t*>(q + 2 * (16 * j + 2 * c4 + 8)) : 0u;
+      } else {
+        // permuted contraction order: lane column c4 owns dims [D/4*c4, D/4*c4 + D/4)
+        const uint2 v = q ? *reinterpret_cast<const uint2*>(q + 2 * ((D / 4) * c4 + 4 * j)) : make_uint2(0u, 0u);
+        qf[j][0] = v.x;
+        qf[j][1] = v.y;
+      }
+    }
+  }
+
+  // One 16-token tile: K at kb, V at vb (shared addresses, 128-byte swizzled
+  // [16 x D] tiles); tokens >= valid are masked out.  sl = softmax scale x log2(e).
+  __device__ __forceinline__ void block(uint32_t kb, uint32_t vb, int valid, float sl, int lane) {
+    const int gid = lane >> 2, c4 = lane & 3;
+    const int mi = lane >> 3, ri = lane & 7;
+    // ---- S^T = K Q^T
+    float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+    if constexpr (!FP8) {
+#pragma unroll
+      for (int j = 0; j < NKT; ++j) {
+        const int tok = ri + ((mi & 1) << 3);
+        const int dim = 16 * j + ((mi >> 1) << 3);
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(kb + tile_off(tok, dim * 2), a0, a1, a2, a3);
+        if (j & 1)
+          mma_16816<BF16>(sb, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+        else
+          mma_16816<BF16>(sa, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+      }
+    } else {
+      constexpr int LB = D / 4;  // bytes of a K row owned by one lane
+      constexpr int LC = LB / 16;
+      uint4 kr[2][LC];
+#pragma unroll
+      for (int u = 0; u < LC; ++u) {
+        kr[0][u] = lds128(kb + tile_off(gid, LB * c4 + 16 * u));
+        kr[1][u] = lds128(kb + tile_off(gid + 8, LB * c4 + 16 * u));
+      }
+      const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&kr[0][0]);
+      const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&kr[1][0]);
+#pragma unroll
+      for (int j = 0; j < NKT; ++j) {
+        uint32_t a0, a1, a2, a3;
+        e4m3x4_to_f16x2x2(w0[j], a0, a2);
+        e4m3x4_to_f16x2x2(w1[j], a1, a3);
+        if (j & 1)
+          mma_16816<false>(sb, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+        else
+          mma_16816<false>(sa, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+      }
+    }
+    // ---- online softmax (log2 domain); rows of S^T are tokens gid, gid+8
+            const float x0 = gid < valid ? (sa[0] + sb[0]) * sl : -INFINITY;
+    const float x1 = gid < valid ? (sa[1] + sb[1]) * sl : -INFINITY;
+    const float x2 = gid + 8 < valid ? (sa[2] + sb[2]) * sl : -INFINITY;
+    const float x3 = gid + 8 < valid ? (sa[3] + sb[3]) * sl : -INFINITY;
+    float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
+      bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
+    }
+    // Lazy rescaling: the reference max only moves (and O, l are
+    // rescaled) when some head's block max exceeds it by more than
+    // 2^kLazy; otherwise weights up to 2^kLazy are accumulated as they are
+    // (exact in fp32, and well inside the 16-bit P range).
+    constexpr float kLazy = 8.f;
+    const bool grow = (bm0 > m0 + kLazy) || (bm1 > m1 + kLazy);
+    if (__any_sync(0xffffffffu, grow)) {
+      const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
+      const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
+      m0 = mn0;
+      m1 = mn1;
+      l0 *= al0;
+      l1 *= al1;
+#pragma unroll
+      for (int t = 0; t < NDT; ++t) {
+        o[t][0] *= al0;
+        o[t][1] *= al1;
+        o[t][2] *= al0;
+        o[t][3] *= al1;
+      }
+    }
+    const float p0 = ex2(x0 - m0), p1 = ex2(x1 - m1), p2 = ex2(x2 - m0), p3 = ex2(x3 - m1);
+    l0 += p0 + p2;
+    l1 += p1 + p3;
+    const uint32_t pb0 = movmatrix_trans(pack2<BF16>(p0, p1));
+    const uint32_t pb1 = movmatrix_trans(pack2<BF16>(p2, p3));
+    // ---- O^T += V^T P^T
+    if constexpr (!FP8) {
+      if (valid == kBS) {
+#pragma unroll
+        for (int t = 0; t < NDT; ++t) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_trans(vb + tile_off(ri + ((mi >> 1) << 3), (16 * t + ((mi & 1) << 3)) * 2), a0, a1, a2, a3);
+          mma_16816<BF16>(o[t], a0, a1, a2, a3, pb0, pb1);
+        }
+      } else {  // zero V of tokens past the end (they may hold NaN/Inf)
+        const uint32_t mlo = (2 * c4 < valid ? 0x0000ffffu : 0u) | (2 * c4 + 1 < valid ? 0xffff0000u : 0u);
+        const uint32_t mhi = (2 * c4 + 8 < valid ? 0x0000ffffu : 0u) | (2 * c4 + 9 < valid ? 0xffff0000u : 0u);
+#pragma unroll
+        for (int t = 0; t < NDT; ++t) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_trans(vb + tile_off(ri + ((mi >> 1) << 3), (16 * t + ((mi & 1) << 3)) * 2), a0, a1, a2, a3);
+          mma_16816<BF16>(o[t], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, pb0, pb1);
+        }
+      }
+    } else {
+      // lane row gid owns dims [D/8*gid, D/8*gid + D/8) of tokens 2c4, 2c4+1, 2c4+8, 2c4+9;
+      // output tile t holds dims D/8*gid + 2t (MMA row gid) and +1 (row gid+8)
+      constexpr int LB = D / 8;
+      constexpr int LC = LB / 16;
+      uint4 vr[4][LC];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int row = 2 * c4 + (r & 1) + ((r >> 1) << 3);
+#pragma unroll
+        for (int u = 0; u < LC; ++u) vr[r][u] = lds128(vb + tile_off(row, LB * gid + 16 * u));
+      }
+      if (valid < kBS) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          const int row = 2 * c4 + (r & 1) + ((r >> 1) << 3);
+          if (row >= valid) {
+#pragma unroll
+            for (int u = 0; u < LC; ++u) vr[r][u] = make_uint4(0u, 0u, 0u, 0u);
+          }
+        }
+      }
+      const uint32_t* r0 = reinterpret_cast<const uint32_t*>(&vr[0][0]);
+      const uint32_t* r1 = reinterpret_cast<const uint32_t*>(&vr[1][0]);
+      const uint32_t* r2 = reinterpret_cast<const uint32_t*>(&vr[2][0]);
+      const uint32_t* r3 = reinterpret_cast<const uint32_t*>(&vr[3][0]);
+#pragma unroll
+      for (int w = 0; w < NDT / 2; ++w) {
+        uint32_t a0, a1, a2, a3;
+        // tile 2w: bytes 0,1 of word w; tile 2w+1: bytes 2,3
+        e4m3x4_to_f16x2x2(prmt(r0[w], r1[w], 0x5140u), a0, a1);
+        e4m3x4_to_f16x2x2(prmt(r2[w], r3[w], 0x5140u), a2, a3);
+        mma_16816<false>(o[2 * w], a0, a1, a2, a3, pb0, pb1);
+        e4m3x4_to_f16x2x2(prmt(r0[w], r1[w], 0x7362u), a0, a1);
+        e4m3x4_to_f16x2x2(prmt(r2[w], r3[w], 0x7362u), a2, a3);
+        mma_16816<false>(o[2 * w + 1], a0, a1, a2, a3, pb0, pb1);
+      }
+    }
+  }
+
+  // Full softmax sums of this lane's two columns (l summed over the 16 token rows).
+  __device__ __forceinline__ void totals(float& L0, float& L1) const {
+    L0 = l0;
+    L1 = l1;
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+      L0 += __shfl_xor_sync(0xffffffffu, L0, off);
+      L1 += __shfl_xor_sync(0xffffffffu, L1, off);
+    }
+  }
+
+  // Output dim of (tile t, MMA row half hi) for this lane: 16-bit path
+  // 16t + gid + 8hi; fp8 path D/8*gid + 2t + hi.
+  __device__ __forceinline__ static int dim(int t, int hi, int gid) {
+    if constexpr (!FP8) return 16 * t + gid + 8 * hi;
+    else return (D / 8) * gid + 2 * t + hi;
+  }
+};
+
 template <class C>
 __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                           const __grid_constant__ CUtensorMap tmV,
@@ -215,9 +455,10 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
       const int s = b + lane;
       if (s < S) {
         const int raw = p.seq_lens[s];
-        const int len = clamp_len(raw, p);
-        lens[s] = len;
+        int len = clamp_len(raw, p);
         bad |= raw != len;
+        if (p.seq_skip) len = max(0, len - p.seq_skip[s] * kBS);  // the private suffix
+        lens[s] = len;
         sum_len += len;
         min_len = min(min_len, len);
         max_len = max(max_len, len);
@@ -299,7 +540,7 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
     };
     // A work item: sequence, partition (piece) index and count, KV unit, block range.
     struct Item {
-      int s, y, part, np, len, b0, nb;
+      int s, y, part, np, len, b0, nb, off;  // off: table entries before the suffix
     };
     auto last_seq_at = [&](int v) {  // last s with prefix[s] <= v (skips empty sequences)
       int lo = 0, hi = S - 1;
@@ -321,6 +562,7 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
       const int nblk = (it.len + kBS - 1) / kBS;
       it.b0 = it.part * pb;
       it.nb = max(0, min(nblk, it.b0 + pb) - it.b0);
+      it.off = p.seq_skip ? __ldg(p.seq_skip + it.s) : 0;
       return it;
     };
     // stream-K mode: this CTA's KV unit of the sequence under global block g, up to `end`
@@ -336,6 +578,7 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
       const Pieces pc = unit_pieces(prefix[it.s], nblk, per_cta);
       it.part = sk_group - pc.c0;
       it.np = pc.count;
+      it.off = p.seq_skip ? __ldg(p.seq_skip + it.s) : 0;
       return it;
     };
     // Lane j's block-table entry of chunk c (blocks 32c + j) of an item; out-of-pool ids are flagged.
@@ -343,7 +586,7 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
       const int i = 32 * c + lane;
       int b = 0;
       if (i < it.nb) {
-        b = __ldg(p.block_tables + (size_t)it.s * p.bt_stride + it.b0 + i);
+        b = __ldg(p.block_tables + (size_t)it.s * p.bt_stride + it.off + it.b0 + i);
         if (b < 0 || b >= p.num_blocks) {
           atomicOr(p.err, kCheckBadBlock);
           b = 0;
@@ -477,10 +720,8 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
   } else {
     // ---------------------------------------------------------------- consumer
     const int gid = lane >> 2, c4 = lane & 3;
-    const int mi = lane >> 3, ri = lane & 7;
-    uint32_t qf[C::NKT][2];
-    float o[C::NDT][4];
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    WarpAttn<D, C::kFp8, C::kBf16> A;
+    A.reset();
     int stage_i = 0, item_i = 0;
     int cur_s = 0, cur_head0 = 0, cur_nheads = 0, cur_part = 0, cur_np = 1;
 
@@ -506,225 +747,49 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
           atomicOr(p.err, kCheckWaitTimeout);
           break;
         }
-        const uint8_t* qsm = smem + L.q + qs * p.q_slot_bytes + gid * D * 2;
-        const bool ok = gid < cur_nheads;
-#pragma unroll
-        for (int j = 0; j < C::NKT; ++j) {
-          if constexpr (!C::kFp8) {
-            qf[j][0] = ok ? *reinterpret_cast<const uint32_t*>(qsm + 2 * (16 * j + 2 * c4)) : 0u;
-            qf[j][1] = ok ? *reinterpret_cast<const uint32_t*>(qsm + 2 * (16 * j + 2 * c4 + 8)) : 0u;
-          } else {
-            // permuted contraction order: lane column c4 owns dims [D/4*c4, D/4*c4 + D/4)
-            const uint2 v = ok ? *reinterpret_cast<const uint2*>(qsm + 2 * ((D / 4) * c4 + 4 * j)) : make_uint2(0u, 0u);
-            qf[j][0] = v.x;
-            qf[j][1] = v.y;
-          }
-        }
+        A.load_q(gid < cur_nheads ? smem + L.q + qs * p.q_slot_bytes + gid * D * 2 : nullptr, c4);
         __syncwarp();
         if (lane == 0) mbar_arrive(qempty0 + 8 * qs);
         ++item_i;
-#pragma unroll
-        for (int t = 0; t < C::NDT; ++t) o[t][0] = o[t][1] = o[t][2] = o[t][3] = 0.f;
-        m0 = m1 = -INFINITY;
-        l0 = l1 = 0.f;
+        A.reset();
       }
       const int valid = (md.w >> 8) & 0xff;
       if (valid > 0) {
         const uint32_t kb = base_u32 + L.ring + st * C::STAGE_BYTES;
-        const uint32_t vb = kb + C::TILE_BYTES;
-        // ---- S^T = K Q^T
-        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
-        if constexpr (!C::kFp8) {
-#pragma unroll
-          for (int j = 0; j < C::NKT; ++j) {
-            const int tok = ri + ((mi & 1) << 3);
-            const int dim = 16 * j + ((mi >> 1) << 3);
-            uint32_t a0, a1, a2, a3;
-            ldsm_x4(kb + tile_off(tok, dim * 2), a0, a1, a2, a3);
-            if (j & 1)
-              mma_16816<C::kBf16>(sb, a0, a1, a2, a3, qf[j][0], qf[j][1]);
-            else
-              mma_16816<C::kBf16>(sa, a0, a1, a2, a3, qf[j][0], qf[j][1]);
-          }
-        } else {
-          constexpr int LB = D / 4;  // bytes of a K row owned by one lane
-          constexpr int LC = LB / 16;
-          uint4 kr[2][LC];
-#pragma unroll
-          for (int u = 0; u < LC; ++u) {
-            kr[0][u] = lds128(kb + tile_off(gid, LB * c4 + 16 * u));
-            kr[1][u] = lds128(kb + tile_off(gid + 8, LB * c4 + 16 * u));
-          }
-          const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&kr[0][0]);
-          const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&kr[1][0]);
-#pragma unroll
-          for (int j = 0; j < C::NKT; ++j) {
-            uint32_t a0, a1, a2, a3;
-            e4m3x4_to_f16x2x2(w0[j], a0, a2);
-            e4m3x4_to_f16x2x2(w1[j], a1, a3);
-            if (j & 1)
-              mma_16816<false>(sb, a0, a1, a2, a3, qf[j][0], qf[j][1]);
-            else
-              mma_16816<false>(sa, a0, a1, a2, a3, qf[j][0], qf[j][1]);
-          }
-        }
-        // ---- online softmax (log2 domain); rows of S^T are tokens gid, gid+8
-        const float sl = p.scale_log2;
-        const float x0 = gid < valid ? (sa[0] + sb[0]) * sl : -INFINITY;
-        const float x1 = gid < valid ? (sa[1] + sb[1]) * sl : -INFINITY;
-        const float x2 = gid + 8 < valid ? (sa[2] + sb[2]) * sl : -INFINITY;
-        const float x3 = gid + 8 < valid ? (sa[3] + sb[3]) * sl : -INFINITY;
-        float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-          bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
-          bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
-        }
-        // Lazy rescaling: the reference max only moves (and O, l are
-        // rescaled) when some head's block max exceeds it by more than
-        // 2^kLazy; otherwise weights up to 2^kLazy are accumulated as they are
-        // (exact in fp32, and well inside the 16-bit P range).
-        constexpr float kLazy = 8.f;
-        const bool grow = (bm0 > m0 + kLazy) || (bm1 > m1 + kLazy);
-        if (__any_sync(0xffffffffu, grow)) {
-          const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
-          const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
-          m0 = mn0;
-          m1 = mn1;
-          l0 *= al0;
-          l1 *= al1;
-#pragma unroll
-          for (int t = 0; t < C::NDT; ++t) {
-            o[t][0] *= al0;
-            o[t][1] *= al1;
-            o[t][2] *= al0;
-            o[t][3] *= al1;
-          }
-        }
-        const float p0 = ex2(x0 - m0), p1 = ex2(x1 - m1), p2 = ex2(x2 - m0), p3 = ex2(x3 - m1);
-        l0 += p0 + p2;
-        l1 += p1 + p3;
-        const uint32_t pb0 = movmatrix_trans(pack2<C::kBf16>(p0, p1));
-        const uint32_t pb1 = movmatrix_trans(pack2<C::kBf16>(p2, p3));
-        // ---- O^T += V^T P^T
-        if constexpr (!C::kFp8) {
-          if (valid == kBS) {
-#pragma unroll
-            for (int t = 0; t < C::NDT; ++t) {
-              uint32_t a0, a1, a2, a3;
-              ldsm_x4_trans(vb + tile_off(ri + ((mi >> 1) << 3), (16 * t + ((mi & 1) << 3)) * 2), a0, a1, a2, a3);
-              mma_16816<C::kBf16>(o[t], a0, a1, a2, a3, pb0, pb1);
-            }
-          } else {  // zero V of tokens past the end (they may hold NaN/Inf)
-            const uint32_t mlo = (2 * c4 < valid ? 0x0000ffffu : 0u) | (2 * c4 + 1 < valid ? 0xffff0000u : 0u);
-            const uint32_t mhi = (2 * c4 + 8 < valid ? 0x0000ffffu : 0u) | (2 * c4 + 9 < valid ? 0xffff0000u : 0u);
-#pragma unroll
-            for (int t = 0; t < C::NDT; ++t) {
-              uint32_t a0, a1, a2, a3;
-              ldsm_x4_trans(vb + tile_off(ri + ((mi >> 1) << 3), (16 * t + ((mi & 1) << 3)) * 2), a0, a1, a2, a3);
-              mma_16816<C::kBf16>(o[t], a0 & mlo, a1 & mlo, a2 & mhi, a3 & mhi, pb0, pb1);
-            }
-          }
-        } else {
-          // lane row gid owns dims [D/8*gid, D/8*gid + D/8) of tokens 2c4, 2c4+1, 2c4+8, 2c4+9;
-          // output tile t holds dims D/8*gid + 2t (MMA row gid) and +1 (row gid+8)
-          constexpr int LB = D / 8;
-          constexpr int LC = LB / 16;
-          uint4 vr[4][LC];
-#pragma unroll
-          for (int r = 0; r < 4; ++r) {
-            const int row = 2 * c4 + (r & 1) + ((r >> 1) << 3);
-#pragma unroll
-            for (int u = 0; u < LC; ++u) vr[r][u] = lds128(vb + tile_off(row, LB * gid + 16 * u));
-          }
-          if (valid < kBS) {
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-              const int row = 2 * c4 + (r & 1) + ((r >> 1) << 3);
-              if (row >= valid) {
-#pragma unroll
-                for (int u = 0; u < LC; ++u) vr[r][u] = make_uint4(0u, 0u, 0u, 0u);
-              }
-            }
-          }
-          const uint32_t* r0 = reinterpret_cast<const uint32_t*>(&vr[0][0]);
-          const uint32_t* r1 = reinterpret_cast<const uint32_t*>(&vr[1][0]);
-          const uint32_t* r2 = reinterpret_cast<const uint32_t*>(&vr[2][0]);
-          const uint32_t* r3 = reinterpret_cast<const uint32_t*>(&vr[3][0]);
-#pragma unroll
-          for (int w = 0; w < C::NDT / 2; ++w) {
-            uint32_t a0, a1, a2, a3;
-            // tile 2w: bytes 0,1 of word w; tile 2w+1: bytes 2,3
-            e4m3x4_to_f16x2x2(prmt(r0[w], r1[w], 0x5140u), a0, a1);
-            e4m3x4_to_f16x2x2(prmt(r2[w], r3[w], 0x5140u), a2, a3);
-            mma_16816<false>(o[2 * w], a0, a1, a2, a3, pb0, pb1);
-            e4m3x4_to_f16x2x2(prmt(r0[w], r1[w], 0x7362u), a0, a1);
-            e4m3x4_to_f16x2x2(prmt(r2[w], r3[w], 0x7362u), a2, a3);
-            mma_16816<false>(o[2 * w + 1], a0, a1, a2, a3, pb0, pb1);
-          }
-        }
+        A.block(kb, kb + C::TILE_BYTES, valid, p.scale_log2, lane);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty0 + 8 * st);
       ++stage_i;
 
       if (md.w & kLast) {
-        // ---- finish the item straight from registers: full l over the 16
-        // token rows; lane (gid, c4) holds heads 2c4, 2c4+1 of 2 dims per tile
-        float L0 = l0, L1 = l1;
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-          L0 += __shfl_xor_sync(0xffffffffu, L0, off);
-          L1 += __shfl_xor_sync(0xffffffffu, L1, off);
-        }
+        // ---- finish the item straight from registers; lane (gid, c4) holds
+        // heads 2c4, 2c4+1 of 2 dims per tile
+        float L0, L1;
+        A.totals(L0, L1);
         const int h0 = 2 * c4, h1 = 2 * c4 + 1;
         const float i0 = L0 > 0.f ? p.v_scale / L0 : 0.f;
         const float i1 = L1 > 0.f ? p.v_scale / L1 : 0.f;
         const bool ok0 = h0 < cur_nheads, ok1 = h1 < cur_nheads;
-        // output dims of (tile t, MMA row r): 16-bit path 16t + r; fp8 path D/8*gid + 2t (+1 for r >= 8)
-        auto dim = [&](int t, int hi) -> int {
-          if constexpr (!C::kFp8) return 16 * t + gid + 8 * hi;
-          else return (D / 8) * gid + 2 * t + hi;
-        };
-        if (cur_np == 1) {
+        if (cur_np == 1 && !p.force_partials) {
           Q* d0 = reinterpret_cast<Q*>(p.out) + ((size_t)cur_s * p.num_heads + cur_head0 + h0) * D;
           Q* d1 = d0 + D;
 #pragma unroll
           for (int t = 0; t < C::NDT; ++t) {
             if (ok0) {
-              d0[dim(t, 0)] = Q(o[t][0] * i0);
-              d0[dim(t, 1)] = Q(o[t][2] * i0);
+              d0[A.dim(t, 0, gid)] = Q(A.o[t][0] * i0);
+              d0[A.dim(t, 1, gid)] = Q(A.o[t][2] * i0);
             }
             if (ok1) {
-              d1[dim(t, 0)] = Q(o[t][1] * i1);
-              d1[dim(t, 1)] = Q(o[t][3] * i1);
+              d1[A.dim(t, 0, gid)] = Q(A.o[t][1] * i1);
+              d1[A.dim(t, 1, gid)] = Q(A.o[t][3] * i1);
             }
           }
         } else {
           const size_t row0 = ((size_t)cur_s * p.num_heads + cur_head0 + h0) * p.max_parts + cur_part;
           const size_t row1 = row0 + p.max_parts;
-          float* d0 = p.part_o + row0 * D;
-          float* d1 = p.part_o + row1 * D;
-#pragma unroll
-          for (int t = 0; t < C::NDT; ++t) {
-            if constexpr (!C::kFp8) {
-              if (ok0) {
-                d0[dim(t, 0)] = o[t][0] * i0;
-                d0[dim(t, 1)] = o[t][2] * i0;
-              }
-              if (ok1) {
-                d1[dim(t, 0)] = o[t][1] * i1;
-                d1[dim(t, 1)] = o[t][3] * i1;
-              }
-            } else {  // adjacent dims: one 8-byte store per head
-              if (ok0) *reinterpret_cast<float2*>(d0 + dim(t, 0)) = make_float2(o[t][0] * i0, o[t][2] * i0);
-              if (ok1) *reinterpret_cast<float2*>(d1 + dim(t, 0)) = make_float2(o[t][1] * i1, o[t][3] * i1);
-            }
-          }
-          if (gid == 0) {
-            if (ok0) *reinterpret_cast<float2*>(p.part_ml + row0 * 2) = make_float2(m0, L0);
-            if (ok1) *reinterpret_cast<float2*>(p.part_ml + row1 * 2) = make_float2(m1, L1);
-          }
+          store_partial<D, C::kFp8>(A.o, A.m0, L0, i0, ok0, A.m1, L1, i1, ok1, p.part_o, p.part_ml, row0, row1,
+                                    lane);
         }
       }
     }
@@ -746,12 +811,13 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
 // Log-sum-exp merge of split sequences.  A CTA of 256 threads covers
 // `merge_hpc` consecutive query heads of one sequence; its threads are
 // (head, partition slice, 4-dim chunk) triples, `merge_slices` slices taking
-// every merge_slices-th partition.  Warp n first finds head n's largest
-// partition max M and weight sum W; each thread then accumulates
-// l_p 2^(m_p - M) o_p over its partitions with 8 partitions' loads in flight,
-// and the slices are summed in shared memory.  Launched as a programmatic
-// dependent of the decode kernel: it may be scheduled early and waits for the
-// decode grid to finish before reading.
+// every merge_slices-th partial.  Warp n first finds head n's largest partial
+// max M and weight sum W; each thread then accumulates l_p 2^(m_p - M) o_p
+// over its partials with 8 partials' loads in flight, and the slices are
+// summed in shared memory.  A head's partials are the decode pass's np
+// partitions, followed, in shared-prefix decode, by the prefix pass's chunks.
+// Launched as a programmatic dependent of the decode kernel: it may be
+// scheduled early and waits for the decode grid to finish before reading.
 template <typename Q, int D, bool BF16>
 __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodeParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -763,37 +829,48 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
   const int hblocks = (p.num_heads + hpc - 1) / hpc;
   const int s = blockIdx.x / hblocks;
   const int h0 = (blockIdx.x - s * hblocks) * hpc;
-  const int len = clamp_len(p.seq_lens[s], p);
+  const bool shared = p.seq_skip != nullptr;
+  const int skip = shared ? p.seq_skip[s] : 0;
+  const int len = shared ? max(0, clamp_len(p.seq_lens[s], p) - skip * kBS) : clamp_len(p.seq_lens[s], p);
   const int nblk = (len + kBS - 1) / kBS;
+  const int nc = shared ? (skip + kPrefixChunkBlocks - 1) / kPrefixChunkBlocks : 0;  // prefix partials
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // the decode launch's hand-out: stream-K or tickets with pb blocks per partition
   const bool sk = p.auto_mode && p.counters[3] != 0;
   const int param = p.auto_mode ? p.counters[2] : p.partition_blocks;
-  // partitions of head h (the same for every head of a sequence)
-  auto parts_of = [&](int h) -> int {
-    (void)h;
-    if (!sk) return num_partitions(len, param, p);
-    if (nblk == 0) return 0;
-    return unit_pieces(p.seq_prefix[s], nblk, param).count;
-  };
-  if (sk && nblk == 0) {  // empty sequence: zero rows (no decode item covered it)
+  // decode-pass partitions (the same for every head of a sequence)
+  int np;
+  if (!sk) np = num_partitions(len, param, p);
+  else np = nblk == 0 ? 0 : unit_pieces(p.seq_prefix[s], nblk, param).count;
+  if (!shared && sk && nblk == 0) {  // empty sequence: zero rows (no decode item covered it)
     for (int i = threadIdx.x; i < hpc * D; i += blockDim.x) {
       const int h = h0 + i / D;
       if (h < p.num_heads) reinterpret_cast<Q*>(p.out)[((size_t)s * p.num_heads + h) * D + i % D] = Q(0.0f);
     }
     return;
   }
+  // without a prefix pass, a single partition was written by the decode kernel
+  const bool merged = shared || np > 1;
+  const int nt = np + nc;
+  if (!merged) return;
+  // partial q of head h: decode partition q < np, else prefix chunk q - np
+  auto ml_of = [&](int h, int q) -> const float* {
+    return q < np ? p.part_ml + (((size_t)s * p.num_heads + h) * p.max_parts + q) * 2
+                  : p.pre_ml + (((size_t)s * p.num_heads + h) * p.max_chunks + (q - np)) * 2;
+  };
+  auto o_of = [&](int h, int q) -> const float* {
+    return q < np ? p.part_o + (((size_t)s * p.num_heads + h) * p.max_parts + q) * D
+                  : p.pre_o + (((size_t)s * p.num_heads + h) * p.max_chunks + (q - np)) * D;
+  };
   if (warp < hpc) {
     const int h = h0 + warp;
-    const int np = h < p.num_heads ? parts_of(h) : 0;
     float M = -INFINITY, W = 0.f;
-    if (np > 1) {
-      const float* ml = p.part_ml + ((size_t)s * p.num_heads + h) * p.max_parts * 2;
-      for (int q = lane; q < np; q += 32) M = fmaxf(M, ml[2 * q]);
+    if (h < p.num_heads) {
+      for (int q = lane; q < nt; q += 32) M = fmaxf(M, ml_of(h, q)[0]);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-      for (int q = lane; q < np; q += 32) {
-        const float2 v = *reinterpret_cast<const float2*>(ml + 2 * q);
+      for (int q = lane; q < nt; q += 32) {
+        const float2 v = *reinterpret_cast<const float2*>(ml_of(h, q));
         if (v.y > 0.f) W += v.y * ex2(v.x - M);
       }
 #pragma unroll
@@ -802,7 +879,7 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
     if (lane == 0) {
       hM[warp] = M;
       hInvW[warp] = W > 0.f ? 1.f / W : 0.f;
-      hNp[warp] = np;
+      hNp[warp] = h < p.num_heads ? nt : 0;
     }
   }
   __syncthreads();
@@ -810,22 +887,19 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
   const int rest = threadIdx.x / CH;
   const int slice = rest % slices, hl = rest / slices;
   const int h = h0 + hl;
-  const int np = hl < hpc ? hNp[hl] : 0;  // <= 1: written by the decode kernel
+  const int nth = hl < hpc ? hNp[hl] : 0;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (np > 1) {
-    const size_t row0 = ((size_t)s * p.num_heads + h) * p.max_parts;
-    const float* ml = p.part_ml + row0 * 2;
-    const float* po = p.part_o + row0 * D + 4 * c;
+  if (nth > 0) {
     const float M = hM[hl];
-    for (int q0 = slice; q0 < np; q0 += 8 * slices) {
+    for (int q0 = slice; q0 < nth; q0 += 8 * slices) {
       float2 mlq[8];
       float4 v[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int q = q0 + u * slices;
-        const bool ok = q < np;
-        mlq[u] = ok ? *reinterpret_cast<const float2*>(ml + 2 * q) : make_float2(-INFINITY, 0.f);
-        v[u] = ok ? *reinterpret_cast<const float4*>(po + (size_t)q * D) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const bool ok = q < nth;
+        mlq[u] = ok ? *reinterpret_cast<const float2*>(ml_of(h, q)) : make_float2(-INFINITY, 0.f);
+        v[u] = ok ? *reinterpret_cast<const float4*>(o_of(h, q) + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -839,7 +913,7 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
   }
   red[threadIdx.x] = acc;
   __syncthreads();
-  if (slice == 0 && np > 1) {
+  if (slice == 0 && hl < hpc && h < p.num_heads) {
     for (int k = 1; k < slices; ++k) {
       const float4 o = red[threadIdx.x + k * CH];
       acc.x += o.x;
@@ -847,7 +921,7 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
       acc.z += o.z;
       acc.w += o.w;
     }
-    const float inv = hInvW[hl];
+    const float inv = hInvW[hl];  // 0 when no partial has weight: a zero row
     Q* dst = reinterpret_cast<Q*>(p.out) + ((size_t)s * p.num_heads + h) * D + 4 * c;
     *reinterpret_cast<uint2*>(dst) = make_uint2(pack2<BF16>(acc.x * inv, acc.y * inv), pack2<BF16>(acc.z * inv, acc.w * inv));
   }

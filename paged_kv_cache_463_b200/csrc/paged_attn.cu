@@ -15,6 +15,7 @@
 #include "paged_attn.h"
 #include "cache_ops.cuh"
 #include "decode.cuh"
+#include "prefix.cuh"
 
 #define PA_API extern "C" __attribute__((visibility("default")))
 
@@ -26,21 +27,26 @@ using pa::DecodeParams;
 struct KernelSet {
   const void* decode = nullptr;
   const void* merge = nullptr;
+  const void* prefix = nullptr;  // shared-prefix pass
   int threads = 0;
   int ns = 0, stage_bytes = 0;  // ring shape (the rest of the layout depends on the call)
+  int prefix_threads = 0, prefix_smem = 0;
   size_t smem(int q_slot_bytes, int max_seqs) const {
     return pa::DecodeLayout(ns, stage_bytes, q_slot_bytes).bytes(max_seqs);
   }
 };
 
-template <class C>
+template <class C, class P>
 KernelSet make_set() {
   KernelSet k;
   k.decode = reinterpret_cast<const void*>(&pa::paged_decode_kernel<C>);
   k.merge = reinterpret_cast<const void*>(&pa::paged_decode_merge_kernel<typename C::Q, C::D, C::kBf16>);
+  k.prefix = reinterpret_cast<const void*>(&pa::paged_prefix_kernel<P>);
   k.threads = C::THREADS;
   k.ns = C::NS;
   k.stage_bytes = C::STAGE_BYTES;
+  k.prefix_threads = P::THREADS;
+  k.prefix_smem = P::SMEM_BYTES;
   return k;
 }
 
@@ -52,7 +58,7 @@ cudaError_t pin_carveout(const void* fn) {
 }
 
 cudaError_t pin_all_carveouts(const KernelSet& ks) {
-  const void* fns[] = {ks.decode, ks.merge, reinterpret_cast<const void*>(&pa::reshape_and_cache_copy_kernel),
+  const void* fns[] = {ks.decode, ks.merge, ks.prefix, reinterpret_cast<const void*>(&pa::reshape_and_cache_copy_kernel),
                        reinterpret_cast<const void*>(&pa::reshape_and_cache_fp8_kernel<true>),
                        reinterpret_cast<const void*>(&pa::reshape_and_cache_fp8_kernel<false>),
                        reinterpret_cast<const void*>(&pa::paged_gather_kernel),
@@ -131,17 +137,42 @@ struct Tuned;
 #ifndef PA_MIN_CTAS_FP8_128
 #define PA_MIN_CTAS_FP8_128 8
 #endif
-template <> struct Tuned<64, __half, __half> { using C = DecodeCfg<64, __half, __half, PA_NS_16B_64, 8>; };
-template <> struct Tuned<128, __half, __half> { using C = DecodeCfg<128, __half, __half, PA_NS_16B_128, 8>; };
-template <> struct Tuned<256, __half, __half> { using C = DecodeCfg<256, __half, __half, PA_NS_16B_256, 3>; };
-template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<64, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_64, 8>; };
-template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128, 8>; };
-template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> { using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_256, 3>; };
-template <> struct Tuned<128, __nv_fp8_e4m3, __half> { using C = DecodeCfg<128, __nv_fp8_e4m3, __half, PA_NS_FP8_128, PA_MIN_CTAS_FP8_128>; };
-template <> struct Tuned<256, __nv_fp8_e4m3, __half> { using C = DecodeCfg<256, __nv_fp8_e4m3, __half, PA_NS_FP8_256, 4>; };
+// The shared-prefix pass's ring: 32-64 KiB of K/V in flight per CTA.
+template <> struct Tuned<64, __half, __half> {
+  using C = DecodeCfg<64, __half, __half, PA_NS_16B_64, 8>;
+  using P = pa::PrefixCfg<64, __half, __half, 8>;
+};
+template <> struct Tuned<128, __half, __half> {
+  using C = DecodeCfg<128, __half, __half, PA_NS_16B_128, 8>;
+  using P = pa::PrefixCfg<128, __half, __half, 6>;
+};
+template <> struct Tuned<256, __half, __half> {
+  using C = DecodeCfg<256, __half, __half, PA_NS_16B_256, 3>;
+  using P = pa::PrefixCfg<256, __half, __half, 4>;
+};
+template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> {
+  using C = DecodeCfg<64, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_64, 8>;
+  using P = pa::PrefixCfg<64, __nv_bfloat16, __nv_bfloat16, 8>;
+};
+template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> {
+  using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128, 8>;
+  using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, 6>;
+};
+template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> {
+  using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_256, 3>;
+  using P = pa::PrefixCfg<256, __nv_bfloat16, __nv_bfloat16, 4>;
+};
+template <> struct Tuned<128, __nv_fp8_e4m3, __half> {
+  using C = DecodeCfg<128, __nv_fp8_e4m3, __half, PA_NS_FP8_128, PA_MIN_CTAS_FP8_128>;
+  using P = pa::PrefixCfg<128, __nv_fp8_e4m3, __half, 8>;
+};
+template <> struct Tuned<256, __nv_fp8_e4m3, __half> {
+  using C = DecodeCfg<256, __nv_fp8_e4m3, __half, PA_NS_FP8_256, 4>;
+  using P = pa::PrefixCfg<256, __nv_fp8_e4m3, __half, 6>;
+};
 
 bool select_kernels(int head_dim, int q_dtype, int kv_dtype, KernelSet* ks) {
-#define PA_CASE(D, KVT, QT) *ks = make_set<typename Tuned<D, KVT, QT>::C>(); return true
+#define PA_CASE(D, KVT, QT) *ks = make_set<typename Tuned<D, KVT, QT>::C, typename Tuned<D, KVT, QT>::P>(); return true
   if (kv_dtype == PA_F16 && q_dtype == PA_F16) {
     if (head_dim == 64) { PA_CASE(64, __half, __half); }
     if (head_dim == 128) { PA_CASE(128, __half, __half); }
@@ -188,6 +219,11 @@ struct pa_ctx {
   float* part_ml = nullptr;
   int* err = nullptr;           // [0] check word, [1..4] decode kernel counters (DecodeParams::counters)
   int* seq_prefix = nullptr;    // [max_num_seqs + 1] stream-K block offsets (decode -> merge)
+  // shared-prefix decode (PA_FLAG_SHARED_PREFIX)
+  int max_chunks = 0;           // prefix partials per (seq, head)
+  float* pre_o = nullptr;
+  float* pre_ml = nullptr;
+  int* seq_skip = nullptr;      // [max_num_seqs] prefix blocks per sequence (prefix pass -> decode, merge)
   int* err_host = nullptr;      // pinned
   int grid = 0;                 // persistent grid: SMs x resident CTAs
   int last_bits = 0;
@@ -269,7 +305,8 @@ PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
   if (!cfg) return PA_ERR_INVALID_ARG;
   const pa_config c = *cfg;
   if (c.num_heads <= 0 || c.num_kv_heads <= 0 || c.num_heads % c.num_kv_heads != 0 || c.num_blocks <= 0 ||
-      c.max_num_seqs <= 0 || c.max_blocks_per_seq <= 0 || c.flags != 0 || c.device < 0)
+      c.max_num_seqs <= 0 || c.max_blocks_per_seq <= 0 || (c.flags & ~PA_FLAG_SHARED_PREFIX) != 0 ||
+      c.device < 0)
     return PA_ERR_INVALID_ARG;
   if (c.block_size != pa::kBS) return PA_ERR_UNSUPPORTED;
   if ((long long)c.num_blocks * c.block_size > 0x7fffffffLL) return PA_ERR_INVALID_ARG;
@@ -312,6 +349,8 @@ PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
       break;
     }
     if ((e = cudaFuncSetAttribute(ks.decode, cudaFuncAttributeMaxDynamicSharedMemorySize, optin)) != cudaSuccess ||
+        (e = cudaFuncSetAttribute(ks.prefix, cudaFuncAttributeMaxDynamicSharedMemorySize, ks.prefix_smem)) !=
+            cudaSuccess ||
         (e = pin_all_carveouts(ks)) != cudaSuccess) {
       st = cuda_fail(ctx, e, "cudaFuncSetAttribute");
       break;
@@ -339,6 +378,17 @@ PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
       break;
     }
 
+    if (c.flags & PA_FLAG_SHARED_PREFIX) {
+      ctx->max_chunks = (c.max_blocks_per_seq + pa::kPrefixChunkBlocks - 1) / pa::kPrefixChunkBlocks;
+      const size_t prow = (size_t)c.max_num_seqs * c.num_heads * ctx->max_chunks;
+      if (cudaMalloc(&ctx->pre_o, prow * c.head_dim * sizeof(float)) != cudaSuccess ||
+          cudaMalloc(&ctx->pre_ml, prow * 2 * sizeof(float)) != cudaSuccess ||
+          cudaMalloc(&ctx->seq_skip, c.max_num_seqs * sizeof(int)) != cudaSuccess) {
+        cudaGetLastError();
+        st = PA_ERR_NO_MEMORY;
+        break;
+      }
+    }
     if ((e = cudaMalloc(&ctx->err, 8 * sizeof(int))) != cudaSuccess ||
         (e = cudaMemset(ctx->err, 0, 8 * sizeof(int))) != cudaSuccess) {
       st = cuda_fail(ctx, e, "cudaMalloc(check word)");
@@ -364,6 +414,9 @@ PA_API int paged_attn_destroy(pa_ctx* ctx) {
   if (ctx->part_ml) cudaFree(ctx->part_ml);
   if (ctx->err) cudaFree(ctx->err);
   if (ctx->seq_prefix) cudaFree(ctx->seq_prefix);
+  if (ctx->pre_o) cudaFree(ctx->pre_o);
+  if (ctx->pre_ml) cudaFree(ctx->pre_ml);
+  if (ctx->seq_skip) cudaFree(ctx->seq_skip);
   if (ctx->err_host) cudaFreeHost(ctx->err_host);
   delete ctx;
   return PA_OK;
@@ -438,10 +491,18 @@ PA_API int reshape_and_cache(pa_ctx* ctx, const void* key, const void* value, in
   return e == cudaSuccess ? PA_OK : cuda_fail(ctx, e, "reshape_and_cache launch");
 }
 
-PA_API int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, const void* key_cache,
-                                  const void* value_cache, const int32_t* block_tables, int bt_stride,
-                                  const int32_t* seq_lens, int num_seqs, int max_seq_len, float scale,
-                                  float k_scale, float v_scale, void* stream) {
+namespace {
+
+// The shared-prefix part of a decode call (absent for plain decode).
+struct PrefixArgs {
+  const int32_t* group_start;
+  const int32_t* group_prefix_len;
+  int num_groups, max_group_size, max_prefix_len;
+};
+
+int decode_impl(pa_ctx* ctx, void* out, const void* query, const void* key_cache, const void* value_cache,
+                const int32_t* block_tables, int bt_stride, const int32_t* seq_lens, int num_seqs, int max_seq_len,
+                float scale, float k_scale, float v_scale, void* stream, const PrefixArgs* pre) {
   if (!ctx) return PA_ERR_INVALID_ARG;
   const pa_config& c = ctx->cfg;
   if (num_seqs < 0 || num_seqs > c.max_num_seqs) return fail(ctx, PA_ERR_INVALID_ARG, "num_seqs out of range");
@@ -458,17 +519,72 @@ PA_API int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, con
   const bool fp8 = c.kv_dtype == PA_FP8_E4M3;
   if (fp8 && !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
     return fail(ctx, PA_ERR_INVALID_ARG, "fp8 scales must be finite and > 0");
+  const int group = c.num_heads / c.num_kv_heads;
+  const int head_splits = (group + pa::kNH - 1) / pa::kNH;
+  const int kv_units = c.num_kv_heads * head_splits;
+  int prefix_chunks = 0, row_blocks = 0;
+  if (pre) {
+    if (!(c.flags & PA_FLAG_SHARED_PREFIX))
+      return fail(ctx, PA_ERR_UNSUPPORTED, "context created without PA_FLAG_SHARED_PREFIX");
+    if (!pre->group_start || !pre->group_prefix_len) return fail(ctx, PA_ERR_INVALID_ARG, "null pointer");
+    if (!aligned(pre->group_start, 4) || !aligned(pre->group_prefix_len, 4))
+      return fail(ctx, PA_ERR_INVALID_ARG, "misaligned pointer");
+    if (pre->num_groups < 1 || pre->num_groups > num_seqs || pre->num_groups > 65535)
+      return fail(ctx, PA_ERR_INVALID_ARG, "num_groups outside [1, num_seqs]");
+    if (pre->max_group_size < 1 || pre->max_group_size > num_seqs)
+      return fail(ctx, PA_ERR_INVALID_ARG, "max_group_size outside [1, num_seqs]");
+    if (pre->max_prefix_len < 0 || pre->max_prefix_len > max_seq_len)
+      return fail(ctx, PA_ERR_INVALID_ARG, "max_prefix_len outside [0, max_seq_len]");
+    const int pblocks = pre->max_prefix_len / c.block_size;
+    prefix_chunks = (pblocks + pa::kPrefixChunkBlocks - 1) / pa::kPrefixChunkBlocks;
+    const int rows_per_unit = pre->max_group_size * (group < pa::kNH ? group : pa::kNH);
+    row_blocks = (rows_per_unit + pa::kPrefixRows - 1) / pa::kPrefixRows;
+    if ((long long)kv_units * row_blocks > 65535)
+      return fail(ctx, PA_ERR_UNSUPPORTED, "max_group_size too large for the prefix grid");
+  }
   cudaSetDevice(ctx->device);
 
   CUtensorMap mk, mv;
   int st = tensor_map(ctx, key_cache, &mk);
   if (st != PA_OK) return st;
   if ((st = tensor_map(ctx, value_cache, &mv)) != PA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  if (pre) {  // shared blocks first: their partials, and each sequence's suffix offset
+    pa::PrefixParams q;
+    q.query = query;
+    q.block_tables = block_tables;
+    q.seq_lens = seq_lens;
+    q.group_start = pre->group_start;
+    q.group_prefix_len = pre->group_prefix_len;
+    q.pre_o = ctx->pre_o;
+    q.pre_ml = ctx->pre_ml;
+    q.seq_skip = ctx->seq_skip;
+    q.err = ctx->err;
+    q.num_seqs = num_seqs;
+    q.num_groups = pre->num_groups;
+    q.max_group_size = pre->max_group_size;
+    q.max_prefix_blocks = pre->max_prefix_len / c.block_size;
+    q.bt_stride = bt_stride;
+    q.num_heads = c.num_heads;
+    q.group = group;
+    q.head_splits = head_splits;
+    q.num_blocks = c.num_blocks;
+    q.max_blocks = max_seq_len > 0 ? (max_seq_len + c.block_size - 1) / c.block_size : 1;
+    q.max_chunks = ctx->max_chunks;
+    q.row_blocks = row_blocks;
+    q.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
+    q.v_scale = fp8 ? v_scale : 1.0f;
+    void* qargs[] = {&mk, &mv, &q};
+    const dim3 grid((unsigned)(prefix_chunks > 0 ? prefix_chunks : 1), (unsigned)(kv_units * row_blocks),
+                    (unsigned)pre->num_groups);
+    cudaError_t e = cudaLaunchKernel(ctx->ks.prefix, grid, dim3(ctx->ks.prefix_threads), qargs,
+                                     ctx->ks.prefix_smem, s);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "prefix launch");
+  }
 
   // PA_PARTITION_AUTO: stream-K ranges (the split follows from the balance);
   // otherwise fixed partitions handed out by tickets
-  const int group = c.num_heads / c.num_kv_heads;
-  const int kv_units = c.num_kv_heads * ((group + pa::kNH - 1) / pa::kNH);
   const bool is_auto = ctx->partition_tokens == PA_PARTITION_AUTO;
   const int max_blocks = (max_seq_len + c.block_size - 1) / c.block_size;
   // auto: the device picks tickets (partitions >= min_partition_tokens) or
@@ -499,12 +615,13 @@ PA_API int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, con
   p.num_seqs = num_seqs;
   p.bt_stride = bt_stride;
   p.num_heads = c.num_heads;
-  p.group = c.num_heads / c.num_kv_heads;
-  p.head_splits = (p.group + pa::kNH - 1) / pa::kNH;
-  p.kv_units = c.num_kv_heads * p.head_splits;
+  p.group = group;
+  p.head_splits = head_splits;
+  p.kv_units = kv_units;
   p.q_slot_bytes = q_slot_bytes(c.num_heads, c.num_kv_heads, c.head_dim);
   p.num_blocks = c.num_blocks;
   p.max_blocks = max_blocks > 0 ? max_blocks : 1;
+  p.force_partials = pre ? 1 : 0;
   p.partition_blocks = part_blocks;
   p.auto_mode = is_auto ? 1 : 0;
   p.min_piece_blocks = kMinPieceBlocks;
@@ -512,16 +629,43 @@ PA_API int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, con
   p.max_parts = ctx->max_parts;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
   p.v_scale = fp8 ? v_scale : 1.0f;
+  if (pre) {
+    p.seq_skip = ctx->seq_skip;
+    p.pre_o = ctx->pre_o;
+    p.pre_ml = ctx->pre_ml;
+    p.max_chunks = ctx->max_chunks;
+  }
 
-  merge_shape(c.head_dim, parts, c.num_heads, &p.merge_hpc, &p.merge_slices);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  merge_shape(c.head_dim, parts + prefix_chunks, c.num_heads, &p.merge_hpc, &p.merge_slices);
   void* args[] = {&mk, &mv, &p};
   cudaError_t e = cudaLaunchKernel(ctx->ks.decode, dim3(ctx->grid), dim3(ctx->ks.threads), args,
                                    ctx->ks.smem(q_slot_bytes(c.num_heads, c.num_kv_heads, c.head_dim), c.max_num_seqs), s);
   if (e != cudaSuccess) return cuda_fail(ctx, e, "decode launch");
-  if ((is_auto || parts > 1) && (e = launch_merge(ctx->ks, p, s)) != cudaSuccess)
+  if ((pre || is_auto || parts > 1) && (e = launch_merge(ctx->ks, p, s)) != cudaSuccess)
     return cuda_fail(ctx, e, "merge launch");
   return PA_OK;
+}
+
+}  // namespace
+
+PA_API int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, const void* key_cache,
+                                  const void* value_cache, const int32_t* block_tables, int bt_stride,
+                                  const int32_t* seq_lens, int num_seqs, int max_seq_len, float scale,
+                                  float k_scale, float v_scale, void* stream) {
+  return decode_impl(ctx, out, query, key_cache, value_cache, block_tables, bt_stride, seq_lens, num_seqs,
+                     max_seq_len, scale, k_scale, v_scale, stream, nullptr);
+}
+
+PA_API int paged_attention_decode_shared_prefix(pa_ctx* ctx, void* out, const void* query, const void* key_cache,
+                                                const void* value_cache, const int32_t* block_tables,
+                                                int bt_stride, const int32_t* seq_lens, int num_seqs,
+                                                int max_seq_len, const int32_t* group_start,
+                                                const int32_t* group_prefix_len, int num_groups,
+                                                int max_group_size, int max_prefix_len, float scale,
+                                                float k_scale, float v_scale, void* stream) {
+  const PrefixArgs pre = {group_start, group_prefix_len, num_groups, max_group_size, max_prefix_len};
+  return decode_impl(ctx, out, query, key_cache, value_cache, block_tables, bt_stride, seq_lens, num_seqs,
+                     max_seq_len, scale, k_scale, v_scale, stream, &pre);
 }
 
 PA_API int paged_attn_get_error(pa_ctx* ctx, void* stream) {
@@ -735,6 +879,7 @@ PA_API int paged_attention_decode_noalloc(void* out, const void* query, const vo
   p.q_slot_bytes = q_slot_bytes(num_heads, num_kv_heads, head_dim);
   p.num_blocks = num_blocks;
   p.max_blocks = max_blocks > 0 ? max_blocks : 1;
+  p.force_partials = 0;
   p.partition_blocks = part_blocks;
   p.auto_mode = 0;
   p.min_piece_blocks = kMinPieceBlocks;

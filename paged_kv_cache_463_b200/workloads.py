@@ -135,6 +135,8 @@ class Workload:
     scale: float = 1.0
     ref_counts: list[int] = field(default_factory=list)
     num_blocks: int = 0
+    group_start: torch.Tensor | None = None       # [G + 1] int32: group g = sequences [start[g], start[g+1])
+    group_prefix_len: torch.Tensor | None = None  # [G] int32: tokens the group's sequences share
 
     @property
     def max_seq_len(self) -> int:
@@ -164,6 +166,8 @@ class Layout:
     slot_mapping: list[int]
     ref_counts: list[int]
     num_blocks: int
+    group_start: list[int] = field(default_factory=list)  # prefix groups: [G + 1] sequence ranges
+    group_prefix_len: list[int] = field(default_factory=list)  # [G] shared tokens (whole blocks)
 
 
 def build_layout(spec: WorkloadSpec, seq_lens: list[int] | None = None) -> Layout:
@@ -213,7 +217,11 @@ def build_layout(spec: WorkloadSpec, seq_lens: list[int] | None = None) -> Layou
             tables[s, :nblk] = torch.tensor(row, dtype=torch.int32)
         last = n - 1
         slots.append(row[last // bs] * bs + last % bs if n > 0 else -1)
-    return Layout(lens, tables, slots, alloc.ref_counts, pool)
+    group_start, group_prefix_len = [], []
+    if groups:
+        group_start = [0] + [next((s for s in range(S) if s * groups // S > g), S) for g in range(groups)]
+        group_prefix_len = [prefix_blocks * bs] * groups
+    return Layout(lens, tables, slots, alloc.ref_counts, pool, group_start, group_prefix_len)
 
 
 def make_workload(spec: WorkloadSpec, device="cpu", seq_lens: list[int] | None = None) -> Workload:
@@ -234,6 +242,9 @@ def make_workload(spec: WorkloadSpec, device="cpu", seq_lens: list[int] | None =
                  query=query, new_key=new_key, new_value=new_value,
                  key_cache=None, value_cache=None, scale=1.0 / math.sqrt(D),
                  ref_counts=lay.ref_counts, num_blocks=pool)
+    if lay.group_start:
+        w.group_start = torch.tensor(lay.group_start, dtype=torch.int32).to(device)
+        w.group_prefix_len = torch.tensor(lay.group_prefix_len, dtype=torch.int32).to(device)
     if spec.kv_dtype == "fp8_e4m3":
         w.key_src = _randn_pool(shape, qdt, dgen, device)
         w.value_src = _randn_pool(shape, qdt, dgen, device)
@@ -262,3 +273,24 @@ def decode_bytes(w: Workload) -> int:
     qb = 2
     S = int(w.seq_lens.numel())
     return kv_read_bytes(w.seq_lens.cpu(), sp.num_kv_heads, sp.head_dim, kvb) + S * sp.num_heads * sp.head_dim * 2 * qb
+
+
+def shared_decode_bytes(w: Workload) -> int:
+    """Algorithmic bytes of one decode call that reads every shared prefix
+    block once per group: the groups' prefixes, every sequence's private
+    suffix, plus q read and out write."""
+    sp = w.spec
+    if w.group_start is None:
+        return decode_bytes(w)
+    kvb = 1 if sp.kv_dtype == "fp8_e4m3" else 2
+    per_token = sp.num_kv_heads * sp.head_dim * 2 * kvb
+    starts = w.group_start.cpu().tolist()
+    plen = w.group_prefix_len.cpu().tolist()
+    lens = w.seq_lens.cpu().tolist()
+    skip = [0] * len(lens)
+    for g, n in enumerate(plen):
+        for s in range(starts[g], starts[g + 1]):
+            skip[s] = n
+    tokens = sum(plen) + sum(max(0, n - k) for n, k in zip(lens, skip))
+    S = len(lens)
+    return tokens * per_token + S * sp.num_heads * sp.head_dim * 2 * 2

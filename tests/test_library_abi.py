@@ -48,7 +48,7 @@ def _create(lib, **kw):
     (dict(num_heads=0), b.PA_ERR_INVALID_ARG),
     (dict(num_blocks=0), b.PA_ERR_INVALID_ARG),
     (dict(max_num_seqs=0), b.PA_ERR_INVALID_ARG),
-    (dict(flags=1), b.PA_ERR_INVALID_ARG),
+    (dict(flags=2), b.PA_ERR_INVALID_ARG),              # unknown flag bit
     (dict(partition_tokens=100), b.PA_ERR_INVALID_ARG),   # not a block multiple
     (dict(partition_tokens=-2), b.PA_ERR_INVALID_ARG),
     (dict(block_size=32), b.PA_ERR_UNSUPPORTED),
