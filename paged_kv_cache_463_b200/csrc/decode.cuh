@@ -748,6 +748,9 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
           break;
         }
         A.load_q(gid < cur_nheads ? smem + L.q + qs * p.q_slot_bytes + gid * D * 2 : nullptr, c4);
+        // the slot's next writer is a bulk copy (async proxy): order these
+        // generic-proxy reads before it
+        fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(qempty0 + 8 * qs);
         ++item_i;
@@ -758,6 +761,7 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
         const uint32_t kb = base_u32 + L.ring + st * C::STAGE_BYTES;
         A.block(kb, kb + C::TILE_BYTES, valid, p.scale_log2, lane);
       }
+      fence_proxy_async_smem();  // (the stage's next writer is TMA)
       __syncwarp();
       if (lane == 0) mbar_arrive(empty0 + 8 * st);
       ++stage_i;

@@ -137,18 +137,18 @@ struct Tuned;
 #ifndef PA_MIN_CTAS_FP8_128
 #define PA_MIN_CTAS_FP8_128 8
 #endif
-// The shared-prefix pass's ring: 32-64 KiB of K/V in flight per CTA.
+// The shared-prefix pass's ring: 24-48 KiB of K/V in flight per CTA.
 template <> struct Tuned<64, __half, __half> {
   using C = DecodeCfg<64, __half, __half, PA_NS_16B_64, 8>;
   using P = pa::PrefixCfg<64, __half, __half, 8>;
 };
 template <> struct Tuned<128, __half, __half> {
   using C = DecodeCfg<128, __half, __half, PA_NS_16B_128, 8>;
-  using P = pa::PrefixCfg<128, __half, __half, 6>;
+  using P = pa::PrefixCfg<128, __half, __half, 4>;
 };
 template <> struct Tuned<256, __half, __half> {
   using C = DecodeCfg<256, __half, __half, PA_NS_16B_256, 3>;
-  using P = pa::PrefixCfg<256, __half, __half, 4>;
+  using P = pa::PrefixCfg<256, __half, __half, 3>;
 };
 template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<64, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_64, 8>;
@@ -156,19 +156,19 @@ template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> {
 };
 template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128, 8>;
-  using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, 6>;
+  using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, 4>;
 };
 template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_256, 3>;
-  using P = pa::PrefixCfg<256, __nv_bfloat16, __nv_bfloat16, 4>;
+  using P = pa::PrefixCfg<256, __nv_bfloat16, __nv_bfloat16, 3>;
 };
 template <> struct Tuned<128, __nv_fp8_e4m3, __half> {
   using C = DecodeCfg<128, __nv_fp8_e4m3, __half, PA_NS_FP8_128, PA_MIN_CTAS_FP8_128>;
-  using P = pa::PrefixCfg<128, __nv_fp8_e4m3, __half, 8>;
+  using P = pa::PrefixCfg<128, __nv_fp8_e4m3, __half, 6>;
 };
 template <> struct Tuned<256, __nv_fp8_e4m3, __half> {
   using C = DecodeCfg<256, __nv_fp8_e4m3, __half, PA_NS_FP8_256, 4>;
-  using P = pa::PrefixCfg<256, __nv_fp8_e4m3, __half, 6>;
+  using P = pa::PrefixCfg<256, __nv_fp8_e4m3, __half, 4>;
 };
 
 bool select_kernels(int head_dim, int q_dtype, int kv_dtype, KernelSet* ks) {

@@ -3,24 +3,32 @@
 // Sequences forked from one prompt share the physical blocks of that prompt
 // (page "5.KV Cache 管理 & PagedAttention", Q18 fork: the child's block table
 // is a copy of the parent's and every shared block's reference count goes up;
-// Q20 / page "paged-attention-and-vllm-inference", PrefixCacheManager: a
-// cached prefix's blocks are reused by later requests).  Attention over a
-// shared block is the same K/V against each member's query, so this pass loads
-// every shared block once and scores it for all members at once; the members'
+// page "paged-attention-and-vllm-inference", prefix caching: a cached
+// prefix's blocks are reused by later requests).  Attention over a shared
+// block is the same K/V against each member's query, so this pass loads every
+// shared block once and scores it for all members at once; the members'
 // private suffixes go through the regular decode kernel, and the merge kernel
 // combines the two sets of (o, m, l) partials by log-sum-exp.
 //
-// Work: one CTA per (group, KV unit, 64 query rows, chunk of 32 prefix blocks).
-// Query rows are (member sequence, query head of the unit) pairs, 8 per
-// consumer warp (the MMA N), so one K/V tile feeds 64 rows.  Warp 0 streams
-// the chunk's K/V tiles with TMA into an NS-stage ring (read from the group's
-// first member's block table); warps 1..8 consume every stage (empty barrier
-// count 8).  An fp8 E4M3 tile is converted once per block, by all 256 consumer
-// threads, into a double-buffered f16 tile in the same 128-byte-swizzled
-// layout, so that the 8 warps use the 16-bit MMA path on it.
+// With all members' query heads of one KV head stacked, a block is a dense
+// contraction: S[128 rows x 16 tokens] = Q K^T, then O[128 x D] += P V.  Both
+// run on the 5th-generation tensor cores (tcgen05.mma, issued by one thread,
+// accumulators in tensor memory), one CTA per (group, KV unit, 128 query
+// rows, chunk of 32 prefix blocks):
+//   warp 8      TMA producer: K/V tiles of the chunk's blocks into an NS-stage ring;
+//   warps 4..7  stage the MMA operands of each block: K as a 16-bit 128-byte-
+//               swizzled tile (fp8 E4M3 codes converted to f16), V transposed
+//               to V^T (tokens contiguous), double-buffered;
+//   warp 9      issues S_i = Q K_i^T into one of two TMEM S buffers, and
+//               O += P_{i-1} V_{i-1} once P_{i-1} is ready;
+//   warps 0..3  one query row per thread: read S_i from TMEM, online softmax
+//               in the log2 domain (lazy: O is rescaled in TMEM only when a
+//               row's maximum grows by more than 2^8), write P_i (16-bit) to
+//               shared memory; at the end read O, normalise, store partials.
 #pragma once
 
 #include "decode.cuh"
+#include "umma.cuh"
 
 namespace pa {
 
@@ -52,8 +60,10 @@ struct PrefixParams {
   float v_scale;
 };
 
-constexpr int kPrefixWarps = 8;                    // consumer warps
-constexpr int kPrefixRows = kPrefixWarps * kNH;    // query rows per CTA
+constexpr int kPrefixRows = 128;  // query rows per CTA (the MMA M)
+
+// Shared memory per SM and the per-CTA reservation, for capping residency.
+constexpr int kSmemPerSM = 233472;
 
 template <int D_, typename KV_, typename Q_, int NS_>
 struct PrefixCfg {
@@ -67,14 +77,32 @@ struct PrefixCfg {
   static constexpr int SUBTILES = ROW_BYTES / 128;
   static constexpr int TILE_BYTES = kBS * ROW_BYTES;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int F16_TILE = kBS * D * 2;      // converted tile (fp8 only)
-  static constexpr int THREADS = 32 * (1 + kPrefixWarps);
-  static constexpr int OFF_RING = 0;
-  static constexpr int OFF_CONV = NS * STAGE_BYTES;                  // 2 x (K, V) f16 tiles
-  static constexpr int OFF_BAR = OFF_CONV + (kFp8 ? 4 * F16_TILE : 0);
-  static constexpr int SMEM_BYTES = 1024 + OFF_BAR + 2 * NS * 8;
+  static constexpr int Q_BYTES = kPrefixRows * D * 2;  // 128-byte swizzled, D/64 sub-tiles of 16 KB
+  static constexpr int KF_BYTES = kBS * D * 2;         // 16-bit K tile, D/64 sub-tiles of 2 KB
+  static constexpr int VT_BYTES = D * kBS * 2;         // V^T, no swizzle
+  static constexpr int P_BYTES = kPrefixRows * kBS * 2;
+  static constexpr int OFF_Q = 0;
+  static constexpr int OFF_RING = OFF_Q + Q_BYTES;
+  static constexpr int OFF_KF = OFF_RING + NS * STAGE_BYTES;  // [2]
+  static constexpr int OFF_VT = OFF_KF + 2 * KF_BYTES;        // [2]
+  static constexpr int OFF_P = OFF_VT + 2 * VT_BYTES;         // [2]
+  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
+  // full[NS] empty[NS] conv_full[2] s_full[2] p_full[2] pv_done[2] fin
+  static constexpr int NBARS = 2 * NS + 9;
+  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem base, dead flag, blocks converted
+  static constexpr int TMEM_COLS = D + 2 * kBS <= 128 ? 128 : (D + 2 * kBS <= 256 ? 256 : 512);
+  static constexpr int O_COL = 0, S_COL = D;  // O: D columns; S buffers: 16 columns each
+  static constexpr int MAX_CTAS = 512 / TMEM_COLS;  // CTAs whose TMEM fits one SM
+  static constexpr int LAYOUT_BYTES = 1024 + OFF_MISC + 16;
+  // at least this much shared memory, so that no more than MAX_CTAS CTAs are resident
+  static constexpr int MIN_BYTES = kSmemPerSM / (MAX_CTAS + 1) + 1024;
+  static constexpr int SMEM_BYTES = LAYOUT_BYTES > MIN_BYTES ? LAYOUT_BYTES : MIN_BYTES;
+  static constexpr int THREADS = 320;
+  static constexpr int REG_CTAS = MAX_CTAS < 2 ? MAX_CTAS : 2;  // register budget hint
   static_assert(ROW_BYTES % 128 == 0, "rows must be whole 128-byte swizzle spans");
+  static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
   static_assert(!kFp8 || std::is_same<Q, __half>::value, "fp8 caches pair with fp16 queries");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
 // Shared blocks of group g that the pass covers: the group's prefix in whole
@@ -90,15 +118,20 @@ __device__ __forceinline__ int group_prefix_blocks(const PrefixParams& p, int g,
 }
 
 template <class C>
-__global__ void __launch_bounds__(C::THREADS, 1) paged_prefix_kernel(const __grid_constant__ CUtensorMap tmK,
-                                                                     const __grid_constant__ CUtensorMap tmV,
-                                                                     const PrefixParams p) {
+__global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
+    paged_prefix_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const PrefixParams p) {
   using Q = typename C::Q;
   constexpr int D = C::D, NS = C::NS;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
   const uint32_t base = smem_u32(smem);
-  const uint32_t full0 = base + C::OFF_BAR, empty0 = full0 + NS * 8;
+  const uint32_t bar0 = base + C::OFF_BAR;
+  const uint32_t full0 = bar0, empty0 = bar0 + 8 * NS, convf0 = bar0 + 16 * NS, sfull0 = convf0 + 16,
+                 pfull0 = sfull0 + 16, pvdone0 = pfull0 + 16, fin = pvdone0 + 16;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* dead = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  volatile int* converted = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const int g = blockIdx.z;
@@ -117,8 +150,7 @@ __global__ void __launch_bounds__(C::THREADS, 1) paged_prefix_kernel(const __gri
     if (threadIdx.x == 0) {
       s_ok = 1;
       const int len = p.group_prefix_len[g];
-      if (range_ok && len != 0 && pblk == 0) atomicOr(p.err, kCheckBadPrefix);
-      if (!range_ok) atomicOr(p.err, kCheckBadPrefix);
+      if (!range_ok || (len != 0 && pblk == 0)) atomicOr(p.err, kCheckBadPrefix);
     }
     __syncthreads();
     // every member is at least as long as the prefix and maps it to the same blocks
@@ -150,25 +182,69 @@ __global__ void __launch_bounds__(C::THREADS, 1) paged_prefix_kernel(const __gri
   const int hs = y - kvh * p.head_splits;
   const int head0 = kvh * p.group + hs * kNH;
   const int hpu = min(kNH, p.group - hs * kNH);  // query heads of this KV unit
-  const int rows = members * hpu;
+  const int rows = members * hpu;                 // (member, head) rows of this KV unit
   const int b0 = chunk * kPrefixChunkBlocks;
   const int nb = min(pblk, b0 + kPrefixChunkBlocks) - b0;
   if (nb <= 0 || rb * kPrefixRows >= rows) return;
 
-  __shared__ int s_dead;  // a consumer warp's wait timed out: the others stop waiting too
+  // query row r of this CTA -> (sequence, head); false past the group's rows
+  auto row_of = [&](int r, int& s, int& h) -> bool {
+    const int idx = rb * kPrefixRows + r;
+    if (idx >= rows) return false;
+    s = first + idx / hpu;
+    h = head0 + idx % hpu;
+    return true;
+  };
+
+  // ---- set-up: barriers, tensor memory, the query tile (128-byte swizzled)
   if (threadIdx.x == 0) {
-    s_dead = 0;
     for (int i = 0; i < NS; ++i) {
       mbar_init(full0 + 8 * i, 1);
-      mbar_init(empty0 + 8 * i, kPrefixWarps);
+      mbar_init(empty0 + 8 * i, 4);  // the four staging warps
     }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(convf0 + 8 * i, 4);
+      mbar_init(sfull0 + 8 * i, 1);  // tcgen05.commit
+      mbar_init(pfull0 + 8 * i, 4);  // the four softmax warps
+      mbar_init(pvdone0 + 8 * i, 1);
+    }
+    mbar_init(fin, 1);
+    *dead = 0;
+    *converted = 0;
     fence_mbar_init();
   }
+  if (warp == 0) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+  if (warp < 4) {
+    const int r = threadIdx.x;
+    int s = 0, h = 0;
+    const bool ok = row_of(r, s, h);
+    const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const Q*>(p.query) +
+                                                      ((size_t)s * p.num_heads + h) * D);
+#pragma unroll 4
+    for (int c = 0; c < D / 8; ++c) {
+      const uint4 v = ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+      const int sub = c >> 3, cc = c & 7;
+      *reinterpret_cast<uint4*>(smem + C::OFF_Q + sub * (kPrefixRows * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
+                                ((cc ^ (r & 7)) << 4)) = v;
+    }
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
 
-  if (warp == 0) {
-    // ---------------------------------------------------------------- producer
-    // the group's blocks, as the first member's table names them
+  // A failed (timed-out) wait marks the CTA dead: every role then stops.
+  auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    if (*dead) return false;
+    if (mbar_wait(bar, parity)) return true;
+    atomicOr(p.err, kCheckWaitTimeout);
+    *dead = 1;
+    return false;
+  };
+
+  if (warp == 8) {
+    // ---------------------------------------------------------------- TMA producer
     int my = 0;
     if (lane < nb) {
       my = __ldg(p.block_tables + (size_t)first * p.bt_stride + b0 + lane);
@@ -177,120 +253,230 @@ __global__ void __launch_bounds__(C::THREADS, 1) paged_prefix_kernel(const __gri
         my = 0;
       }
     }
+    int issued = 0;
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
     for (int i = 0; i < nb; ++i) {
       const int phys = __shfl_sync(0xffffffffu, my, i);
-      int stop = 0;
       if (lane == 0) {
         const int st = i % NS;
-        if (i >= NS && !mbar_wait(empty0 + 8 * st, ((i / NS) - 1) & 1)) {
-          atomicOr(p.err, kCheckWaitTimeout);
-          stop = 1;
-        } else {
-          const uint32_t fb = full0 + 8 * st;
-          mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
-          const uint32_t kdst = base + C::OFF_RING + st * C::STAGE_BYTES;
+        if (i >= NS && !wait(empty0 + 8 * st, ((i / NS) - 1) & 1)) break;
+        mbar_arrive_expect_tx(full0 + 8 * st, C::STAGE_BYTES);
+        const uint32_t kdst = base + C::OFF_RING + st * C::STAGE_BYTES;
 #pragma unroll
-          for (int sub = 0; sub < C::SUBTILES; ++sub) {
-            const int x = kvh * D + sub * (128 / (int)sizeof(typename C::KV));
-            tma_load_2d(kdst + sub * kBS * 128, &tmK, x, phys * kBS, fb);
-            tma_load_2d(kdst + C::TILE_BYTES + sub * kBS * 128, &tmV, x, phys * kBS, fb);
-          }
+        for (int sub = 0; sub < C::SUBTILES; ++sub) {
+          const int x = kvh * D + sub * (128 / (int)sizeof(typename C::KV));
+          tma_load_2d(kdst + sub * kBS * 128, &tmK, x, phys * kBS, full0 + 8 * st);
+          tma_load_2d(kdst + C::TILE_BYTES + sub * kBS * 128, &tmV, x, phys * kBS, full0 + 8 * st);
         }
-      }
-      if (__shfl_sync(0xffffffffu, stop, 0)) break;
-    }
-    return;
-  }
-
-  // ---------------------------------------------------------------- consumers
-  const int cw = warp - 1;
-  const int gid = lane >> 2, c4 = lane & 3;
-  // query row n of this warp's 8 -> (sequence, head); false past the group's rows
-  auto row_of = [&](int n, int& s, int& h) -> bool {
-    const int r = rb * kPrefixRows + cw * kNH + n;
-    if (r >= rows) return false;
-    s = first + r / hpu;
-    h = head0 + r % hpu;
-    return true;
-  };
-  WarpAttn<D, false, C::kBf16> A;
-  A.reset();
-  {
-    int s = 0, h = 0;
-    const bool ok = row_of(gid, s, h);
-    A.load_q(ok ? reinterpret_cast<const Q*>(p.query) + ((size_t)s * p.num_heads + h) * D : nullptr, c4);
-  }
-  // A timed-out wait (the check bit reports it) stops this warp's work, but it
-  // keeps meeting the consumers' named barrier once per block, so that no
-  // other warp waits for it there.
-  bool dead = false;
-  for (int i = 0; i < nb; ++i) {
-    const int st = i % NS;
-    if (!dead) {  // (warp-uniform)
-      bool fail = *reinterpret_cast<volatile int*>(&s_dead) != 0;
-      if (!fail) fail = !mbar_wait(full0 + 8 * st, (i / NS) & 1);
-      dead = __any_sync(0xffffffffu, fail);
-      if (dead && lane == 0) {
-        atomicOr(p.err, kCheckWaitTimeout);
-        s_dead = 1;
+        ++issued;
       }
     }
-    const uint32_t kb = base + C::OFF_RING + st * C::STAGE_BYTES;
-    uint32_t ka = kb, va = kb + C::TILE_BYTES;
-    if constexpr (C::kFp8) {
-      // The 256 consumer threads convert the K and V tiles (16 rows x D/16
-      // 16-byte chunks each) into f16 tiles with the 16-bit layout; buffer
-      // i & 1, so that converting block i + 1 never overwrites a tile a slower
-      // warp still reads (the barrier below orders block i's reads before any
-      // warp converts block i + 2).
-      if (!dead) {
-        const int t = threadIdx.x - 32;
-        const int which = t >> 7;
-        constexpr int CPR = D / 16;  // 16-byte fp8 chunks per row
-        const uint32_t dst = base + C::OFF_CONV + ((i & 1) * 2 + which) * C::F16_TILE;
-#pragma unroll
-        for (int k = t & 127; k < kBS * CPR; k += 128) {
-          const int r = k / CPR, cc = k - r * CPR;
-          const uint4 v = lds128(kb + which * C::TILE_BYTES + tile_off(r, 16 * cc));
+    // copies still in flight after a failure: wait for them (bounded) before the CTA exits
+    if (lane == 0)
+      for (int i = *converted; i < issued; ++i) mbar_wait(full0 + 8 * (i % NS), (i / NS) & 1);
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------------------------------------------------------- operand staging
+    const int t = threadIdx.x - 128;
+    for (int i = 0; i < nb; ++i) {
+      const int st = i % NS, cb = i & 1;
+      if (!wait(full0 + 8 * st, (i / NS) & 1)) break;
+      if (i >= 2 && !wait(pvdone0 + 8 * cb, ((i - 2) >> 1) & 1)) break;  // buffer cb free
+      const uint32_t ks = base + C::OFF_RING + st * C::STAGE_BYTES, vs = ks + C::TILE_BYTES;
+      uint8_t* kf = smem + C::OFF_KF + cb * C::KF_BYTES;
+      uint8_t* vt = smem + C::OFF_VT + cb * C::VT_BYTES;
+      // K: 16-bit, 128-byte swizzled, as the MMA's B operand reads it
+      if constexpr (C::kFp8) {
+        for (int k = t; k < kBS * (D / 16); k += 128) {  // 16 fp8 codes -> 16 halves
+          const int r = k / (D / 16), cc = k - r * (D / 16);
+          const uint4 v = lds128(ks + tile_off(r, 16 * cc));
           uint32_t h[8];
           e4m3x4_to_f16x2x2(v.x, h[0], h[1]);
           e4m3x4_to_f16x2x2(v.y, h[2], h[3]);
           e4m3x4_to_f16x2x2(v.z, h[4], h[5]);
           e4m3x4_to_f16x2x2(v.w, h[6], h[7]);
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + tile_off(r, 32 * cc)), "r"(h[0]),
-                       "r"(h[1]), "r"(h[2]), "r"(h[3])
-                       : "memory");
-          asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst + tile_off(r, 32 * cc + 16)),
-                       "r"(h[4]), "r"(h[5]), "r"(h[6]), "r"(h[7])
-                       : "memory");
+          *reinterpret_cast<uint4*>(kf + tile_off(r, 32 * cc)) = make_uint4(h[0], h[1], h[2], h[3]);
+          *reinterpret_cast<uint4*>(kf + tile_off(r, 32 * cc + 16)) = make_uint4(h[4], h[5], h[6], h[7]);
+        }
+      } else {
+        for (int k = t; k < kBS * (D / 8); k += 128) {
+          const int r = k / (D / 8), cc = k - r * (D / 8);
+          *reinterpret_cast<uint4*>(kf + tile_off(r, 16 * cc)) = lds128(ks + tile_off(r, 16 * cc));
         }
       }
-      named_bar_sync(1, kPrefixWarps * 32);  // converted tiles complete; the fp8 stage is free
-      if (!dead && lane == 0) mbar_arrive(empty0 + 8 * st);
-      ka = base + C::OFF_CONV + ((i & 1) * 2) * C::F16_TILE;
-      va = ka + C::F16_TILE;
-    }
-    if (dead) continue;
-    // the prefix covers whole blocks: all 16 tokens valid
-    A.block(ka, va, kBS, p.scale_log2, lane);
-    if constexpr (!C::kFp8) {
+      // V^T: element (dim n, token j) at (n/8)*256 + (j/8)*128 + (n%8)*16 + (j%8)*2;
+      // item = (8 dims, a pair of tokens) -> eight 32-bit (token pair) stores
+      for (int it = t; it < D; it += 128) {
+        const int c = it >> 3, pr = it & 7;  // dims [8c, 8c + 8), tokens 2pr, 2pr + 1
+        uint32_t a[4], b[4];
+        if constexpr (C::kFp8) {
+          uint32_t lo0, hi0;
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo0), "=r"(hi0) : "r"(vs + tile_off(2 * pr, 8 * c)));
+          e4m3x4_to_f16x2x2(lo0, a[0], a[1]);
+          e4m3x4_to_f16x2x2(hi0, a[2], a[3]);
+          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo0), "=r"(hi0) : "r"(vs + tile_off(2 * pr + 1, 8 * c)));
+          e4m3x4_to_f16x2x2(lo0, b[0], b[1]);
+          e4m3x4_to_f16x2x2(hi0, b[2], b[3]);
+        } else {
+          const uint4 u = lds128(vs + tile_off(2 * pr, 16 * c));
+          const uint4 w = lds128(vs + tile_off(2 * pr + 1, 16 * c));
+          a[0] = u.x; a[1] = u.y; a[2] = u.z; a[3] = u.w;
+          b[0] = w.x; b[1] = w.y; b[2] = w.z; b[3] = w.w;
+        }
+        uint8_t* dst = vt + c * 256 + (pr >> 2) * 128 + (pr & 3) * 4;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          *reinterpret_cast<uint32_t*>(dst + (2 * j) * 16) = prmt(a[j], b[j], 0x5410u);
+          *reinterpret_cast<uint32_t*>(dst + (2 * j + 1) * 16) = prmt(a[j], b[j], 0x7632u);
+        }
+      }
+      fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
       __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8 * st);
+      if (lane == 0) {
+        mbar_arrive(convf0 + 8 * cb);
+        mbar_arrive(empty0 + 8 * st);
+      }
+      if (t == 0) *converted = i + 1;
+    }
+  } else if (warp == 9) {
+    // ---------------------------------------------------------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t idS = umma_idesc_f16(kPrefixRows, kBS, C::kBf16);
+      constexpr uint32_t idO = umma_idesc_f16(kPrefixRows, D, C::kBf16);
+      const uint32_t qa = base + C::OFF_Q;
+      auto pv = [&](int j) {  // O += P_j V_j
+        const int cb = j & 1;
+        const uint64_t a = umma_desc(base + C::OFF_P + cb * C::P_BYTES, 128, 256, kUmmaNoSwizzle);
+        const uint64_t b = umma_desc(base + C::OFF_VT + cb * C::VT_BYTES, 128, 256, kUmmaNoSwizzle);
+        umma_f16(tmem + C::O_COL, a, b, idO, j > 0);
+        umma_commit(pvdone0 + 8 * cb);
+      };
+      int i = 0;
+      for (; i < nb; ++i) {
+        const int cb = i & 1;
+        if (!wait(convf0 + 8 * cb, (i >> 1) & 1)) break;
+        tc_fence_after();
+        const uint32_t kb = base + C::OFF_KF + cb * C::KF_BYTES;
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {  // S_i = Q K_i^T over 16-wide slices of D
+          const uint64_t a = umma_desc(qa + (k >> 2) * (kPrefixRows * 128) + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
+          const uint64_t b = umma_desc(kb + (k >> 2) * (kBS * 128) + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
+          umma_f16(tmem + C::S_COL + cb * kBS, a, b, idS, k > 0);
+        }
+        umma_commit(sfull0 + 8 * cb);
+        if (i >= 1) {
+          if (!wait(pfull0 + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1)) break;
+          tc_fence_after();
+          pv(i - 1);
+        }
+      }
+      if (i == nb && wait(pfull0 + 8 * ((nb - 1) & 1), ((nb - 1) >> 1) & 1)) {
+        tc_fence_after();
+        pv(nb - 1);
+      }
+      // every MMA issued has completed before the CTA releases tensor memory
+      umma_commit(fin);
+      mbar_wait(fin, 0);
+    }
+  } else {
+    // ---------------------------------------------------------------- softmax (warps 0..3)
+    const int r = threadIdx.x;
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int i = 0; i < nb && ok; ++i) {
+      const int cb = i & 1;
+      ok = wait(sfull0 + 8 * cb, (i >> 1) & 1);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sv[16];
+      tmem_ld16(trow + C::S_COL + cb * kBS, sv);
+      tmem_wait_ld();
+      float x[16];
+      float bm = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        x[j] = __uint_as_float(sv[j]) * p.scale_log2;
+        bm = fmaxf(bm, x[j]);
+      }
+      // lazy rescaling: move the reference max (and rescale l, O) only when
+      // this block's max exceeds it by more than 2^8
+      const bool grow = bm > m + 8.f;
+      if (i > 0 && __any_sync(0xffffffffu, grow)) {
+        ok = wait(pvdone0 + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1);  // O holds P_{i-1} V_{i-1}
+        if (!ok) break;
+        tc_fence_after();
+        const float al = grow ? ex2(m - bm) : 1.f;
+#pragma unroll 1
+        for (int c0 = 0; c0 < D; c0 += 16) {
+          uint32_t o[16];
+          tmem_ld16(trow + C::O_COL + c0, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * al);
+          tmem_st16(trow + C::O_COL + c0, o);
+        }
+        tmem_wait_st();
+        l *= al;
+      }
+      if (grow) m = bm;
+      uint32_t pk[8];
+      float sum = 0.f;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float p0 = ex2(x[2 * j] - m), p1 = ex2(x[2 * j + 1] - m);
+        sum += p0 + p1;
+        pk[j] = pack2<C::kBf16>(p0, p1);
+      }
+      l += sum;
+      // P_i row r: tokens 0..7 and 8..15 as two 16-byte core-matrix rows
+      if (i >= 2) {
+        ok = wait(pvdone0 + 8 * cb, ((i - 2) >> 1) & 1);  // P buffer cb free
+        if (!ok) break;
+      }
+      uint8_t* pr = smem + C::OFF_P + cb * C::P_BYTES + (r >> 3) * 256 + (r & 7) * 16;
+      *reinterpret_cast<uint4*>(pr) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      *reinterpret_cast<uint4*>(pr + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(pfull0 + 8 * cb);
+    }
+    if (ok) ok = wait(pvdone0 + 8 * ((nb - 1) & 1), ((nb - 1) >> 1) & 1);  // the last P V
+    if (ok) {
+      tc_fence_after();
+      int s = 0, h = 0;
+      const bool valid = row_of(r, s, h);
+      const float inv = l > 0.f ? p.v_scale / l : 0.f;
+      const size_t row = ((size_t)s * p.num_heads + h) * p.max_chunks + chunk;
+      float* dst = p.pre_o + row * D;
+#pragma unroll 1
+      for (int c0 = 0; c0 < D; c0 += 16) {
+        uint32_t o[16];
+        tmem_ld16(trow + C::O_COL + c0, o);
+        tmem_wait_ld();
+        if (valid) {
+#pragma unroll
+          for (int j = 0; j < 16; j += 4)
+            *reinterpret_cast<float4*>(dst + c0 + j) =
+                make_float4(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv,
+                            __uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
+        }
+      }
+      if (valid) *reinterpret_cast<float2*>(p.pre_ml + row * 2) = make_float2(m, l);
     }
   }
-  if (dead) return;
-  float L0, L1;
-  A.totals(L0, L1);
-  int s0 = 0, h0 = 0, s1 = 0, h1 = 0;
-  const bool ok0 = row_of(2 * c4, s0, h0), ok1 = row_of(2 * c4 + 1, s1, h1);
-  const size_t row0 = ((size_t)s0 * p.num_heads + h0) * p.max_chunks + chunk;
-  const size_t row1 = ((size_t)s1 * p.num_heads + h1) * p.max_chunks + chunk;
-  store_partial<D, false>(A.o, A.m0, L0, L0 > 0.f ? p.v_scale / L0 : 0.f, ok0, A.m1, L1,
-                          L1 > 0.f ? p.v_scale / L1 : 0.f, ok1, p.pre_o, p.pre_ml, row0, row1, lane);
+
+  // ---- tear-down: every tcgen05 operation has completed (the MMA thread
+  // waited for its last commit; loads were waited for); release TMEM
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
 }
 
 }  // namespace pa
