@@ -137,38 +137,38 @@ struct Tuned;
 #ifndef PA_MIN_CTAS_FP8_128
 #define PA_MIN_CTAS_FP8_128 8
 #endif
-// The shared-prefix pass's ring: 24-48 KiB of K/V in flight per CTA.
+// The shared-prefix pass: ring stages (blocks) and blocks per tensor-core step.
 template <> struct Tuned<64, __half, __half> {
   using C = DecodeCfg<64, __half, __half, PA_NS_16B_64, 8>;
-  using P = pa::PrefixCfg<64, __half, __half, 8>;
+  using P = pa::PrefixCfg<64, __half, __half, 8, 4>;
 };
 template <> struct Tuned<128, __half, __half> {
   using C = DecodeCfg<128, __half, __half, PA_NS_16B_128, 8>;
-  using P = pa::PrefixCfg<128, __half, __half, 4>;
+  using P = pa::PrefixCfg<128, __half, __half, 8, 4>;
 };
 template <> struct Tuned<256, __half, __half> {
   using C = DecodeCfg<256, __half, __half, PA_NS_16B_256, 3>;
-  using P = pa::PrefixCfg<256, __half, __half, 3>;
+  using P = pa::PrefixCfg<256, __half, __half, 4, 2>;
 };
 template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<64, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_64, 8>;
-  using P = pa::PrefixCfg<64, __nv_bfloat16, __nv_bfloat16, 8>;
+  using P = pa::PrefixCfg<64, __nv_bfloat16, __nv_bfloat16, 8, 4>;
 };
 template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128, 8>;
-  using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, 4>;
+  using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, 8, 4>;
 };
 template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_256, 3>;
-  using P = pa::PrefixCfg<256, __nv_bfloat16, __nv_bfloat16, 3>;
+  using P = pa::PrefixCfg<256, __nv_bfloat16, __nv_bfloat16, 4, 2>;
 };
 template <> struct Tuned<128, __nv_fp8_e4m3, __half> {
   using C = DecodeCfg<128, __nv_fp8_e4m3, __half, PA_NS_FP8_128, PA_MIN_CTAS_FP8_128>;
-  using P = pa::PrefixCfg<128, __nv_fp8_e4m3, __half, 6>;
+  using P = pa::PrefixCfg<128, __nv_fp8_e4m3, __half, 8, 4>;
 };
 template <> struct Tuned<256, __nv_fp8_e4m3, __half> {
   using C = DecodeCfg<256, __nv_fp8_e4m3, __half, PA_NS_FP8_256, 4>;
-  using P = pa::PrefixCfg<256, __nv_fp8_e4m3, __half, 4>;
+  using P = pa::PrefixCfg<256, __nv_fp8_e4m3, __half, 4, 2>;
 };
 
 bool select_kernels(int head_dim, int q_dtype, int kv_dtype, KernelSet* ks) {

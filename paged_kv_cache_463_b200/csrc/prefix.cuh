@@ -10,21 +10,24 @@
 // private suffixes go through the regular decode kernel, and the merge kernel
 // combines the two sets of (o, m, l) partials by log-sum-exp.
 //
-// With all members' query heads of one KV head stacked, a block is a dense
-// contraction: S[128 rows x 16 tokens] = Q K^T, then O[128 x D] += P V.  Both
-// run on the 5th-generation tensor cores (tcgen05.mma, issued by one thread,
+// With all members' query heads of one KV head stacked, attention over the
+// prefix is a dense contraction: for a step of T tokens (SB blocks),
+// S[128 rows x T] = Q K^T, then O[128 x D] += P V.  Both run on the
+// 5th-generation tensor cores (tcgen05.mma, issued by one thread,
 // accumulators in tensor memory), one CTA per (group, KV unit, 128 query
 // rows, chunk of 32 prefix blocks):
-//   warp 8      TMA producer: K/V tiles of the chunk's blocks into an NS-stage ring;
-//   warps 4..7  stage the MMA operands of each block: K as a 16-bit 128-byte-
-//               swizzled tile (fp8 E4M3 codes converted to f16), V transposed
-//               to V^T (tokens contiguous), double-buffered;
-//   warp 9      issues S_i = Q K_i^T into one of two TMEM S buffers, and
-//               O += P_{i-1} V_{i-1} once P_{i-1} is ready;
-//   warps 0..3  one query row per thread: read S_i from TMEM, online softmax
-//               in the log2 domain (lazy: O is rescaled in TMEM only when a
-//               row's maximum grows by more than 2^8), write P_i (16-bit) to
-//               shared memory; at the end read O, normalise, store partials.
+//   warp 8      TMA producer: each block's K/V tiles into an NS-stage ring;
+//   warps 4..7  stage a step's MMA operands: K as a 16-bit 128-byte-swizzled
+//               [T x D] tile (fp8 E4M3 codes converted to f16), V transposed
+//               to V^T [D x T] (tokens contiguous); two step buffers;
+//   warp 9      polls the barriers and issues S for a step once its operands
+//               are staged (into one of two TMEM S buffers) and O += P V once
+//               the softmax has written that step's P;
+//   warps 0..3  one query row per thread: read the step's S row from TMEM,
+//               online softmax in the log2 domain (lazy: O is rescaled in
+//               TMEM only when a row's maximum grows by more than 2^8), write
+//               P (16-bit) to shared memory; at the end read O, normalise,
+//               store the partial.
 #pragma once
 
 #include "decode.cuh"
@@ -62,47 +65,56 @@ struct PrefixParams {
 
 constexpr int kPrefixRows = 128;  // query rows per CTA (the MMA M)
 
-// Shared memory per SM and the per-CTA reservation, for capping residency.
+// Shared memory per SM, for capping residency.
 constexpr int kSmemPerSM = 233472;
 
-template <int D_, typename KV_, typename Q_, int NS_>
+template <int D_, typename KV_, typename Q_, int NS_, int SB_>
 struct PrefixCfg {
   static constexpr int D = D_;
   using KV = KV_;
   using Q = Q_;
-  static constexpr int NS = NS_;
+  static constexpr int NS = NS_;   // ring stages (blocks)
+  static constexpr int SB = SB_;   // blocks per step
+  static constexpr int T = SB * kBS;  // tokens per step (the S MMA's N, the P V MMA's K)
+  static constexpr int B = 2;      // step buffers (operands, S, P)
   static constexpr bool kFp8 = sizeof(KV) == 1;
   static constexpr bool kBf16 = std::is_same<Q, __nv_bfloat16>::value;
   static constexpr int ROW_BYTES = D * (int)sizeof(KV);
   static constexpr int SUBTILES = ROW_BYTES / 128;
   static constexpr int TILE_BYTES = kBS * ROW_BYTES;
   static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
-  static constexpr int Q_BYTES = kPrefixRows * D * 2;  // 128-byte swizzled, D/64 sub-tiles of 16 KB
-  static constexpr int KF_BYTES = kBS * D * 2;         // 16-bit K tile, D/64 sub-tiles of 2 KB
-  static constexpr int VT_BYTES = D * kBS * 2;         // V^T, no swizzle
-  static constexpr int P_BYTES = kPrefixRows * kBS * 2;
+  static constexpr int Q_BYTES = kPrefixRows * D * 2;  // 128-byte swizzled, D/64 sub-tiles of 128 rows
+  static constexpr int KF_BYTES = T * D * 2;           // 128-byte swizzled, D/64 sub-tiles of T rows
+  static constexpr int VT_BYTES = D * T * 2;           // no swizzle: (8 dims x 8 tokens) core matrices
+  static constexpr int P_BYTES = kPrefixRows * T * 2;  // no swizzle: (8 rows x 8 tokens) core matrices
+  static constexpr int CM_STRIDE = T * 16;             // bytes between 8-row groups of V^T and P
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING = OFF_Q + Q_BYTES;
-  static constexpr int OFF_KF = OFF_RING + NS * STAGE_BYTES;  // [2]
-  static constexpr int OFF_VT = OFF_KF + 2 * KF_BYTES;        // [2]
-  static constexpr int OFF_P = OFF_VT + 2 * VT_BYTES;         // [2]
-  static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-  // full[NS] empty[NS] conv_full[2] s_full[2] p_full[2] pv_done[2] fin
-  static constexpr int NBARS = 2 * NS + 9;
+  static constexpr int OFF_KF = OFF_RING + NS * STAGE_BYTES;  // [B]
+  static constexpr int OFF_VT = OFF_KF + B * KF_BYTES;        // [B]
+  static constexpr int OFF_P = OFF_VT + B * VT_BYTES;         // [B]
+  static constexpr int OFF_BAR = OFF_P + B * P_BYTES;
+  // full[NS] empty[NS] conv_full[B] s_full[B] p_full[B] pv_done[B] fin
+  static constexpr int NBARS = 2 * NS + 4 * B + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem base, dead flag, blocks converted
-  static constexpr int TMEM_COLS = D + 2 * kBS <= 128 ? 128 : (D + 2 * kBS <= 256 ? 256 : 512);
-  static constexpr int O_COL = 0, S_COL = D;  // O: D columns; S buffers: 16 columns each
+  static constexpr int TMEM_COLS = D + B * T <= 128 ? 128 : (D + B * T <= 256 ? 256 : 512);
+  static constexpr int O_COL = 0, S_COL = D;  // O: D columns; S buffers: T columns each
   static constexpr int MAX_CTAS = 512 / TMEM_COLS;  // CTAs whose TMEM fits one SM
   static constexpr int LAYOUT_BYTES = 1024 + OFF_MISC + 16;
   // at least this much shared memory, so that no more than MAX_CTAS CTAs are resident
   static constexpr int MIN_BYTES = kSmemPerSM / (MAX_CTAS + 1) + 1024;
   static constexpr int SMEM_BYTES = LAYOUT_BYTES > MIN_BYTES ? LAYOUT_BYTES : MIN_BYTES;
   static constexpr int THREADS = 320;
-  static constexpr int REG_CTAS = MAX_CTAS < 2 ? MAX_CTAS : 2;  // register budget hint
+  static constexpr int REG_CTAS = 1;  // register budget hint (shared memory allows one CTA per SM)
   static_assert(ROW_BYTES % 128 == 0, "rows must be whole 128-byte swizzle spans");
   static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
+  static_assert(T % 16 == 0 && T <= 256, "step tokens");
   static_assert(!kFp8 || std::is_same<Q, __half>::value, "fp8 caches pair with fp16 queries");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
+  // byte offset of (row, byte-in-row) in a 128-byte-swizzled tile of `rows` rows
+  __device__ static uint32_t sw128(int rows, int row, int byte) {
+    return (uint32_t)((byte >> 7) * (rows * 128) + row * 128 + (((((byte & 127) >> 4) ^ (row & 7)) << 4) | (byte & 15)));
+  }
 };
 
 // Shared blocks of group g that the pass covers: the group's prefix in whole
@@ -127,8 +139,8 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
   const uint32_t base = smem_u32(smem);
   const uint32_t bar0 = base + C::OFF_BAR;
-  const uint32_t full0 = bar0, empty0 = bar0 + 8 * NS, convf0 = bar0 + 16 * NS, sfull0 = convf0 + 16,
-                 pfull0 = sfull0 + 16, pvdone0 = pfull0 + 16, fin = pvdone0 + 16;
+  const uint32_t full0 = bar0, empty0 = bar0 + 8 * NS, convf0 = bar0 + 16 * NS, sfull0 = convf0 + 8 * C::B,
+                 pfull0 = sfull0 + 8 * C::B, pvdone0 = pfull0 + 8 * C::B, fin = pvdone0 + 8 * C::B;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* dead = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   volatile int* converted = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
@@ -197,12 +209,14 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
   };
 
   // ---- set-up: barriers, tensor memory, the query tile (128-byte swizzled)
+  constexpr int B = C::B, SB = C::SB, T = C::T;
+  const int nsteps = (nb + SB - 1) / SB;
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
       mbar_init(full0 + 8 * i, 1);
       mbar_init(empty0 + 8 * i, 4);  // the four staging warps
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < B; ++i) {
       mbar_init(convf0 + 8 * i, 4);
       mbar_init(sfull0 + 8 * i, 1);  // tcgen05.commit
       mbar_init(pfull0 + 8 * i, 4);  // the four softmax warps
@@ -223,9 +237,7 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
 #pragma unroll 4
     for (int c = 0; c < D / 8; ++c) {
       const uint4 v = ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-      const int sub = c >> 3, cc = c & 7;
-      *reinterpret_cast<uint4*>(smem + C::OFF_Q + sub * (kPrefixRows * 128) + (r >> 3) * 1024 + (r & 7) * 128 +
-                                ((cc ^ (r & 7)) << 4)) = v;
+      *reinterpret_cast<uint4*>(smem + C::OFF_Q + C::sw128(kPrefixRows, r, 16 * c)) = v;
     }
     fence_proxy_async_smem();
   }
@@ -280,101 +292,133 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
   } else if (warp >= 4 && warp < 8) {
     // ---------------------------------------------------------------- operand staging
     const int t = threadIdx.x - 128;
-    for (int i = 0; i < nb; ++i) {
-      const int st = i % NS, cb = i & 1;
-      if (!wait(full0 + 8 * st, (i / NS) & 1)) break;
-      if (i >= 2 && !wait(pvdone0 + 8 * cb, ((i - 2) >> 1) & 1)) break;  // buffer cb free
-      const uint32_t ks = base + C::OFF_RING + st * C::STAGE_BYTES, vs = ks + C::TILE_BYTES;
+    for (int u = 0; u < nsteps; ++u) {
+      const int cb = u % B;
+      if (u >= B && !wait(pvdone0 + 8 * cb, ((u - B) / B) & 1)) break;  // step buffer cb free
       uint8_t* kf = smem + C::OFF_KF + cb * C::KF_BYTES;
       uint8_t* vt = smem + C::OFF_VT + cb * C::VT_BYTES;
-      // K: 16-bit, 128-byte swizzled, as the MMA's B operand reads it
-      if constexpr (C::kFp8) {
-        for (int k = t; k < kBS * (D / 16); k += 128) {  // 16 fp8 codes -> 16 halves
-          const int r = k / (D / 16), cc = k - r * (D / 16);
-          const uint4 v = lds128(ks + tile_off(r, 16 * cc));
-          uint32_t h[8];
-          e4m3x4_to_f16x2x2(v.x, h[0], h[1]);
-          e4m3x4_to_f16x2x2(v.y, h[2], h[3]);
-          e4m3x4_to_f16x2x2(v.z, h[4], h[5]);
-          e4m3x4_to_f16x2x2(v.w, h[6], h[7]);
-          *reinterpret_cast<uint4*>(kf + tile_off(r, 32 * cc)) = make_uint4(h[0], h[1], h[2], h[3]);
-          *reinterpret_cast<uint4*>(kf + tile_off(r, 32 * cc + 16)) = make_uint4(h[4], h[5], h[6], h[7]);
-        }
-      } else {
-        for (int k = t; k < kBS * (D / 8); k += 128) {
-          const int r = k / (D / 8), cc = k - r * (D / 8);
-          *reinterpret_cast<uint4*>(kf + tile_off(r, 16 * cc)) = lds128(ks + tile_off(r, 16 * cc));
-        }
-      }
-      // V^T: element (dim n, token j) at (n/8)*256 + (j/8)*128 + (n%8)*16 + (j%8)*2;
-      // item = (8 dims, a pair of tokens) -> eight 32-bit (token pair) stores
-      for (int it = t; it < D; it += 128) {
-        const int c = it >> 3, pr = it & 7;  // dims [8c, 8c + 8), tokens 2pr, 2pr + 1
-        uint32_t a[4], b[4];
-        if constexpr (C::kFp8) {
-          uint32_t lo0, hi0;
-          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo0), "=r"(hi0) : "r"(vs + tile_off(2 * pr, 8 * c)));
-          e4m3x4_to_f16x2x2(lo0, a[0], a[1]);
-          e4m3x4_to_f16x2x2(hi0, a[2], a[3]);
-          asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo0), "=r"(hi0) : "r"(vs + tile_off(2 * pr + 1, 8 * c)));
-          e4m3x4_to_f16x2x2(lo0, b[0], b[1]);
-          e4m3x4_to_f16x2x2(hi0, b[2], b[3]);
-        } else {
-          const uint4 u = lds128(vs + tile_off(2 * pr, 16 * c));
-          const uint4 w = lds128(vs + tile_off(2 * pr + 1, 16 * c));
-          a[0] = u.x; a[1] = u.y; a[2] = u.z; a[3] = u.w;
-          b[0] = w.x; b[1] = w.y; b[2] = w.z; b[3] = w.w;
-        }
-        uint8_t* dst = vt + c * 256 + (pr >> 2) * 128 + (pr & 3) * 4;
+      bool stop = false;
+#pragma unroll 1
+      for (int j = 0; j < SB; ++j) {
+        const int i = u * SB + j;  // block of the chunk
+        if (i >= nb) {
+          // past the prefix: zero V^T (P is 0 there, and 0 * garbage could be NaN)
+          for (int it = t; it < D; it += 128) {
+            uint8_t* dst = vt + (it >> 3) * C::CM_STRIDE + ((16 * j + 2 * (it & 7)) >> 3) * 128 + ((2 * (it & 7)) & 7) * 2;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          *reinterpret_cast<uint32_t*>(dst + (2 * j) * 16) = prmt(a[j], b[j], 0x5410u);
-          *reinterpret_cast<uint32_t*>(dst + (2 * j + 1) * 16) = prmt(a[j], b[j], 0x7632u);
+            for (int q = 0; q < 8; ++q) *reinterpret_cast<uint32_t*>(dst + q * 16) = 0u;
+          }
+          continue;
         }
+        const int st = i % NS;
+        if (!wait(full0 + 8 * st, (i / NS) & 1)) {
+          stop = true;
+          break;
+        }
+        const uint32_t ks = base + C::OFF_RING + st * C::STAGE_BYTES, vs = ks + C::TILE_BYTES;
+        // K rows 16j..16j+15 of the step's tile
+        if constexpr (C::kFp8) {
+          for (int k = t; k < kBS * (D / 16); k += 128) {  // 16 fp8 codes -> 16 halves
+            const int r = k / (D / 16), cc = k - r * (D / 16);
+            const uint4 v = lds128(ks + tile_off(r, 16 * cc));
+            uint32_t h[8];
+            e4m3x4_to_f16x2x2(v.x, h[0], h[1]);
+            e4m3x4_to_f16x2x2(v.y, h[2], h[3]);
+            e4m3x4_to_f16x2x2(v.z, h[4], h[5]);
+            e4m3x4_to_f16x2x2(v.w, h[6], h[7]);
+            *reinterpret_cast<uint4*>(kf + C::sw128(T, 16 * j + r, 32 * cc)) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4*>(kf + C::sw128(T, 16 * j + r, 32 * cc + 16)) = make_uint4(h[4], h[5], h[6], h[7]);
+          }
+        } else {
+          for (int k = t; k < kBS * (D / 8); k += 128) {
+            const int r = k / (D / 8), cc = k - r * (D / 8);
+            *reinterpret_cast<uint4*>(kf + C::sw128(T, 16 * j + r, 16 * cc)) = lds128(ks + tile_off(r, 16 * cc));
+          }
+        }
+        // V^T: element (dim n, token tt) at (n/8)*CM_STRIDE + (tt/8)*128 + (n%8)*16 + (tt%8)*2;
+        // item = (8 dims, a pair of tokens) -> eight 32-bit (token pair) stores
+        for (int it = t; it < D; it += 128) {
+          const int c = it >> 3, pr = it & 7;  // dims [8c, 8c + 8), tokens 2pr, 2pr + 1 of the block
+          uint32_t a[4], bb[4];
+          if constexpr (C::kFp8) {
+            uint32_t lo0, hi0;
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo0), "=r"(hi0) : "r"(vs + tile_off(2 * pr, 8 * c)));
+            e4m3x4_to_f16x2x2(lo0, a[0], a[1]);
+            e4m3x4_to_f16x2x2(hi0, a[2], a[3]);
+            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo0), "=r"(hi0) : "r"(vs + tile_off(2 * pr + 1, 8 * c)));
+            e4m3x4_to_f16x2x2(lo0, bb[0], bb[1]);
+            e4m3x4_to_f16x2x2(hi0, bb[2], bb[3]);
+          } else {
+            const uint4 x0 = lds128(vs + tile_off(2 * pr, 16 * c));
+            const uint4 x1 = lds128(vs + tile_off(2 * pr + 1, 16 * c));
+            a[0] = x0.x; a[1] = x0.y; a[2] = x0.z; a[3] = x0.w;
+            bb[0] = x1.x; bb[1] = x1.y; bb[2] = x1.z; bb[3] = x1.w;
+          }
+          const int tt = 16 * j + 2 * pr;
+          uint8_t* dst = vt + c * C::CM_STRIDE + (tt >> 3) * 128 + (tt & 7) * 2;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            *reinterpret_cast<uint32_t*>(dst + (2 * q) * 16) = prmt(a[q], bb[q], 0x5410u);
+            *reinterpret_cast<uint32_t*>(dst + (2 * q + 1) * 16) = prmt(a[q], bb[q], 0x7632u);
+          }
+        }
+        fence_proxy_async_smem();  // (the ring stage's next writer is TMA)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * st);
+        if (t == 0) *converted = i + 1;
       }
+      if (stop) break;
       fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(convf0 + 8 * cb);
-        mbar_arrive(empty0 + 8 * st);
-      }
-      if (t == 0) *converted = i + 1;
+      if (lane == 0) mbar_arrive(convf0 + 8 * cb);
     }
   } else if (warp == 9) {
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
-      constexpr uint32_t idS = umma_idesc_f16(kPrefixRows, kBS, C::kBf16);
+      constexpr uint32_t idS = umma_idesc_f16(kPrefixRows, T, C::kBf16);
       constexpr uint32_t idO = umma_idesc_f16(kPrefixRows, D, C::kBf16);
       const uint32_t qa = base + C::OFF_Q;
-      auto pv = [&](int j) {  // O += P_j V_j
-        const int cb = j & 1;
-        const uint64_t a = umma_desc(base + C::OFF_P + cb * C::P_BYTES, 128, 256, kUmmaNoSwizzle);
-        const uint64_t b = umma_desc(base + C::OFF_VT + cb * C::VT_BYTES, 128, 256, kUmmaNoSwizzle);
-        umma_f16(tmem + C::O_COL, a, b, idO, j > 0);
-        umma_commit(pvdone0 + 8 * cb);
-      };
-      int i = 0;
-      for (; i < nb; ++i) {
-        const int cb = i & 1;
-        if (!wait(convf0 + 8 * cb, (i >> 1) & 1)) break;
-        tc_fence_after();
-        const uint32_t kb = base + C::OFF_KF + cb * C::KF_BYTES;
-#pragma unroll
-        for (int k = 0; k < D / 16; ++k) {  // S_i = Q K_i^T over 16-wide slices of D
-          const uint64_t a = umma_desc(qa + (k >> 2) * (kPrefixRows * 128) + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
-          const uint64_t b = umma_desc(kb + (k >> 2) * (kBS * 128) + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
-          umma_f16(tmem + C::S_COL + cb * kBS, a, b, idS, k > 0);
-        }
-        umma_commit(sfull0 + 8 * cb);
-        if (i >= 1) {
-          if (!wait(pfull0 + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1)) break;
+      // Issue S for a step as soon as its operands are staged (at most B
+      // steps ahead of the softmax), and O += P V as soon as the softmax has
+      // written that step's P: both polled without blocking.
+      int ns_ = 0, npv = 0;
+      long long idle_since = clock64();
+      while (npv < nsteps && !*dead) {
+        bool progress = false;
+        if (ns_ < nsteps && ns_ - npv < B && mbar_test_wait(convf0 + 8 * (ns_ % B), (ns_ / B) & 1)) {
           tc_fence_after();
-          pv(i - 1);
+          const int cb = ns_ % B;
+          const uint32_t kb = base + C::OFF_KF + cb * C::KF_BYTES;
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {  // S = Q K^T over 16-wide slices of D
+            const uint64_t a = umma_desc(qa + (k >> 2) * (kPrefixRows * 128) + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
+            const uint64_t b = umma_desc(kb + (k >> 2) * (T * 128) + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
+            umma_f16(tmem + C::S_COL + cb * T, a, b, idS, k > 0);
+          }
+          umma_commit(sfull0 + 8 * cb);
+          ++ns_;
+          progress = true;
         }
-      }
-      if (i == nb && wait(pfull0 + 8 * ((nb - 1) & 1), ((nb - 1) >> 1) & 1)) {
-        tc_fence_after();
-        pv(nb - 1);
+        if (npv < ns_ && mbar_test_wait(pfull0 + 8 * (npv % B), (npv / B) & 1)) {
+          tc_fence_after();
+          const int cb = npv % B;
+          const uint32_t pa_ = base + C::OFF_P + cb * C::P_BYTES, va = base + C::OFF_VT + cb * C::VT_BYTES;
+#pragma unroll
+          for (int k = 0; k < T / 16; ++k) {  // O += P V over 16-token slices
+            const uint64_t a = umma_desc(pa_ + k * 256, 128, C::CM_STRIDE, kUmmaNoSwizzle);
+            const uint64_t b = umma_desc(va + k * 256, 128, C::CM_STRIDE, kUmmaNoSwizzle);
+            umma_f16(tmem + C::O_COL, a, b, idO, (npv > 0 || k > 0) ? 1 : 0);
+          }
+          umma_commit(pvdone0 + 8 * cb);
+          ++npv;
+          progress = true;
+        }
+        if (progress) {
+          idle_since = clock64();
+        } else if (clock64() - idle_since > kWaitLimitCycles) {
+          atomicOr(p.err, kCheckWaitTimeout);
+          *dead = 1;
+        }
       }
       // every MMA issued has completed before the CTA releases tensor memory
       umma_commit(fin);
@@ -386,26 +430,32 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int i = 0; i < nb && ok; ++i) {
-      const int cb = i & 1;
-      ok = wait(sfull0 + 8 * cb, (i >> 1) & 1);
+    for (int u = 0; u < nsteps && ok; ++u) {
+      const int cb = u % B;
+      ok = wait(sfull0 + 8 * cb, (u / B) & 1);
       if (!ok) break;
       tc_fence_after();
-      uint32_t sv[16];
-      tmem_ld16(trow + C::S_COL + cb * kBS, sv);
+      float x[T];
+#pragma unroll
+      for (int c0 = 0; c0 < T; c0 += 16) {
+        uint32_t sv[16];
+        tmem_ld16(trow + C::S_COL + cb * T + c0, sv);
+#pragma unroll
+        for (int j = 0; j < 16; ++j) x[c0 + j] = __uint_as_float(sv[j]);
+      }
       tmem_wait_ld();
-      float x[16];
+      const int valid = min(T, (nb - u * SB) * kBS);  // tokens of the prefix in this step
       float bm = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        x[j] = __uint_as_float(sv[j]) * p.scale_log2;
+      for (int j = 0; j < T; ++j) {
+        x[j] = j < valid ? x[j] * p.scale_log2 : -INFINITY;
         bm = fmaxf(bm, x[j]);
       }
       // lazy rescaling: move the reference max (and rescale l, O) only when
-      // this block's max exceeds it by more than 2^8
+      // this step's max exceeds it by more than 2^8
       const bool grow = bm > m + 8.f;
-      if (i > 0 && __any_sync(0xffffffffu, grow)) {
-        ok = wait(pvdone0 + 8 * ((i - 1) & 1), ((i - 1) >> 1) & 1);  // O holds P_{i-1} V_{i-1}
+      if (u > 0 && __any_sync(0xffffffffu, grow)) {
+        ok = wait(pvdone0 + 8 * ((u - 1) % B), ((u - 1) / B) & 1);  // O holds every earlier step
         if (!ok) break;
         tc_fence_after();
         const float al = grow ? ex2(m - bm) : 1.f;
@@ -422,29 +472,31 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
         l *= al;
       }
       if (grow) m = bm;
-      uint32_t pk[8];
-      float sum = 0.f;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const float p0 = ex2(x[2 * j] - m), p1 = ex2(x[2 * j + 1] - m);
-        sum += p0 + p1;
-        pk[j] = pack2<C::kBf16>(p0, p1);
-      }
-      l += sum;
-      // P_i row r: tokens 0..7 and 8..15 as two 16-byte core-matrix rows
-      if (i >= 2) {
-        ok = wait(pvdone0 + 8 * cb, ((i - 2) >> 1) & 1);  // P buffer cb free
+      if (u >= B) {
+        ok = wait(pvdone0 + 8 * cb, ((u - B) / B) & 1);  // P buffer cb free
         if (!ok) break;
       }
-      uint8_t* pr = smem + C::OFF_P + cb * C::P_BYTES + (r >> 3) * 256 + (r & 7) * 16;
-      *reinterpret_cast<uint4*>(pr) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-      *reinterpret_cast<uint4*>(pr + 128) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+      // P row r: token groups of 8 as 16-byte core-matrix rows
+      uint8_t* prow = smem + C::OFF_P + cb * C::P_BYTES + (r >> 3) * C::CM_STRIDE + (r & 7) * 16;
+      float sum = 0.f;
+#pragma unroll
+      for (int g8 = 0; g8 < T / 8; ++g8) {
+        uint32_t pk[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float p0 = ex2(x[8 * g8 + 2 * q] - m), p1 = ex2(x[8 * g8 + 2 * q + 1] - m);
+          sum += p0 + p1;
+          pk[q] = pack2<C::kBf16>(p0, p1);
+        }
+        *reinterpret_cast<uint4*>(prow + g8 * 128) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+      }
+      l += sum;
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(pfull0 + 8 * cb);
     }
-    if (ok) ok = wait(pvdone0 + 8 * ((nb - 1) & 1), ((nb - 1) >> 1) & 1);  // the last P V
+    if (ok) ok = wait(pvdone0 + 8 * ((nsteps - 1) % B), ((nsteps - 1) / B) & 1);  // the last P V
     if (ok) {
       tc_fence_after();
       int s = 0, h = 0;
