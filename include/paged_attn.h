@@ -47,6 +47,7 @@ extern "C" {
 #define PA_ERR_DEVICE_CHECK (-4) /* a device-side check fired; paged_attn_last_check_bits() says which */
 #define PA_ERR_NO_MEMORY (-5)    /* workspace allocation failed */
 #define PA_ERR_SCRATCH_TOO_SMALL (-6) /* paged_attention_decode_noalloc: partials exceed PA_NOALLOC_SCRATCH_BYTES */
+#define PA_ERR_OUT_OF_BLOCKS (-7)     /* block manager: no free block and nothing evictable (block_manager.h) */
 
 /* ---- device check bits (paged_attn_last_check_bits) */
 #define PA_CHECK_BAD_BLOCK 1    /* block-table entry outside [0, num_blocks): read block 0 instead */

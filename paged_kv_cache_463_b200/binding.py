@@ -17,6 +17,7 @@ import torch
 _PKG = os.path.dirname(os.path.abspath(__file__))
 DEFAULT_LIB = os.path.join(_PKG, "lib", "libpaged_attn.so")
 HEADER = os.path.join(os.path.dirname(_PKG), "include", "paged_attn.h")
+HEADERS = [HEADER, os.path.join(os.path.dirname(_PKG), "include", "block_manager.h")]
 
 PA_OK = 0
 PA_ERR_INVALID_ARG = -1
@@ -25,6 +26,7 @@ PA_ERR_CUDA = -3
 PA_ERR_DEVICE_CHECK = -4
 PA_ERR_NO_MEMORY = -5
 PA_ERR_SCRATCH_TOO_SMALL = -6
+PA_ERR_OUT_OF_BLOCKS = -7
 PA_NOALLOC_SCRATCH_BYTES = 16 * 1024 * 1024
 PA_CHECK_BAD_BLOCK, PA_CHECK_BAD_SLOT, PA_CHECK_SEQ_TOO_LONG, PA_CHECK_WAIT_TIMEOUT = 1, 2, 4, 8
 PA_CHECK_BAD_PREFIX = 16
@@ -76,6 +78,22 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "paged_copy_blocks": (i, [_P, _P, _P, i64, _P, _P, i64, _P, i, _P]),
         "paged_attention_decode_noalloc": (i, [_P, _P, _P, _P, _P, i, _P, i, i, i, i, i, i, i, i, i, i, f, f, f,
                                                _P, _P]),
+        # block manager (include/block_manager.h)
+        "pa_bm_create": (i, [i, i, ctypes.POINTER(_P)]),
+        "pa_bm_destroy": (i, [_P]),
+        "pa_bm_num_free": (i, [_P, _P]),
+        "pa_bm_ref_count": (i, [_P, i, _P]),
+        "pa_bm_cached_blocks": (i, [_P, _P]),
+        "pa_bm_add_sequence": (i, [_P, i64]),
+        "pa_bm_free_sequence": (i, [_P, i64]),
+        "pa_bm_ensure_capacity": (i, [_P, i64, i64]),
+        "pa_bm_append_tokens": (i, [_P, i64, i, _P, _P, _P, _P]),
+        "pa_bm_fork": (i, [_P, i64, i64]),
+        "pa_bm_seq_len": (i, [_P, i64, _P]),
+        "pa_bm_block_table": (i, [_P, i64, _P, i, _P]),
+        "pa_bm_build_batch": (i, [_P, _P, i, _P, i, _P]),
+        "pa_bm_evict_lru_sequence": (i, [_P, i64, i, _P]),
+        "pa_bm_allocate_with_prefix": (i, [_P, i64, _P, i, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -85,8 +103,10 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
     return lib
 
 
-def header_functions(header: str = HEADER) -> list[str]:
-    """Names of the functions include/paged_attn.h declares."""
+def header_functions(header: str | None = None) -> list[str]:
+    """Names of the functions the headers under include/ declare (or one header)."""
+    if header is None:
+        return sorted(set(n for h in HEADERS for n in header_functions(h)))
     text = open(header, encoding="utf-8").read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
     return sorted(set(re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w ]*?\**\s*\b([a-z_][a-z0-9_]*)\s*\(", text, flags=re.M)))
@@ -239,3 +259,105 @@ class PagedAttention:
         c = self.cfg
         return torch.empty((c.num_blocks, c.block_size, c.num_kv_heads, c.head_dim), dtype=TORCH_OF[self.kv_dtype],
                            device=f"cuda:{self.device}")
+
+
+class BlockManager:
+    """Host block manager of the library (include/block_manager.h): argument
+    marshalling only; failures raise PagedAttnError with the status code."""
+
+    def __init__(self, num_blocks: int, block_size: int = 16, lib_path: str | None = None):
+        self.lib = load_library(lib_path)
+        h = _P()
+        self._check(self.lib.pa_bm_create(int(num_blocks), int(block_size), ctypes.byref(h)), "pa_bm_create")
+        self.h = h
+        self.block_size = block_size
+
+    def _check(self, st: int, what: str) -> None:
+        if st != PA_OK:
+            raise PagedAttnError(st, f"{what}: {self.lib.paged_attn_status_string(st).decode()}")
+
+    def close(self) -> None:
+        if getattr(self, "h", None):
+            self.lib.pa_bm_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def _int_out(self, fn, *args) -> int:
+        v = ctypes.c_int(0)
+        self._check(fn(self.h, *args, ctypes.byref(v)), fn.__name__)
+        return v.value
+
+    def num_free(self) -> int:
+        return self._int_out(self.lib.pa_bm_num_free)
+
+    def ref_count(self, block: int) -> int:
+        return self._int_out(self.lib.pa_bm_ref_count, int(block))
+
+    def cached_blocks(self) -> int:
+        return self._int_out(self.lib.pa_bm_cached_blocks)
+
+    def add_sequence(self, sid: int) -> None:
+        self._check(self.lib.pa_bm_add_sequence(self.h, int(sid)), "pa_bm_add_sequence")
+
+    def free_sequence(self, sid: int) -> None:
+        self._check(self.lib.pa_bm_free_sequence(self.h, int(sid)), "pa_bm_free_sequence")
+
+    def ensure_capacity(self, sid: int, required_tokens: int) -> None:
+        self._check(self.lib.pa_bm_ensure_capacity(self.h, int(sid), int(required_tokens)), "pa_bm_ensure_capacity")
+
+    def append_tokens(self, sid: int, n: int):
+        """Returns (status, slots, copy pairs) for the positions appended
+        (all n on PA_OK, fewer on PA_ERR_OUT_OF_BLOCKS); other failures raise."""
+        slots = (ctypes.c_int64 * max(1, n))()
+        pairs = (ctypes.c_int64 * max(2, 2 * n))()
+        nc, na = ctypes.c_int(0), ctypes.c_int(0)
+        st = self.lib.pa_bm_append_tokens(self.h, int(sid), int(n), slots, pairs, ctypes.byref(nc), ctypes.byref(na))
+        if st not in (PA_OK, PA_ERR_OUT_OF_BLOCKS):
+            self._check(st, "pa_bm_append_tokens")
+        return st, list(slots[:na.value]), [(pairs[2 * k], pairs[2 * k + 1]) for k in range(nc.value)]
+
+    def fork(self, parent: int, child: int) -> None:
+        self._check(self.lib.pa_bm_fork(self.h, int(parent), int(child)), "pa_bm_fork")
+
+    def seq_len(self, sid: int) -> int:
+        v = ctypes.c_int64(0)
+        self._check(self.lib.pa_bm_seq_len(self.h, int(sid), ctypes.byref(v)), "pa_bm_seq_len")
+        return v.value
+
+    def block_table(self, sid: int) -> list[int]:
+        n = ctypes.c_int(0)
+        self._check(self.lib.pa_bm_block_table(self.h, int(sid), None, 0, ctypes.byref(n)), "pa_bm_block_table")
+        buf = (ctypes.c_int32 * max(1, n.value))()
+        self._check(self.lib.pa_bm_block_table(self.h, int(sid), buf, n.value, ctypes.byref(n)), "pa_bm_block_table")
+        return list(buf[:n.value])
+
+    def build_batch(self, sids, bt_stride: int):
+        """int32 tables [n, bt_stride] (-1 padded) and lengths [n], as torch CPU tensors."""
+        n = len(sids)
+        ids = (ctypes.c_int64 * max(1, n))(*[int(x) for x in sids])
+        tables = torch.empty((n, bt_stride), dtype=torch.int32)
+        lens = torch.empty((n,), dtype=torch.int32)
+        self._check(self.lib.pa_bm_build_batch(self.h, ids, n, tables.data_ptr() if n else None, int(bt_stride),
+                                               lens.data_ptr() if n else None), "pa_bm_build_batch")
+        return tables, lens
+
+    def evict_lru_sequence(self, exclude: int | None = None) -> int:
+        v = ctypes.c_int64(0)
+        self._check(self.lib.pa_bm_evict_lru_sequence(self.h, int(exclude or 0), 0 if exclude is None else 1,
+                                                      ctypes.byref(v)), "pa_bm_evict_lru_sequence")
+        return v.value
+
+    def allocate_with_prefix(self, sid: int, tokens):
+        """Returns (matched tokens, slots of the positions from the match on)."""
+        n = len(tokens)
+        toks = (ctypes.c_int32 * max(1, n))(*[int(t) for t in tokens])
+        slots = (ctypes.c_int64 * max(1, n))()
+        m, ns = ctypes.c_int(0), ctypes.c_int(0)
+        self._check(self.lib.pa_bm_allocate_with_prefix(self.h, int(sid), toks, n, ctypes.byref(m), slots,
+                                                        ctypes.byref(ns)), "pa_bm_allocate_with_prefix")
+        return m.value, list(slots[:ns.value])

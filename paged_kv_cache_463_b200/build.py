@@ -21,9 +21,10 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libpaged_attn.so")
-SOURCES = ["paged_attn.cu"]
-DEPS = ["paged_attn.cu", "decode.cuh", "cache_ops.cuh", "ptx.cuh"]
+SOURCES = ["paged_attn.cu", "block_manager.cpp"]
+DEPS = ["paged_attn.cu", "block_manager.cpp", "decode.cuh", "prefix.cuh", "umma.cuh", "cache_ops.cuh", "ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+HEADERS = ["paged_attn.h", "block_manager.h"]
 
 
 def nvcc() -> str:
@@ -43,7 +44,7 @@ def up_to_date(out: str = LIB) -> bool:
     if not os.path.exists(out):
         return False
     t = os.path.getmtime(out)
-    deps = [os.path.join(CSRC, d) for d in DEPS] + [os.path.join(ROOT, "include", "paged_attn.h"), __file__]
+    deps = [os.path.join(CSRC, d) for d in DEPS] + [os.path.join(ROOT, "include", h) for h in HEADERS] + [__file__]
     return all(os.path.getmtime(d) <= t for d in deps)
 
 

@@ -291,6 +291,7 @@ PA_API const char* paged_attn_status_string(int status) {
     case PA_ERR_DEVICE_CHECK: return "device-side check fired";
     case PA_ERR_NO_MEMORY: return "out of device memory";
     case PA_ERR_SCRATCH_TOO_SMALL: return "split-KV partials exceed the no-alloc scratch (PA_NOALLOC_SCRATCH_BYTES)";
+    case PA_ERR_OUT_OF_BLOCKS: return "no free KV-cache block (block manager)";
     default: return "unknown status";
   }
 }
