@@ -475,14 +475,82 @@ def run_copy_blocks(args, world, rank, local):
     return 0
 
 
+def run_block_manager(args, world, rank, local):
+    """Host bookkeeping of a decode step with the native block manager, on the
+    256-sequence shared-prefix workload's shape: 8 prompts of 1024 tokens are
+    admitted through the prefix cache (the first one per group allocates, the
+    other 31 share its 64 blocks), every sequence gets its private suffix, and
+    then each step appends one token to all 256 sequences (slots and any
+    copy-on-write pairs) and exports the batch's block tables and lengths.
+    Host wall time (this is CPU code); the oracle's manager is timed on a
+    bounded number of steps beside it."""
+    import time
+    from oracle.block_manager import BlockManager as OracleBM  # CPU-baseline leg only
+    spec = wl.SPEC_BY_NAME["shared-prefix-fp8"]
+    lay = wl.build_layout(spec)
+    S, bs = spec.num_seqs, spec.block_size
+    nb = lay.num_blocks + S * (args.steps + args.warmup) // bs + 2 * S
+    bt_stride = lay.block_tables.shape[1] + (args.steps + args.warmup) // bs + 2
+
+    def admit(bm, alloc, append):
+        for g in range(spec.prefix_groups):
+            prompt = [g * 100000 + t for t in range(spec.prefix_tokens)]
+            for s in range(lay.group_start[g], lay.group_start[g + 1]):
+                alloc(bm, s, prompt)
+                append(bm, s, lay.seq_lens[s] - spec.prefix_tokens)
+
+    sids = list(range(S))
+
+    def run(step, steps):
+        t0 = time.perf_counter()
+        for _ in range(steps):
+            step()
+        return (time.perf_counter() - t0) / steps
+
+    nat = pab.BlockManager(nb, bs)
+    admit(nat, lambda bm, s, p: bm.allocate_with_prefix(s, p), lambda bm, s, n: bm.append_tokens(s, n))
+
+    def nat_step():  # one batched append call + the batch's tables
+        nat.append_batch(sids)
+        nat.build_batch(sids, bt_stride)
+
+    run(nat_step, args.warmup)
+    sec = run(nat_step, args.steps)
+    ora = OracleBM(nb, bs)
+    admit(ora, lambda bm, s, p: bm.allocate_with_prefix(s, p), lambda bm, s, n: bm.append_tokens(s, n))
+
+    def ora_step():
+        for s in sids:
+            ora.append_tokens(s, 1)
+        ora.build_batch(sids, bt_stride)
+
+    osteps = max(3, min(args.steps, 50))
+    osec = run(ora_step, osteps)
+    line = {"metric": "block-manager decode-step bookkeeping (append 1 token x 256 sequences + batch tables): "
+                      "steps/s", "value": 1.0 / sec, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * sec, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "int64", "data": "synthetic",
+            "config": {"workload": "shared-prefix-fp8 layout: 256 sequences, 8 prompts of 1024 tokens through the "
+                                   "prefix cache, private suffixes U[16,1024]", "blocks": nb, "bt_stride": bt_stride,
+                       "timing": "host wall clock (CPU code), through the ctypes binding"},
+            "cached_blocks": nat.cached_blocks(),
+            "cpu_baseline": {"value": 1.0 / osec, "unit": "steps/s", "cores": 1, "kind": "oracle",
+                             "sample": f"{osteps} steps of the same loop with the Python oracle manager"}}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    nat.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["decode-step", "copy-blocks"], default="decode-step",
-                    help="decode-step: the hot path (default); copy-blocks: block copies for COW / swap")
+    ap.add_argument("--op", choices=["decode-step", "copy-blocks", "block-manager"], default="decode-step",
+                    help="decode-step: the hot path (default); copy-blocks: block copies for COW / swap; "
+                         "block-manager: host bookkeeping of a decode step")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(wl.SPEC_BY_NAME))
     ap.add_argument("--partition", default="auto", help="auto | none | tokens per partition")
     ap.add_argument("--num-seqs", type=int, default=0, help="smaller batch of the same workload (profiling)")
@@ -499,6 +567,8 @@ def main():
             return run_reference(args, world, rank)
         if args.op == "copy-blocks":
             return run_copy_blocks(args, world, rank, local)
+        if args.op == "block-manager":
+            return run_block_manager(args, world, rank, local)
         return run_ours(args, world, rank, local)
     finally:
         if world > 1:

@@ -66,6 +66,14 @@ int pa_bm_ensure_capacity(pa_block_manager* bm, int64_t seq_id, int64_t required
 int pa_bm_append_tokens(pa_block_manager* bm, int64_t seq_id, int num_tokens, int64_t* slots,
                         int64_t* copy_pairs, int* num_copies, int* num_appended);
 
+/* One decode step's appends for a batch: one position for each of the n
+ * sequences, in order (as n calls of pa_bm_append_tokens with one token).
+ * slots [n]; copy_pairs [n][2] with the count in *num_copies; *num_appended
+ * = n on PA_OK, or the number of sequences served before PA_ERR_OUT_OF_BLOCKS
+ * (or before an unknown id, PA_ERR_INVALID_ARG). */
+int pa_bm_append_batch(pa_block_manager* bm, const int64_t* seq_ids, int n, int64_t* slots, int64_t* copy_pairs,
+                       int* num_copies, int* num_appended);
+
 /* Q18: child (a new id) gets a copy of the parent's table and length; every
  * block's count is raised by one. */
 int pa_bm_fork(pa_block_manager* bm, int64_t parent_id, int64_t child_id);

@@ -88,6 +88,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "pa_bm_free_sequence": (i, [_P, i64]),
         "pa_bm_ensure_capacity": (i, [_P, i64, i64]),
         "pa_bm_append_tokens": (i, [_P, i64, i, _P, _P, _P, _P]),
+        "pa_bm_append_batch": (i, [_P, _P, i, _P, _P, _P, _P]),
         "pa_bm_fork": (i, [_P, i64, i64]),
         "pa_bm_seq_len": (i, [_P, i64, _P]),
         "pa_bm_block_table": (i, [_P, i64, _P, i, _P]),
@@ -320,6 +321,21 @@ class BlockManager:
         if st not in (PA_OK, PA_ERR_OUT_OF_BLOCKS):
             self._check(st, "pa_bm_append_tokens")
         return st, list(slots[:na.value]), [(pairs[2 * k], pairs[2 * k + 1]) for k in range(nc.value)]
+
+    def append_batch(self, sids):
+        """One position for each sequence in ``sids``: returns (status, slots
+        as an int64 tensor, copy pairs as an int64 [k, 2] tensor); only the
+        sequences served before a PA_ERR_OUT_OF_BLOCKS are in the slots."""
+        n = len(sids)
+        ids = torch.as_tensor(sids, dtype=torch.int64)
+        slots = torch.empty((max(1, n),), dtype=torch.int64)
+        pairs = torch.empty((max(1, n), 2), dtype=torch.int64)
+        nc, na = ctypes.c_int(0), ctypes.c_int(0)
+        st = self.lib.pa_bm_append_batch(self.h, ids.data_ptr() if n else None, n, slots.data_ptr(),
+                                         pairs.data_ptr(), ctypes.byref(nc), ctypes.byref(na))
+        if st not in (PA_OK, PA_ERR_OUT_OF_BLOCKS):
+            self._check(st, "pa_bm_append_batch")
+        return st, slots[:na.value], pairs[:nc.value]
 
     def fork(self, parent: int, child: int) -> None:
         self._check(self.lib.pa_bm_fork(self.h, int(parent), int(child)), "pa_bm_fork")

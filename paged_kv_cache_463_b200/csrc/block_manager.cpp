@@ -227,6 +227,45 @@ PA_API int pa_bm_append_tokens(pa_block_manager* bm, int64_t seq_id, int num_tok
   return PA_OK;
 }
 
+PA_API int pa_bm_append_batch(pa_block_manager* bm, const int64_t* seq_ids, int n, int64_t* slots, int64_t* copy_pairs,
+                              int* num_copies, int* num_appended) {
+  BM_GUARD(bm);
+  if (n < 0 || (n > 0 && (!seq_ids || !slots || !copy_pairs)) || !num_copies || !num_appended)
+    return PA_ERR_INVALID_ARG;
+  *num_copies = 0;
+  *num_appended = 0;
+  const int bs = bm->block_size;
+  try {
+    for (int k = 0; k < n; ++k) {
+      Seq* s = bm->use(seq_ids[k]);
+      if (!s) return PA_ERR_INVALID_ARG;
+      const int64_t pos = s->len;
+      const int64_t lb = pos / bs, off = pos % bs;
+      if (lb == (int64_t)s->table.size()) {
+        s->table.push_back(bm->allocate());
+      } else if (bm->ref[s->table[lb]] > 1) {
+        const int32_t old = s->table[lb];
+        const int32_t fresh = bm->allocate();
+        if (off > 0) {
+          copy_pairs[2 * *num_copies] = old;
+          copy_pairs[2 * *num_copies + 1] = fresh;
+          ++*num_copies;
+        }
+        bm->decref(old);
+        s->table[lb] = fresh;
+      }
+      slots[k] = (int64_t)s->table[lb] * bs + off;
+      s->len = pos + 1;
+      *num_appended = k + 1;
+    }
+  } catch (const OutOfBlocks&) {
+    return PA_ERR_OUT_OF_BLOCKS;
+  } catch (const std::bad_alloc&) {
+    return PA_ERR_NO_MEMORY;
+  }
+  return PA_OK;
+}
+
 PA_API int pa_bm_fork(pa_block_manager* bm, int64_t parent_id, int64_t child_id) {
   BM_GUARD(bm);
   Seq* p = bm->use(parent_id);

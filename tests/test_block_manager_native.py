@@ -23,7 +23,7 @@ def _apply(o, n, op, args):
         try:
             return ("ok", fn())
         except OutOfBlocks as e:
-            return ("oob", (e.done, e.slots, [tuple(c) for c in e.copies]) if op == "append" else None)
+            return ("oob", (e.done, e.slots, [tuple(c) for c in e.copies]) if op in ("append", "append_batch") else None)
         except BlockManagerError:
             return ("err", None)
         except b.PagedAttnError as e:
@@ -50,6 +50,22 @@ def _apply(o, n, op, args):
             t, l = n.build_batch(*args)
             return t.tolist(), l.tolist()
         return run(lambda: o.build_batch(*args)), run(nat)
+    if op == "append_batch":
+        def orc():
+            slots, copies = [], []
+            for k, sid in enumerate(args[0]):
+                try:
+                    sl, cp = o.append_tokens(sid, 1)
+                except OutOfBlocks:
+                    raise OutOfBlocks("oob", k, slots, copies)
+                slots += sl
+                copies += cp
+            return slots, [tuple(c) for c in copies]
+        ro = run(orc)
+        st, slots, pairs = n.append_batch(args[0])
+        sl, pr = slots.tolist(), [tuple(x) for x in pairs.tolist()]
+        rn = ("ok", (sl, pr)) if st == b.PA_OK else ("oob", (len(sl), sl, pr))
+        return ro, rn
     if op == "append":
         ro = run(lambda: o.append_tokens(*args))
         try:
@@ -90,9 +106,11 @@ def test_random_calls_match_the_oracle(seed):
             op, args = "table", (rnd.choice(live),)
         elif r < 0.88:
             op, args = "len", (rnd.choice(live + [10 ** 6]),)
-        elif r < 0.94:
+        elif r < 0.91:
             k = rnd.randint(1, min(6, len(live)))
             op, args = "batch", (rnd.sample(live, k), rnd.choice([4, 8, 16]))
+        elif r < 0.94:
+            op, args = "append_batch", (rnd.sample(live, rnd.randint(1, len(live))),)
         else:
             op, args = "add", (rnd.choice(live),)  # duplicate id: an error on both sides
         ro, rn = _apply(o, n, op, args)
