@@ -129,3 +129,51 @@ def merge_partitions(parts) -> np.ndarray:
         num = num + w * o
         den = den + w
     return num / den
+
+
+def prefill_attention(query, key_cache, value_cache, block_tables, seq_lens, query_start, scale,
+                      q_dtype="f16", kv_dtype="f16", k_scale=1.0, v_scale=1.0, rows=None) -> np.ndarray:
+    """fp64 multi-query (prefill / chunked prefill) attention over the paged cache.
+
+    Page "5.KV Cache 管理 & PagedAttention", Q6 ``MHAWithCache`` prefill branch:
+    every query position attends causally (the ``torch.tril`` mask) to the
+    keys at its own and earlier positions; Q3.3 / Q19: the keys are the
+    sequence's cached K/V, read block by block through its table.  Sequence s
+    has seq_lens[s] cached tokens (this chunk's K/V already written) and the
+    query rows query_start[s] .. query_start[s+1]-1, which are its last
+    q_len = query_start[s+1] - query_start[s] positions: row i of the chunk is
+    position p = seq_lens[s] - q_len + i and sees keys 0..p.
+
+    query        [T, Hq, D] raw storage of ``q_dtype`` (T = query_start[-1])
+    rows         optional iterable of (t, h): compute only those (others NaN)
+    Returns [T, Hq, D] fp64.
+    """
+    T, Hq, D = query.shape
+    Hkv = key_cache.shape[2]
+    if Hq % Hkv != 0:
+        raise ValueError("num_heads must be a multiple of num_kv_heads")
+    q = dtypes.to_f64(query, q_dtype)
+    out = np.full((T, Hq, D), np.nan)
+    wanted = None
+    if rows is not None:
+        wanted = {}
+        for t, h in rows:
+            wanted.setdefault(int(t), []).append(int(h))
+    for s in range(len(seq_lens)):
+        a, b = int(query_start[s]), int(query_start[s + 1])
+        n = int(seq_lens[s])
+        if b <= a:
+            continue
+        if b - a > n:
+            raise ValueError("more query rows than cached tokens")
+        K = _kv_f64(key_cache, block_tables[s], n, kv_dtype, k_scale)
+        V = _kv_f64(value_cache, block_tables[s], n, kv_dtype, v_scale)
+        for t in range(a, b):
+            heads = range(Hq) if wanted is None else wanted.get(t, [])
+            p = n - (b - a) + (t - a)  # this row's position
+            for h in heads:
+                g = kv_head_of(h, Hq, Hkv)
+                x = float(scale) * (K[:p + 1, g, :] @ q[t, h])
+                w = softmax_weights(x)
+                out[t, h] = w @ V[:p + 1, g, :]
+    return out
