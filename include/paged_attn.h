@@ -211,6 +211,34 @@ int paged_attention_decode_shared_prefix(pa_ctx* ctx, void* out, const void* que
                                          float k_scale, float v_scale, void* stream);
 
 /*
+ * Multi-query paged attention: prefill and chunked prefill (page "5.KV Cache
+ * 管理 & PagedAttention", Q6 MHAWithCache prefill branch: each query position
+ * attends causally to the keys at its own and earlier positions; Q3.3 / Q19:
+ * blockwise over the paged cache through the block table, with an online
+ * softmax).  The chunk's K/V must already be in the cache (reshape_and_cache).
+ * Sequence s holds seq_lens[s] cached tokens; its query rows are
+ * query[query_start[s] .. query_start[s+1]) ([num_tokens, num_heads,
+ * head_dim], q_dtype), the sequence's last q_len = query_start[s+1] -
+ * query_start[s] positions, so row i is position p = seq_lens[s] - q_len + i:
+ *     out[row, h, :] = sum_{j <= p} softmax_j(scale * q[row,h,:] . K[s,j,:]) V[s,j,:]
+ * (q_len = seq_lens[s]: a whole prompt; 1: a decode step).  out has the
+ * query's shape and dtype.  query_start: device int32 [num_seqs + 1],
+ * non-decreasing, query_start[num_seqs] = num_tokens.  Host bounds:
+ * max_query_len >= every q_len, max_seq_len >= every seq_len (both <=
+ * max_blocks_per_seq * block_size).  A sequence with q_len > seq_len, or
+ * longer than max_seq_len / bt_stride * block_size, or whose query rows fall
+ * outside [0, num_tokens), sets PA_CHECK_SEQ_TOO_LONG (the rows of a
+ * sequence with q_len > seq_len or rows outside the array are not written).
+ * Arithmetic: 16-bit products accumulated in fp32 on the tensor cores (fp8
+ * caches decoded to f16 first); one rounding of the output.
+ * Returns PA_OK, PA_ERR_INVALID_ARG, PA_ERR_CUDA.
+ */
+int paged_attention_prefill(pa_ctx* ctx, void* out, const void* query, const void* key_cache, const void* value_cache,
+                            const int32_t* block_tables, int bt_stride, const int32_t* seq_lens,
+                            const int32_t* query_start, int num_seqs, int num_tokens, int max_query_len,
+                            int max_seq_len, float scale, float k_scale, float v_scale, void* stream);
+
+/*
  * Synchronise `stream`, read and clear the context's device check word.
  * Returns PA_OK when no check fired since the last call, PA_ERR_DEVICE_CHECK
  * otherwise (the bits are then in paged_attn_last_check_bits), PA_ERR_CUDA if

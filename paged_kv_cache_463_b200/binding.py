@@ -68,6 +68,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
         "paged_attention_decode": (i, [_P, _P, _P, _P, _P, _P, i, _P, i, i, f, f, f, _P]),
         "paged_attention_decode_shared_prefix": (i, [_P, _P, _P, _P, _P, _P, i, _P, i, i, _P, _P, i, i, i, f, f, f,
                                                      _P]),
+        "paged_attention_prefill": (i, [_P, _P, _P, _P, _P, _P, i, _P, _P, i, i, i, i, f, f, f, _P]),
         "paged_attn_get_error": (i, [_P, _P]),
         "paged_attn_last_check_bits": (i, [_P]),
         "paged_attn_status_string": (ctypes.c_char_p, [i]),
@@ -213,6 +214,18 @@ class PagedAttention:
             _ptr(group_prefix_len), group_prefix_len.shape[0], int(max_group_size), int(max_prefix_len),
             float(scale), float(k_scale), float(v_scale), _stream_ptr(stream))
         self._check(st, "paged_attention_decode_shared_prefix")
+
+    def paged_attention_prefill(self, out, query, key_cache, value_cache, block_tables, seq_lens, query_start,
+                                max_query_len: int, max_seq_len: int, scale: float, k_scale=1.0, v_scale=1.0,
+                                stream=None) -> None:
+        """Causal multi-query attention: the rows query[query_start[s]:query_start[s+1]]
+        are sequence s's last positions (device int32 tensors for the index arrays)."""
+        st = self.lib.paged_attention_prefill(self.ctx, _ptr(out), _ptr(query), _ptr(key_cache), _ptr(value_cache),
+                                              _ptr(block_tables), block_tables.stride(0), _ptr(seq_lens),
+                                              _ptr(query_start), query_start.shape[0] - 1, query.shape[0],
+                                              int(max_query_len), int(max_seq_len), float(scale), float(k_scale),
+                                              float(v_scale), _stream_ptr(stream))
+        self._check(st, "paged_attention_prefill")
 
     def paged_gather_kv(self, k_out, v_out, key_cache, value_cache, block_table_row, seq_len: int,
                         stream=None) -> None:

@@ -22,7 +22,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "lib")
 LIB = os.path.join(LIB_DIR, "libpaged_attn.so")
 SOURCES = ["paged_attn.cu", "block_manager.cpp"]
-DEPS = ["paged_attn.cu", "block_manager.cpp", "decode.cuh", "prefix.cuh", "umma.cuh", "cache_ops.cuh", "ptx.cuh"]
+DEPS = ["paged_attn.cu", "block_manager.cpp", "decode.cuh", "prefix.cuh", "prefill.cuh", "umma.cuh", "cache_ops.cuh", "ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 HEADERS = ["paged_attn.h", "block_manager.h"]
 

@@ -15,6 +15,7 @@
 #include "paged_attn.h"
 #include "cache_ops.cuh"
 #include "decode.cuh"
+#include "prefill.cuh"
 #include "prefix.cuh"
 
 #define PA_API extern "C" __attribute__((visibility("default")))
@@ -27,7 +28,8 @@ using pa::DecodeParams;
 struct KernelSet {
   const void* decode = nullptr;
   const void* merge = nullptr;
-  const void* prefix = nullptr;  // shared-prefix pass
+  const void* prefix = nullptr;   // shared-prefix pass
+  const void* prefill = nullptr;  // multi-query (prefill) attention, same CTA shape as the prefix pass
   int threads = 0;
   int ns = 0, stage_bytes = 0;  // ring shape (the rest of the layout depends on the call)
   int prefix_threads = 0, prefix_smem = 0;
@@ -42,6 +44,7 @@ KernelSet make_set() {
   k.decode = reinterpret_cast<const void*>(&pa::paged_decode_kernel<C>);
   k.merge = reinterpret_cast<const void*>(&pa::paged_decode_merge_kernel<typename C::Q, C::D, C::kBf16>);
   k.prefix = reinterpret_cast<const void*>(&pa::paged_prefix_kernel<P>);
+  k.prefill = reinterpret_cast<const void*>(&pa::paged_prefill_kernel<P>);
   k.threads = C::THREADS;
   k.ns = C::NS;
   k.stage_bytes = C::STAGE_BYTES;
@@ -58,7 +61,7 @@ cudaError_t pin_carveout(const void* fn) {
 }
 
 cudaError_t pin_all_carveouts(const KernelSet& ks) {
-  const void* fns[] = {ks.decode, ks.merge, ks.prefix, reinterpret_cast<const void*>(&pa::reshape_and_cache_copy_kernel),
+  const void* fns[] = {ks.decode, ks.merge, ks.prefix, ks.prefill, reinterpret_cast<const void*>(&pa::reshape_and_cache_copy_kernel),
                        reinterpret_cast<const void*>(&pa::reshape_and_cache_fp8_kernel<true>),
                        reinterpret_cast<const void*>(&pa::reshape_and_cache_fp8_kernel<false>),
                        reinterpret_cast<const void*>(&pa::paged_gather_kernel),
@@ -351,6 +354,8 @@ PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
     }
     if ((e = cudaFuncSetAttribute(ks.decode, cudaFuncAttributeMaxDynamicSharedMemorySize, optin)) != cudaSuccess ||
         (e = cudaFuncSetAttribute(ks.prefix, cudaFuncAttributeMaxDynamicSharedMemorySize, ks.prefix_smem)) !=
+            cudaSuccess ||
+        (e = cudaFuncSetAttribute(ks.prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, ks.prefix_smem)) !=
             cudaSuccess ||
         (e = pin_all_carveouts(ks)) != cudaSuccess) {
       st = cuda_fail(ctx, e, "cudaFuncSetAttribute");
@@ -667,6 +672,61 @@ PA_API int paged_attention_decode_shared_prefix(pa_ctx* ctx, void* out, const vo
   const PrefixArgs pre = {group_start, group_prefix_len, num_groups, max_group_size, max_prefix_len};
   return decode_impl(ctx, out, query, key_cache, value_cache, block_tables, bt_stride, seq_lens, num_seqs,
                      max_seq_len, scale, k_scale, v_scale, stream, &pre);
+}
+
+PA_API int paged_attention_prefill(pa_ctx* ctx, void* out, const void* query, const void* key_cache,
+                                   const void* value_cache, const int32_t* block_tables, int bt_stride,
+                                   const int32_t* seq_lens, const int32_t* query_start, int num_seqs, int num_tokens,
+                                   int max_query_len, int max_seq_len, float scale, float k_scale, float v_scale,
+                                   void* stream) {
+  if (!ctx) return PA_ERR_INVALID_ARG;
+  const pa_config& c = ctx->cfg;
+  if (num_seqs < 0 || num_seqs > 65535) return fail(ctx, PA_ERR_INVALID_ARG, "num_seqs outside [0, 65535]");
+  if (num_tokens < 0 || max_query_len < 0) return fail(ctx, PA_ERR_INVALID_ARG, "negative size");
+  if (num_seqs == 0 || num_tokens == 0 || max_query_len == 0) return PA_OK;
+  if (!out || !query || !key_cache || !value_cache || !block_tables || !seq_lens || !query_start)
+    return fail(ctx, PA_ERR_INVALID_ARG, "null pointer");
+  if (bt_stride < 1) return fail(ctx, PA_ERR_INVALID_ARG, "bt_stride < 1");
+  if (max_seq_len < 1 || max_seq_len > c.max_blocks_per_seq * c.block_size)
+    return fail(ctx, PA_ERR_INVALID_ARG, "max_seq_len outside [1, max_blocks_per_seq*block_size]");
+  if (max_query_len > max_seq_len) return fail(ctx, PA_ERR_INVALID_ARG, "max_query_len > max_seq_len");
+  if (!aligned(out, 16) || !aligned(query, 16) || !aligned(key_cache, 16) || !aligned(value_cache, 16) ||
+      !aligned(block_tables, 4) || !aligned(seq_lens, 4) || !aligned(query_start, 4))
+    return fail(ctx, PA_ERR_INVALID_ARG, "misaligned pointer");
+  if (!std::isfinite(scale)) return fail(ctx, PA_ERR_INVALID_ARG, "scale not finite");
+  const bool fp8 = c.kv_dtype == PA_FP8_E4M3;
+  if (fp8 && !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
+    return fail(ctx, PA_ERR_INVALID_ARG, "fp8 scales must be finite and > 0");
+  cudaSetDevice(ctx->device);
+  CUtensorMap mk, mv;
+  int st = tensor_map(ctx, key_cache, &mk);
+  if (st != PA_OK) return st;
+  if ((st = tensor_map(ctx, value_cache, &mv)) != PA_OK) return st;
+  pa::PrefillParams p;
+  p.out = out;
+  p.query = query;
+  p.block_tables = block_tables;
+  p.seq_lens = seq_lens;
+  p.query_start = query_start;
+  p.err = ctx->err;
+  p.num_seqs = num_seqs;
+  p.num_tokens = num_tokens;
+  p.bt_stride = bt_stride;
+  p.num_heads = c.num_heads;
+  p.group = c.num_heads / c.num_kv_heads;
+  p.head_splits = (p.group + pa::kNH - 1) / pa::kNH;
+  p.num_blocks = c.num_blocks;
+  p.max_blocks = (max_seq_len + c.block_size - 1) / c.block_size;
+  p.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
+  p.v_scale = fp8 ? v_scale : 1.0f;
+  const int hmax = p.group < pa::kNH ? p.group : pa::kNH;
+  const int tpb = pa::kPrefixRows / hmax;  // query tokens per CTA (fewest: the widest KV unit)
+  const dim3 grid((unsigned)((max_query_len + tpb - 1) / tpb), (unsigned)(c.num_kv_heads * p.head_splits),
+                  (unsigned)num_seqs);
+  void* args[] = {&mk, &mv, &p};
+  cudaError_t e = cudaLaunchKernel(ctx->ks.prefill, grid, dim3(ctx->ks.prefix_threads), args, ctx->ks.prefix_smem,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? PA_OK : cuda_fail(ctx, e, "prefill launch");
 }
 
 PA_API int paged_attn_get_error(pa_ctx* ctx, void* stream) {

@@ -129,10 +129,27 @@ __device__ __forceinline__ int group_prefix_blocks(const PrefixParams& p, int g,
   return len / kBS;
 }
 
-template <class C>
-__global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
-    paged_prefix_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                        const PrefixParams p) {
+// A block range's contribution to 128 stacked query rows on the tensor
+// cores (the roles described at the top of this file).  `job` names the
+// range: the block-table entries of its nb blocks, the number of its tokens
+// that exist (later ones are masked and their V zeroed) and the KV head.
+// `rows` maps the CTA's 128 rows to queries and outputs:
+//   const void* q_row(r)          query row (16-bit, D values) or nullptr (zero row)
+//   int limit(r)                  keys of the range row r sees (a prefix of it)
+//   void store(r, c0, v[16])      normalised output dims c0..c0+15 (times v_scale)
+//   void store_ml(r, m, l)        the row's max (log2 units) and sum
+// Called by all 320 threads of the CTA; returns after tensor memory is freed.
+struct StackedJob {
+  const int32_t* table;  // nb block ids
+  int nb;
+  int kv_valid;          // tokens 0..kv_valid-1 of the range exist
+  int kvh;
+  int num_blocks;        // physical pool size (ids outside it are flagged and replaced by block 0)
+};
+
+template <class C, class Rows>
+__device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const CUtensorMap& tmV, const StackedJob& job,
+                                                  const Rows& rows, float scale_log2, float v_scale, int* err) {
   using Q = typename C::Q;
   constexpr int D = C::D, NS = C::NS;
   extern __shared__ uint8_t smem_dyn[];
@@ -145,68 +162,8 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
   volatile int* dead = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   volatile int* converted = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  const int g = blockIdx.z;
-  const int y = blockIdx.y / p.row_blocks;
-  const int rb = blockIdx.y - y * p.row_blocks;
-  const int chunk = blockIdx.x;
-  const int first = p.group_start[g], members = p.group_start[g + 1] - first;
-  const int pblk = group_prefix_blocks(p, g, first, members);
-
-  if (blockIdx.x == 0 && blockIdx.y == 0) {
-    // One CTA per group: the group's description, and the suffix offsets of
-    // its members (plus those of the sequences before the first group / from
-    // the last group's end on, which have no shared prefix).
-    __shared__ int s_ok;
-    const bool range_ok = first >= 0 && members >= 0 && first + members <= p.num_seqs;
-    if (threadIdx.x == 0) {
-      s_ok = 1;
-      const int len = p.group_prefix_len[g];
-      if (!range_ok || (len != 0 && pblk == 0)) atomicOr(p.err, kCheckBadPrefix);
-    }
-    __syncthreads();
-    // every member is at least as long as the prefix and maps it to the same blocks
-    for (int k = threadIdx.x; k < members * pblk; k += blockDim.x) {
-      const int m = k / pblk, b = k - m * pblk;
-      const int s = first + m;
-      bool ok = p.seq_lens[s] >= pblk * kBS;
-      if (m > 0)
-        ok = ok && __ldg(p.block_tables + (size_t)s * p.bt_stride + b) ==
-                       __ldg(p.block_tables + (size_t)first * p.bt_stride + b);
-      if (!ok) s_ok = 0;
-    }
-    __syncthreads();
-    if (threadIdx.x == 0 && !s_ok) atomicOr(p.err, kCheckBadPrefix);
-    const int skip = s_ok ? pblk : 0;
-    if (range_ok)
-      for (int m = threadIdx.x; m < members; m += blockDim.x) p.seq_skip[first + m] = skip;
-    if (g == 0) {
-      const int lo = min(max(first, 0), p.num_seqs);
-      for (int s = threadIdx.x; s < lo; s += blockDim.x) p.seq_skip[s] = 0;
-    }
-    if (g == p.num_groups - 1) {
-      const int hi = max(min(first + members, p.num_seqs), 0);
-      for (int s = hi + threadIdx.x; s < p.num_seqs; s += blockDim.x) p.seq_skip[s] = 0;
-    }
-  }
-
-  const int kvh = y / p.head_splits;
-  const int hs = y - kvh * p.head_splits;
-  const int head0 = kvh * p.group + hs * kNH;
-  const int hpu = min(kNH, p.group - hs * kNH);  // query heads of this KV unit
-  const int rows = members * hpu;                 // (member, head) rows of this KV unit
-  const int b0 = chunk * kPrefixChunkBlocks;
-  const int nb = min(pblk, b0 + kPrefixChunkBlocks) - b0;
-  if (nb <= 0 || rb * kPrefixRows >= rows) return;
-
-  // query row r of this CTA -> (sequence, head); false past the group's rows
-  auto row_of = [&](int r, int& s, int& h) -> bool {
-    const int idx = rb * kPrefixRows + r;
-    if (idx >= rows) return false;
-    s = first + idx / hpu;
-    h = head0 + idx % hpu;
-    return true;
-  };
+  const int nb = job.nb;
+  (void)sizeof(Q);
 
   // ---- set-up: barriers, tensor memory, the query tile (128-byte swizzled)
   constexpr int B = C::B, SB = C::SB, T = C::T;
@@ -230,13 +187,10 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
   if (warp < 4) {
     const int r = threadIdx.x;
-    int s = 0, h = 0;
-    const bool ok = row_of(r, s, h);
-    const uint4* src = reinterpret_cast<const uint4*>(reinterpret_cast<const Q*>(p.query) +
-                                                      ((size_t)s * p.num_heads + h) * D);
+    const uint4* src = reinterpret_cast<const uint4*>(rows.q_row(r));
 #pragma unroll 4
     for (int c = 0; c < D / 8; ++c) {
-      const uint4 v = ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 v = src ? src[c] : make_uint4(0u, 0u, 0u, 0u);
       *reinterpret_cast<uint4*>(smem + C::OFF_Q + C::sw128(kPrefixRows, r, 16 * c)) = v;
     }
     fence_proxy_async_smem();
@@ -250,28 +204,30 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
   auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
     if (*dead) return false;
     if (mbar_wait(bar, parity)) return true;
-    atomicOr(p.err, kCheckWaitTimeout);
+    atomicOr(err, kCheckWaitTimeout);
     *dead = 1;
     return false;
   };
 
   if (warp == 8) {
     // ---------------------------------------------------------------- TMA producer
-    int my = 0;
-    if (lane < nb) {
-      my = __ldg(p.block_tables + (size_t)first * p.bt_stride + b0 + lane);
-      if (my < 0 || my >= p.num_blocks) {
-        atomicOr(p.err, kCheckBadBlock);
-        my = 0;
-      }
-    }
-    int issued = 0;
+    int issued = 0, my = 0;
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
     }
     for (int i = 0; i < nb; ++i) {
-      const int phys = __shfl_sync(0xffffffffu, my, i);
+      if ((i & 31) == 0) {  // the next 32 table entries, one per lane
+        my = 0;
+        if (i + lane < nb) {
+          my = __ldg(job.table + i + lane);
+          if (my < 0 || my >= job.num_blocks) {
+            atomicOr(err, kCheckBadBlock);
+            my = 0;
+          }
+        }
+      }
+      const int phys = __shfl_sync(0xffffffffu, my, i & 31);
       if (lane == 0) {
         const int st = i % NS;
         if (i >= NS && !wait(empty0 + 8 * st, ((i / NS) - 1) & 1)) break;
@@ -279,7 +235,7 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
         const uint32_t kdst = base + C::OFF_RING + st * C::STAGE_BYTES;
 #pragma unroll
         for (int sub = 0; sub < C::SUBTILES; ++sub) {
-          const int x = kvh * D + sub * (128 / (int)sizeof(typename C::KV));
+          const int x = job.kvh * D + sub * (128 / (int)sizeof(typename C::KV));
           tma_load_2d(kdst + sub * kBS * 128, &tmK, x, phys * kBS, full0 + 8 * st);
           tma_load_2d(kdst + C::TILE_BYTES + sub * kBS * 128, &tmV, x, phys * kBS, full0 + 8 * st);
         }
@@ -355,6 +311,10 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
             bb[0] = x1.x; bb[1] = x1.y; bb[2] = x1.z; bb[3] = x1.w;
           }
           const int tt = 16 * j + 2 * pr;
+          // keys past the range's valid tokens: P is 0 there and the cache slot may hold anything
+          const int kidx = 16 * i + 2 * pr;
+          if (kidx >= job.kv_valid) a[0] = a[1] = a[2] = a[3] = 0u;
+          if (kidx + 1 >= job.kv_valid) bb[0] = bb[1] = bb[2] = bb[3] = 0u;
           uint8_t* dst = vt + c * C::CM_STRIDE + (tt >> 3) * 128 + (tt & 7) * 2;
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -416,7 +376,7 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
         if (progress) {
           idle_since = clock64();
         } else if (clock64() - idle_since > kWaitLimitCycles) {
-          atomicOr(p.err, kCheckWaitTimeout);
+          atomicOr(err, kCheckWaitTimeout);
           *dead = 1;
         }
       }
@@ -428,6 +388,7 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
     // ---------------------------------------------------------------- softmax (warps 0..3)
     const int r = threadIdx.x;
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
+    const int lim = min(rows.limit(r), job.kv_valid);  // keys this row sees, from the range start
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int u = 0; u < nsteps && ok; ++u) {
@@ -444,11 +405,11 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
         for (int j = 0; j < 16; ++j) x[c0 + j] = __uint_as_float(sv[j]);
       }
       tmem_wait_ld();
-      const int valid = min(T, (nb - u * SB) * kBS);  // tokens of the prefix in this step
+      const int valid = min(T, lim - u * T);  // keys of this step the row sees
       float bm = -INFINITY;
 #pragma unroll
       for (int j = 0; j < T; ++j) {
-        x[j] = j < valid ? x[j] * p.scale_log2 : -INFINITY;
+        x[j] = j < valid ? x[j] * scale_log2 : -INFINITY;
         bm = fmaxf(bm, x[j]);
       }
       // lazy rescaling: move the reference max (and rescale l, O) only when
@@ -499,25 +460,18 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
     if (ok) ok = wait(pvdone0 + 8 * ((nsteps - 1) % B), ((nsteps - 1) / B) & 1);  // the last P V
     if (ok) {
       tc_fence_after();
-      int s = 0, h = 0;
-      const bool valid = row_of(r, s, h);
-      const float inv = l > 0.f ? p.v_scale / l : 0.f;
-      const size_t row = ((size_t)s * p.num_heads + h) * p.max_chunks + chunk;
-      float* dst = p.pre_o + row * D;
+      const float inv = l > 0.f ? v_scale / l : 0.f;
 #pragma unroll 1
       for (int c0 = 0; c0 < D; c0 += 16) {
         uint32_t o[16];
         tmem_ld16(trow + C::O_COL + c0, o);
         tmem_wait_ld();
-        if (valid) {
+        float v[16];
 #pragma unroll
-          for (int j = 0; j < 16; j += 4)
-            *reinterpret_cast<float4*>(dst + c0 + j) =
-                make_float4(__uint_as_float(o[j]) * inv, __uint_as_float(o[j + 1]) * inv,
-                            __uint_as_float(o[j + 2]) * inv, __uint_as_float(o[j + 3]) * inv);
-        }
+        for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(o[j]) * inv;
+        rows.store(r, c0, v);
       }
-      if (valid) *reinterpret_cast<float2*>(p.pre_ml + row * 2) = make_float2(m, l);
+      rows.store_ml(r, m, l);
     }
   }
 
@@ -529,6 +483,102 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }
+}
+
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
+    paged_prefix_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const PrefixParams p) {
+  using Q = typename C::Q;
+  constexpr int D = C::D;
+
+  const int g = blockIdx.z;
+  const int y = blockIdx.y / p.row_blocks;
+  const int rb = blockIdx.y - y * p.row_blocks;
+  const int chunk = blockIdx.x;
+  const int first = p.group_start[g], members = p.group_start[g + 1] - first;
+  const int pblk = group_prefix_blocks(p, g, first, members);
+
+  if (blockIdx.x == 0 && blockIdx.y == 0) {
+    // One CTA per group: the group's description, and the suffix offsets of
+    // its members (plus those of the sequences before the first group / from
+    // the last group's end on, which have no shared prefix).
+    __shared__ int s_ok;
+    const bool range_ok = first >= 0 && members >= 0 && first + members <= p.num_seqs;
+    if (threadIdx.x == 0) {
+      s_ok = 1;
+      const int len = p.group_prefix_len[g];
+      if (!range_ok || (len != 0 && pblk == 0)) atomicOr(p.err, kCheckBadPrefix);
+    }
+    __syncthreads();
+    // every member is at least as long as the prefix and maps it to the same blocks
+    for (int k = threadIdx.x; k < members * pblk; k += blockDim.x) {
+      const int m = k / pblk, b = k - m * pblk;
+      const int s = first + m;
+      bool ok = p.seq_lens[s] >= pblk * kBS;
+      if (m > 0)
+        ok = ok && __ldg(p.block_tables + (size_t)s * p.bt_stride + b) ==
+                       __ldg(p.block_tables + (size_t)first * p.bt_stride + b);
+      if (!ok) s_ok = 0;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !s_ok) atomicOr(p.err, kCheckBadPrefix);
+    const int skip = s_ok ? pblk : 0;
+    if (range_ok)
+      for (int m = threadIdx.x; m < members; m += blockDim.x) p.seq_skip[first + m] = skip;
+    if (g == 0) {
+      const int lo = min(max(first, 0), p.num_seqs);
+      for (int s = threadIdx.x; s < lo; s += blockDim.x) p.seq_skip[s] = 0;
+    }
+    if (g == p.num_groups - 1) {
+      const int hi = max(min(first + members, p.num_seqs), 0);
+      for (int s = hi + threadIdx.x; s < p.num_seqs; s += blockDim.x) p.seq_skip[s] = 0;
+    }
+  }
+
+  const int kvh = y / p.head_splits;
+  const int hs = y - kvh * p.head_splits;
+  const int head0 = kvh * p.group + hs * kNH;
+  const int hpu = min(kNH, p.group - hs * kNH);  // query heads of this KV unit
+  const int rows = members * hpu;                 // (member, head) rows of this KV unit
+  const int b0 = chunk * kPrefixChunkBlocks;
+  const int nb = min(pblk, b0 + kPrefixChunkBlocks) - b0;
+  if (nb <= 0 || rb * kPrefixRows >= rows) return;
+
+  // query row r of this CTA: (member, head) pair idx = rb * 128 + r of the
+  // group (heads fastest); partials go to prefix chunk `chunk`
+  struct Rows {
+    const PrefixParams* p;
+    int rb, rows, first, hpu, head0, chunk;
+    __device__ bool at(int r, int& s, int& h) const {
+      const int idx = rb * kPrefixRows + r;
+      if (idx >= rows) return false;
+      s = first + idx / hpu;
+      h = head0 + idx % hpu;
+      return true;
+    }
+    __device__ const void* q_row(int r) const {
+      int s, h;
+      if (!at(r, s, h)) return nullptr;
+      return reinterpret_cast<const Q*>(p->query) + ((size_t)s * p->num_heads + h) * D;
+    }
+    __device__ int limit(int) const { return 1 << 30; }  // whole blocks: every key of the range
+    __device__ size_t row(int s, int h) const { return ((size_t)s * p->num_heads + h) * p->max_chunks + chunk; }
+    __device__ void store(int r, int c0, const float (&v)[16]) const {
+      int s, h;
+      if (!at(r, s, h)) return;
+      float* dst = p->pre_o + row(s, h) * D + c0;
+#pragma unroll
+      for (int j = 0; j < 16; j += 4) *reinterpret_cast<float4*>(dst + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+    }
+    __device__ void store_ml(int r, float m, float l) const {
+      int s, h;
+      if (at(r, s, h)) *reinterpret_cast<float2*>(p->pre_ml + row(s, h) * 2) = make_float2(m, l);
+    }
+  };
+  const Rows rw{&p, rb, rows, first, hpu, head0, chunk};
+  const StackedJob job{p.block_tables + (size_t)first * p.bt_stride + b0, nb, nb * kBS, kvh, p.num_blocks};
+  stacked_attention<C>(tmK, tmV, job, rw, p.scale_log2, p.v_scale, p.err);
 }
 
 }  // namespace pa
