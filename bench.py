@@ -542,15 +542,125 @@ def run_block_manager(args, world, rank, local):
     return 0
 
 
+def run_prefill(args, world, rank, local):
+    """Prefill step: write the prompts' K/V into the paged cache
+    (reshape_and_cache) and run causal multi-query paged attention over them
+    (paged_attention_prefill).  Workload: 16 prompts x 2048 tokens of the GQA
+    70B-like layer (64 query / 8 KV heads, head_dim 128, bf16), blocks
+    shuffled across the pool.  Metric: attention TFLOP/s counting the causal
+    half only, 4 * Hq * D * L(L+1)/2 per sequence."""
+    import numpy as np
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA GPU")
+    from paged_kv_cache_463_b200 import build
+    build.build()
+    S, L = (args.num_seqs or 16), 2048
+    spec = wl.WorkloadSpec("prefill-gqa-70b-like", S, 64, 8, 128, 16, "bf16", "bf16", L, L, seed=1010,
+                           description=f"{S} prompts x {L} tokens, 64 q / 8 kv heads, head_dim 128, bf16")
+    dev = f"cuda:{local}"
+    w = wl.make_workload(spec, dev)
+    T = S * L
+    gen = torch.Generator(device=dev).manual_seed(1010)
+    q = torch.randn((T, spec.num_heads, spec.head_dim), generator=gen, device=dev).bfloat16()
+    k_new = torch.randn((T, spec.num_kv_heads, spec.head_dim), generator=gen, device=dev).bfloat16()
+    v_new = torch.randn_like(k_new)
+    # every prompt position's slot, from the block tables
+    bt = w.block_tables.long()
+    pos = torch.arange(L, device=dev)
+    slots = (bt[:, pos // 16] * 16 + pos % 16).reshape(-1)
+    qstart = torch.arange(0, T + 1, L, dtype=torch.int32, device=dev)
+    pa = pab.PagedAttention(spec.num_heads, spec.num_kv_heads, spec.head_dim, w.num_blocks, q_dtype="bf16",
+                            kv_dtype="bf16", max_num_seqs=S, max_blocks_per_seq=w.block_tables.shape[1], device=local)
+    kc, vc = w.key_cache, w.value_cache
+    out = torch.empty_like(q)
+    stream = torch.cuda.current_stream()
+    flops = 4.0 * spec.num_heads * spec.head_dim * S * L * (L + 1) / 2
+
+    def step():
+        pa.reshape_and_cache(k_new, v_new, kc, vc, slots, stream=stream)
+        pa.paged_attention_prefill(out, q, kc, vc, w.block_tables, w.seq_lens, qstart, L, L, w.scale, stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if pa.get_error() != 0:
+        raise SystemExit("device check fired during warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for a, m, e in ev:
+            a.record(stream)
+            pa.reshape_and_cache(k_new, v_new, kc, vc, slots, stream=stream)
+            m.record(stream)
+            pa.paged_attention_prefill(out, q, kc, vc, w.block_tables, w.seq_lens, qstart, L, L, w.scale,
+                                       stream=stream)
+            e.record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    total_ms = max_over_ranks(t0.elapsed_time(t1), world)
+    if pa.get_error() != 0:
+        raise SystemExit("device check fired during the timed region")
+    attn_ms = sum(m.elapsed_time(e) for _, m, e in ev) / args.steps
+    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    achieved = flops / (attn_ms * 1e-3) / 1e12
+    peaks = json.load(open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "MEASURED_PEAKS.json")))
+    peak = peaks["bf16_tflops"]
+    line = {"metric": "paged prefill attention: TFLOP/s (causal half) and tokens/s", "value": value,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": spec.name, "description": spec.description, "num_seqs": S, "prompt_tokens": L,
+                       "step": "reshape_and_cache of every prompt token + paged_attention_prefill",
+                       "l2": "K/V and queries (1.1 GB) larger than L2, no flush"},
+            "tokens_per_s": world * T * args.steps / (total_ms * 1e-3),
+            "attention_ms": attn_ms,
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "paged_prefill_kernel",
+                         "peak_kind": "measured cuBLAS bf16 burst (MEASURED_PEAKS.json bf16_tflops)"},
+            "gpu_launches": 2 * args.steps, "clocks": clk.summary()}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import time
+        from oracle import attention  # CPU-baseline leg only
+        rows = [(t, h) for t in range(L - 4, L) for h in range(spec.num_heads)]
+        hq = q.cpu().view(torch.int16).numpy().view(np.uint16)
+        t_a = time.perf_counter()
+        attention.prefill_attention(hq[:L], raw_np(kc), raw_np(vc), w.block_tables.cpu().numpy()[:1],
+                                    w.seq_lens.cpu().numpy()[:1], np.array([0, L]), w.scale, q_dtype="bf16",
+                                    kv_dtype="bf16", rows=rows)
+        el = time.perf_counter() - t_a
+        f = 4.0 * spec.num_heads * spec.head_dim * sum(t + 1 for t in range(L - 4, L))
+        line["cpu_baseline"] = {"value": f / el / 1e12, "unit": "TFLOP/s", "cores": 1, "kind": "oracle",
+                                "sample": f"the last 4 positions x {spec.num_heads} heads of one 2048-token prompt"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    pa.close()
+    return 0
+
+
+def raw_np(t):
+    import numpy as np
+    t = t.detach().cpu().contiguous()
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).numpy().view(np.uint16)
+    if t.dtype == torch.float8_e4m3fn:
+        return t.view(torch.uint8).numpy()
+    return t.numpy()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--op", choices=["decode-step", "copy-blocks", "block-manager"], default="decode-step",
+    ap.add_argument("--op", choices=["decode-step", "copy-blocks", "block-manager", "prefill"], default="decode-step",
                     help="decode-step: the hot path (default); copy-blocks: block copies for COW / swap; "
-                         "block-manager: host bookkeeping of a decode step")
+                         "block-manager: host bookkeeping of a decode step; prefill: causal multi-query attention")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(wl.SPEC_BY_NAME))
     ap.add_argument("--partition", default="auto", help="auto | none | tokens per partition")
     ap.add_argument("--num-seqs", type=int, default=0, help="smaller batch of the same workload (profiling)")
@@ -569,6 +679,8 @@ def main():
             return run_copy_blocks(args, world, rank, local)
         if args.op == "block-manager":
             return run_block_manager(args, world, rank, local)
+        if args.op == "prefill":
+            return run_prefill(args, world, rank, local)
         return run_ours(args, world, rank, local)
     finally:
         if world > 1:

@@ -76,23 +76,28 @@ struct PrefixCfg {
   static constexpr int NS = NS_;   // ring stages (blocks)
   static constexpr int SB = SB_;   // blocks per step
   static constexpr int T = SB * kBS;  // tokens per step (the S MMA's N, the P V MMA's K)
-  static constexpr int B = 2;      // step buffers (operands, S, P)
+  static constexpr int B = 2;      // step buffers (S, P, and the fp8 operands)
   static constexpr bool kFp8 = sizeof(KV) == 1;
   static constexpr bool kBf16 = std::is_same<Q, __nv_bfloat16>::value;
   static constexpr int ROW_BYTES = D * (int)sizeof(KV);
   static constexpr int SUBTILES = ROW_BYTES / 128;
   static constexpr int TILE_BYTES = kBS * ROW_BYTES;
-  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;
+  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // K + V of one block
+  // The K and V rings are each [SUBTILES][NS][16 rows x 128 B] (TMA 128-byte
+  // swizzle): the SB consecutive stages of a step hold its tokens' rows of one
+  // sub-tile contiguously, so a 16-bit ring is itself the MMA operand
+  // (K K-major, V MN-major; 8-row atoms 1024 bytes apart).
+  static constexpr int RING_SUB = NS * kBS * 128;      // bytes between a ring's sub-tiles
   static constexpr int Q_BYTES = kPrefixRows * D * 2;  // 128-byte swizzled, D/64 sub-tiles of 128 rows
-  static constexpr int KF_BYTES = T * D * 2;           // 128-byte swizzled, D/64 sub-tiles of T rows
-  static constexpr int VT_BYTES = D * T * 2;           // no swizzle: (8 dims x 8 tokens) core matrices
+  static constexpr int F_BYTES = kFp8 ? T * D * 2 : 0;  // fp8 only: a step's K or V as f16, D/64 sub-tiles of T rows
   static constexpr int P_BYTES = kPrefixRows * T * 2;  // no swizzle: (8 rows x 8 tokens) core matrices
-  static constexpr int CM_STRIDE = T * 16;             // bytes between 8-row groups of V^T and P
+  static constexpr int CM_STRIDE = T * 16;             // bytes between 8-row groups of P
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_RING = OFF_Q + Q_BYTES;
-  static constexpr int OFF_KF = OFF_RING + NS * STAGE_BYTES;  // [B]
-  static constexpr int OFF_VT = OFF_KF + B * KF_BYTES;        // [B]
-  static constexpr int OFF_P = OFF_VT + B * VT_BYTES;         // [B]
+  static constexpr int OFF_RING_K = OFF_Q + Q_BYTES;
+  static constexpr int OFF_RING_V = OFF_RING_K + NS * TILE_BYTES;
+  static constexpr int OFF_KF = OFF_RING_V + NS * TILE_BYTES;  // [B] (fp8)
+  static constexpr int OFF_VF = OFF_KF + B * F_BYTES;          // [B] (fp8)
+  static constexpr int OFF_P = OFF_VF + B * F_BYTES;           // [B]
   static constexpr int OFF_BAR = OFF_P + B * P_BYTES;
   // full[NS] empty[NS] conv_full[B] s_full[B] p_full[B] pv_done[B] fin
   static constexpr int NBARS = 2 * NS + 4 * B + 1;
@@ -109,11 +114,17 @@ struct PrefixCfg {
   static_assert(ROW_BYTES % 128 == 0, "rows must be whole 128-byte swizzle spans");
   static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
   static_assert(T % 16 == 0 && T <= 256, "step tokens");
+  static_assert(NS % SB == 0, "a step's blocks occupy consecutive ring stages");
   static_assert(!kFp8 || std::is_same<Q, __half>::value, "fp8 caches pair with fp16 queries");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   // byte offset of (row, byte-in-row) in a 128-byte-swizzled tile of `rows` rows
   __device__ static uint32_t sw128(int rows, int row, int byte) {
     return (uint32_t)((byte >> 7) * (rows * 128) + row * 128 + (((((byte & 127) >> 4) ^ (row & 7)) << 4) | (byte & 15)));
+  }
+  // byte offset of (row, byte-in-row) of ring stage st, in a K or V ring
+  __device__ static uint32_t ring(int st, int row, int byte) {
+    return (uint32_t)((byte >> 7) * RING_SUB + st * (kBS * 128) + row * 128 +
+                      (((((byte & 127) >> 4) ^ (row & 7)) << 4) | (byte & 15)));
   }
 };
 
@@ -171,7 +182,8 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
       mbar_init(full0 + 8 * i, 1);
-      mbar_init(empty0 + 8 * i, 4);  // the four staging warps
+      // released by the four converting warps (fp8) or by the tensor core (16-bit: tcgen05.commit after P V)
+      mbar_init(empty0 + 8 * i, C::kFp8 ? 4 : 1);
     }
     for (int i = 0; i < B; ++i) {
       mbar_init(convf0 + 8 * i, 4);
@@ -232,12 +244,12 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
         const int st = i % NS;
         if (i >= NS && !wait(empty0 + 8 * st, ((i / NS) - 1) & 1)) break;
         mbar_arrive_expect_tx(full0 + 8 * st, C::STAGE_BYTES);
-        const uint32_t kdst = base + C::OFF_RING + st * C::STAGE_BYTES;
 #pragma unroll
         for (int sub = 0; sub < C::SUBTILES; ++sub) {
           const int x = job.kvh * D + sub * (128 / (int)sizeof(typename C::KV));
-          tma_load_2d(kdst + sub * kBS * 128, &tmK, x, phys * kBS, full0 + 8 * st);
-          tma_load_2d(kdst + C::TILE_BYTES + sub * kBS * 128, &tmV, x, phys * kBS, full0 + 8 * st);
+          const uint32_t off = sub * C::RING_SUB + st * (kBS * 128);
+          tma_load_2d(base + C::OFF_RING_K + off, &tmK, x, phys * kBS, full0 + 8 * st);
+          tma_load_2d(base + C::OFF_RING_V + off, &tmV, x, phys * kBS, full0 + 8 * st);
         }
         ++issued;
       }
@@ -247,85 +259,59 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
       for (int i = *converted; i < issued; ++i) mbar_wait(full0 + 8 * (i % NS), (i / NS) & 1);
   } else if (warp >= 4 && warp < 8) {
     // ---------------------------------------------------------------- operand staging
+    // fp8: convert each block's K and V rows to f16 (row for row, 128-byte
+    // swizzled, the step's SB blocks stacked) and release the ring stage.
+    // 16-bit: the ring is the operand; only V rows past the range's valid
+    // keys are zeroed (P is 0 there, and 0 * garbage could be NaN; the stage
+    // of a block past the range still holds an older block).
     const int t = threadIdx.x - 128;
     for (int u = 0; u < nsteps; ++u) {
       const int cb = u % B;
-      if (u >= B && !wait(pvdone0 + 8 * cb, ((u - B) / B) & 1)) break;  // step buffer cb free
-      uint8_t* kf = smem + C::OFF_KF + cb * C::KF_BYTES;
-      uint8_t* vt = smem + C::OFF_VT + cb * C::VT_BYTES;
+      if (u >= B && !wait(pvdone0 + 8 * cb, ((u - B) / B) & 1)) break;  // step u - B's operands are free
       bool stop = false;
 #pragma unroll 1
       for (int j = 0; j < SB; ++j) {
-        const int i = u * SB + j;  // block of the chunk
-        if (i >= nb) {
-          // past the prefix: zero V^T (P is 0 there, and 0 * garbage could be NaN)
-          for (int it = t; it < D; it += 128) {
-            uint8_t* dst = vt + (it >> 3) * C::CM_STRIDE + ((16 * j + 2 * (it & 7)) >> 3) * 128 + ((2 * (it & 7)) & 7) * 2;
-#pragma unroll
-            for (int q = 0; q < 8; ++q) *reinterpret_cast<uint32_t*>(dst + q * 16) = 0u;
-          }
-          continue;
-        }
+        const int i = u * SB + j;  // block of the range
         const int st = i % NS;
-        if (!wait(full0 + 8 * st, (i / NS) & 1)) {
+        const int valid = min(kBS, max(0, job.kv_valid - i * kBS));  // tokens of this block that exist
+        if (i < nb && !wait(full0 + 8 * st, (i / NS) & 1)) {
           stop = true;
           break;
         }
-        const uint32_t ks = base + C::OFF_RING + st * C::STAGE_BYTES, vs = ks + C::TILE_BYTES;
-        // K rows 16j..16j+15 of the step's tile
         if constexpr (C::kFp8) {
-          for (int k = t; k < kBS * (D / 16); k += 128) {  // 16 fp8 codes -> 16 halves
-            const int r = k / (D / 16), cc = k - r * (D / 16);
-            const uint4 v = lds128(ks + tile_off(r, 16 * cc));
-            uint32_t h[8];
-            e4m3x4_to_f16x2x2(v.x, h[0], h[1]);
-            e4m3x4_to_f16x2x2(v.y, h[2], h[3]);
-            e4m3x4_to_f16x2x2(v.z, h[4], h[5]);
-            e4m3x4_to_f16x2x2(v.w, h[6], h[7]);
-            *reinterpret_cast<uint4*>(kf + C::sw128(T, 16 * j + r, 32 * cc)) = make_uint4(h[0], h[1], h[2], h[3]);
-            *reinterpret_cast<uint4*>(kf + C::sw128(T, 16 * j + r, 32 * cc + 16)) = make_uint4(h[4], h[5], h[6], h[7]);
+          uint8_t* kf = smem + C::OFF_KF + cb * C::F_BYTES;
+          uint8_t* vf = smem + C::OFF_VF + cb * C::F_BYTES;
+          for (int k = t; k < 2 * kBS * (D / 16); k += 128) {  // (K|V, row, 16 codes) -> 16 halves
+            const int which = k / (kBS * (D / 16));
+            const int kk = k - which * (kBS * (D / 16));
+            const int r = kk / (D / 16), cc = kk - r * (D / 16);
+            uint32_t h[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            if (i < nb && (which == 0 || r < valid)) {
+              const uint4 v = lds128(base + (which ? C::OFF_RING_V : C::OFF_RING_K) + C::ring(st, r, 16 * cc));
+              e4m3x4_to_f16x2x2(v.x, h[0], h[1]);
+              e4m3x4_to_f16x2x2(v.y, h[2], h[3]);
+              e4m3x4_to_f16x2x2(v.z, h[4], h[5]);
+              e4m3x4_to_f16x2x2(v.w, h[6], h[7]);
+            }
+            uint8_t* dst = which ? vf : kf;
+            *reinterpret_cast<uint4*>(dst + C::sw128(T, 16 * j + r, 32 * cc)) = make_uint4(h[0], h[1], h[2], h[3]);
+            *reinterpret_cast<uint4*>(dst + C::sw128(T, 16 * j + r, 32 * cc + 16)) = make_uint4(h[4], h[5], h[6], h[7]);
+          }
+          if (i < nb) {
+            fence_proxy_async_smem();  // (the ring stage's next writer is TMA)
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty0 + 8 * st);
+            if (t == 0) *converted = i + 1;
           }
         } else {
-          for (int k = t; k < kBS * (D / 8); k += 128) {
-            const int r = k / (D / 8), cc = k - r * (D / 8);
-            *reinterpret_cast<uint4*>(kf + C::sw128(T, 16 * j + r, 16 * cc)) = lds128(ks + tile_off(r, 16 * cc));
+          if (valid < kBS) {  // zero V rows valid..15 of this stage, every sub-tile
+            for (int k = t; k < (kBS - valid) * C::SUBTILES * 8; k += 128) {
+              const int r = valid + k / (C::SUBTILES * 8), rest = k % (C::SUBTILES * 8);
+              *reinterpret_cast<uint4*>(smem + C::OFF_RING_V + C::ring(st, r, 16 * rest)) = make_uint4(0u, 0u, 0u, 0u);
+            }
           }
+          if (t == 0 && i < nb) *converted = i + 1;
         }
-        // V^T: element (dim n, token tt) at (n/8)*CM_STRIDE + (tt/8)*128 + (n%8)*16 + (tt%8)*2;
-        // item = (8 dims, a pair of tokens) -> eight 32-bit (token pair) stores
-        for (int it = t; it < D; it += 128) {
-          const int c = it >> 3, pr = it & 7;  // dims [8c, 8c + 8), tokens 2pr, 2pr + 1 of the block
-          uint32_t a[4], bb[4];
-          if constexpr (C::kFp8) {
-            uint32_t lo0, hi0;
-            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo0), "=r"(hi0) : "r"(vs + tile_off(2 * pr, 8 * c)));
-            e4m3x4_to_f16x2x2(lo0, a[0], a[1]);
-            e4m3x4_to_f16x2x2(hi0, a[2], a[3]);
-            asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(lo0), "=r"(hi0) : "r"(vs + tile_off(2 * pr + 1, 8 * c)));
-            e4m3x4_to_f16x2x2(lo0, bb[0], bb[1]);
-            e4m3x4_to_f16x2x2(hi0, bb[2], bb[3]);
-          } else {
-            const uint4 x0 = lds128(vs + tile_off(2 * pr, 16 * c));
-            const uint4 x1 = lds128(vs + tile_off(2 * pr + 1, 16 * c));
-            a[0] = x0.x; a[1] = x0.y; a[2] = x0.z; a[3] = x0.w;
-            bb[0] = x1.x; bb[1] = x1.y; bb[2] = x1.z; bb[3] = x1.w;
-          }
-          const int tt = 16 * j + 2 * pr;
-          // keys past the range's valid tokens: P is 0 there and the cache slot may hold anything
-          const int kidx = 16 * i + 2 * pr;
-          if (kidx >= job.kv_valid) a[0] = a[1] = a[2] = a[3] = 0u;
-          if (kidx + 1 >= job.kv_valid) bb[0] = bb[1] = bb[2] = bb[3] = 0u;
-          uint8_t* dst = vt + c * C::CM_STRIDE + (tt >> 3) * 128 + (tt & 7) * 2;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            *reinterpret_cast<uint32_t*>(dst + (2 * q) * 16) = prmt(a[q], bb[q], 0x5410u);
-            *reinterpret_cast<uint32_t*>(dst + (2 * q + 1) * 16) = prmt(a[q], bb[q], 0x7632u);
-          }
-        }
-        fence_proxy_async_smem();  // (the ring stage's next writer is TMA)
-        __syncwarp();
-        if (lane == 0) mbar_arrive(empty0 + 8 * st);
-        if (t == 0) *converted = i + 1;
       }
       if (stop) break;
       fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
@@ -336,7 +322,7 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
     // ---------------------------------------------------------------- MMA issue
     if (lane == 0) {
       constexpr uint32_t idS = umma_idesc_f16(kPrefixRows, T, C::kBf16);
-      constexpr uint32_t idO = umma_idesc_f16(kPrefixRows, D, C::kBf16);
+      constexpr uint32_t idO = umma_idesc_f16(kPrefixRows, D, C::kBf16, /*b_mn_major=*/true);
       const uint32_t qa = base + C::OFF_Q;
       // Issue S for a step as soon as its operands are staged (at most B
       // steps ahead of the softmax), and O += P V as soon as the softmax has
@@ -348,11 +334,14 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
         if (ns_ < nsteps && ns_ - npv < B && mbar_test_wait(convf0 + 8 * (ns_ % B), (ns_ / B) & 1)) {
           tc_fence_after();
           const int cb = ns_ % B;
-          const uint32_t kb = base + C::OFF_KF + cb * C::KF_BYTES;
+          // K operand: the f16 copy (fp8) or the ring stages of the step (16-bit)
+          const uint32_t kb = C::kFp8 ? base + C::OFF_KF + cb * C::F_BYTES
+                                      : base + C::OFF_RING_K + ((ns_ * SB) % NS) * (kBS * 128);
+          constexpr int KSUB = C::kFp8 ? T * 128 : C::RING_SUB;  // bytes between 64-dim sub-tiles
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {  // S = Q K^T over 16-wide slices of D
             const uint64_t a = umma_desc(qa + (k >> 2) * (kPrefixRows * 128) + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
-            const uint64_t b = umma_desc(kb + (k >> 2) * (T * 128) + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
+            const uint64_t b = umma_desc(kb + (k >> 2) * KSUB + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
             umma_f16(tmem + C::S_COL + cb * T, a, b, idS, k > 0);
           }
           umma_commit(sfull0 + 8 * cb);
@@ -362,14 +351,22 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
         if (npv < ns_ && mbar_test_wait(pfull0 + 8 * (npv % B), (npv / B) & 1)) {
           tc_fence_after();
           const int cb = npv % B;
-          const uint32_t pa_ = base + C::OFF_P + cb * C::P_BYTES, va = base + C::OFF_VT + cb * C::VT_BYTES;
+          const uint32_t pa_ = base + C::OFF_P + cb * C::P_BYTES;
+          // V operand, MN-major (dims contiguous in 128-byte rows, one row per
+          // token): the f16 copy (fp8) or the ring stages of the step (16-bit)
+          const uint32_t va = C::kFp8 ? base + C::OFF_VF + cb * C::F_BYTES
+                                      : base + C::OFF_RING_V + ((npv * SB) % NS) * (kBS * 128);
+          constexpr int VSUB = C::kFp8 ? T * 128 : C::RING_SUB;  // bytes between 64-dim sub-tiles
 #pragma unroll
-          for (int k = 0; k < T / 16; ++k) {  // O += P V over 16-token slices
+          for (int k = 0; k < T / 16; ++k) {  // O += P V over 16-token slices (one block each)
             const uint64_t a = umma_desc(pa_ + k * 256, 128, C::CM_STRIDE, kUmmaNoSwizzle);
-            const uint64_t b = umma_desc(va + k * 256, 128, C::CM_STRIDE, kUmmaNoSwizzle);
+            const uint64_t b = umma_desc(va + k * (kBS * 128), VSUB, 1024, kUmmaSwizzle128);
             umma_f16(tmem + C::O_COL, a, b, idO, (npv > 0 || k > 0) ? 1 : 0);
           }
           umma_commit(pvdone0 + 8 * cb);
+          if constexpr (!C::kFp8) {  // the step's ring stages are free once these MMAs complete
+            for (int j = 0; j < SB && npv * SB + j < nb; ++j) umma_commit(empty0 + 8 * ((npv * SB + j) % NS));
+          }
           ++npv;
           progress = true;
         }

@@ -11,6 +11,11 @@
 //   * no swizzle (type 0): 8-row x 16-byte core matrices; leading offset =
 //     distance between core matrices along K, stride offset = distance
 //     between 8-row groups.
+// and one MN-major layout (B operand with the N index contiguous, the
+// instruction descriptor's B-major bit set):
+//   * 128-byte swizzle: 128-byte rows holding 64 N-elements, one row per K
+//     index, 8-row atoms; leading offset = distance between 64-element
+//     groups along N, stride offset = distance between 8-row atoms along K.
 // Instruction descriptor (kind::f16, 32 bits): accumulator format (1 = f32)
 // in [4,6), A / B format (0 = f16, 1 = bf16) in [7,10) / [10,13), A / B
 // major-ness (0 = K-major) in bits 15 / 16, N >> 3 in [17,23), M >> 4 in
@@ -27,9 +32,9 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t saddr, uint32_t lbo, uint
 }
 constexpr uint32_t kUmmaSwizzle128 = 2, kUmmaNoSwizzle = 0;
 
-__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool bf16) {
-  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((uint32_t)(N >> 3) << 17) |
-         ((uint32_t)(M >> 4) << 24);
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N, bool bf16, bool b_mn_major = false) {
+  return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+         ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 
 // D[tmem] (+)= A[smem] . B[smem]^T, issued by one thread.
