@@ -815,20 +815,19 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
 // Log-sum-exp merge of split sequences.  A CTA of 256 threads covers
 // `merge_hpc` consecutive query heads of one sequence; its threads are
 // (head, partition slice, 4-dim chunk) triples, `merge_slices` slices taking
-// every merge_slices-th partial.  Warp n first finds head n's largest partial
-// max M and weight sum W; each thread then accumulates l_p 2^(m_p - M) o_p
-// over its partials with 8 partials' loads in flight, and the slices are
-// summed in shared memory.  A head's partials are the decode pass's np
-// partitions, followed, in shared-prefix decode, by the prefix pass's chunks.
-// Launched as a programmatic dependent of the decode kernel: it may be
-// scheduled early and waits for the decode grid to finish before reading.
+// every merge_slices-th partial.  Each thread folds its partials into a
+// running (max M, weight sum W, weighted sum) in one pass, 8 partials' loads
+// in flight, and the slices are folded together in shared memory with the
+// same rule; out = weighted sum / W.  A head's partials are the decode pass's
+// np partitions, followed, in shared-prefix decode, by the prefix pass's
+// chunks.  Launched as a programmatic dependent of the decode kernel: it may
+// be scheduled early and waits for the decode grid to finish before reading.
 template <typename Q, int D, bool BF16>
 __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodeParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int CH = D / 4;  // float4 chunks per head
-  __shared__ float hM[kNH], hInvW[kNH];
-  __shared__ int hNp[kNH];
   __shared__ float4 red[256];
+  __shared__ float2 redm[256];
   const int hpc = p.merge_hpc, slices = p.merge_slices;
   const int hblocks = (p.num_heads + hpc - 1) / hpc;
   const int s = blockIdx.x / hblocks;
@@ -838,7 +837,6 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
   const int len = shared ? max(0, clamp_len(p.seq_lens[s], p) - skip * kBS) : clamp_len(p.seq_lens[s], p);
   const int nblk = (len + kBS - 1) / kBS;
   const int nc = shared ? (skip + kPrefixChunkBlocks - 1) / kPrefixChunkBlocks : 0;  // prefix partials
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // the decode launch's hand-out: stream-K or tickets with pb blocks per partition
   const bool sk = p.auto_mode && p.counters[3] != 0;
   const int param = p.auto_mode ? p.counters[2] : p.partition_blocks;
@@ -866,66 +864,59 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
     return q < np ? p.part_o + (((size_t)s * p.num_heads + h) * p.max_parts + q) * D
                   : p.pre_o + (((size_t)s * p.num_heads + h) * p.max_chunks + (q - np)) * D;
   };
-  if (warp < hpc) {
-    const int h = h0 + warp;
-    float M = -INFINITY, W = 0.f;
-    if (h < p.num_heads) {
-      for (int q = lane; q < nt; q += 32) M = fmaxf(M, ml_of(h, q)[0]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-      for (int q = lane; q < nt; q += 32) {
-        const float2 v = *reinterpret_cast<const float2*>(ml_of(h, q));
-        if (v.y > 0.f) W += v.y * ex2(v.x - M);
-      }
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) W += __shfl_xor_sync(0xffffffffu, W, off);
-    }
-    if (lane == 0) {
-      hM[warp] = M;
-      hInvW[warp] = W > 0.f ? 1.f / W : 0.f;
-      hNp[warp] = h < p.num_heads ? nt : 0;
-    }
-  }
-  __syncthreads();
+  // One pass: each thread keeps a running (max, weight sum, weighted sum of
+  // its 4 dims) over its partials, loading 8 partials at a time; slices are
+  // then combined with the same rule.
   const int c = threadIdx.x % CH;
   const int rest = threadIdx.x / CH;
   const int slice = rest % slices, hl = rest / slices;
   const int h = h0 + hl;
-  const int nth = hl < hpc ? hNp[hl] : 0;
+  const bool active = hl < hpc && h < p.num_heads;
+  float M = -INFINITY, W = 0.f;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  if (nth > 0) {
-    const float M = hM[hl];
-    for (int q0 = slice; q0 < nth; q0 += 8 * slices) {
+  // fold in a summary (m, w, a4) with w = sum l 2^(m_q - m) and a4 = sum l 2^(m_q - m) o_q
+  auto combine = [&](float m, float w, const float4& a4) {
+    if (!(w > 0.f)) return;
+    const float mn = fmaxf(M, m);
+    const float a = ex2(M - mn), b = ex2(m - mn);
+    acc.x = fmaf(b, a4.x, acc.x * a);
+    acc.y = fmaf(b, a4.y, acc.y * a);
+    acc.z = fmaf(b, a4.z, acc.z * a);
+    acc.w = fmaf(b, a4.w, acc.w * a);
+    W = fmaf(W, a, w * b);
+    M = mn;
+  };
+  if (active) {
+    for (int q0 = slice; q0 < nt; q0 += 8 * slices) {
       float2 mlq[8];
       float4 v[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int q = q0 + u * slices;
-        const bool ok = q < nth;
+        const bool ok = q < nt;
         mlq[u] = ok ? *reinterpret_cast<const float2*>(ml_of(h, q)) : make_float2(-INFINITY, 0.f);
         v[u] = ok ? *reinterpret_cast<const float4*>(o_of(h, q) + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const float w = mlq[u].y > 0.f ? mlq[u].y * ex2(mlq[u].x - M) : 0.f;
-        acc.x = fmaf(w, v[u].x, acc.x);
-        acc.y = fmaf(w, v[u].y, acc.y);
-        acc.z = fmaf(w, v[u].z, acc.z);
-        acc.w = fmaf(w, v[u].w, acc.w);
+      for (int u = 0; u < 8; ++u) {  // a partial (o, m, l) is the summary (m, l, l o)
+        const float l = mlq[u].y;
+        combine(mlq[u].x, l, make_float4(l * v[u].x, l * v[u].y, l * v[u].z, l * v[u].w));
       }
     }
   }
-  red[threadIdx.x] = acc;
-  __syncthreads();
-  if (slice == 0 && hl < hpc && h < p.num_heads) {
-    for (int k = 1; k < slices; ++k) {
-      const float4 o = red[threadIdx.x + k * CH];
-      acc.x += o.x;
-      acc.y += o.y;
-      acc.z += o.z;
-      acc.w += o.w;
+  if (slices > 1) {
+    red[threadIdx.x] = acc;
+    redm[threadIdx.x] = make_float2(M, W);
+    __syncthreads();
+    if (slice == 0 && active) {
+      for (int k = 1; k < slices; ++k) {
+        const float2 mw = redm[threadIdx.x + k * CH];
+        combine(mw.x, mw.y, red[threadIdx.x + k * CH]);
+      }
     }
-    const float inv = hInvW[hl];  // 0 when no partial has weight: a zero row
+  }
+  if (slice == 0 && active) {
+    const float inv = W > 0.f ? 1.f / W : 0.f;  // no weighted partial: a zero row
     Q* dst = reinterpret_cast<Q*>(p.out) + ((size_t)s * p.num_heads + h) * D + 4 * c;
     *reinterpret_cast<uint2*>(dst) = make_uint2(pack2<BF16>(acc.x * inv, acc.y * inv), pack2<BF16>(acc.z * inv, acc.w * inv));
   }

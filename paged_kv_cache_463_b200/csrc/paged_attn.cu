@@ -545,7 +545,7 @@ int decode_impl(pa_ctx* ctx, void* out, const void* query, const void* key_cache
     prefix_chunks = (pblocks + pa::kPrefixChunkBlocks - 1) / pa::kPrefixChunkBlocks;
     const int rows_per_unit = pre->max_group_size * (group < pa::kNH ? group : pa::kNH);
     row_blocks = (rows_per_unit + pa::kPrefixRows - 1) / pa::kPrefixRows;
-    if ((long long)kv_units * row_blocks > 65535)
+    if ((long long)kv_units * row_blocks + 1 > 65535)
       return fail(ctx, PA_ERR_UNSUPPORTED, "max_group_size too large for the prefix grid");
   }
   cudaSetDevice(ctx->device);
@@ -582,7 +582,8 @@ int decode_impl(pa_ctx* ctx, void* out, const void* query, const void* key_cache
     q.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
     q.v_scale = fp8 ? v_scale : 1.0f;
     void* qargs[] = {&mk, &mv, &q};
-    const dim3 grid((unsigned)(prefix_chunks > 0 ? prefix_chunks : 1), (unsigned)(kv_units * row_blocks),
+    // grid.y: the attention CTAs, plus one row whose x = 0 CTA checks each group
+    const dim3 grid((unsigned)(prefix_chunks > 0 ? prefix_chunks : 1), (unsigned)(kv_units * row_blocks + 1),
                     (unsigned)pre->num_groups);
     cudaError_t e = cudaLaunchKernel(ctx->ks.prefix, grid, dim3(ctx->ks.prefix_threads), qargs,
                                      ctx->ks.prefix_smem, s);

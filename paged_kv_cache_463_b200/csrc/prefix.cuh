@@ -197,14 +197,18 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
-  if (warp < 4) {
+  if (warp < 4) {  // row r's D values: every 16-byte chunk in flight at once (cp.async)
     const int r = threadIdx.x;
-    const uint4* src = reinterpret_cast<const uint4*>(rows.q_row(r));
-#pragma unroll 4
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(rows.q_row(r));
+#pragma unroll
     for (int c = 0; c < D / 8; ++c) {
-      const uint4 v = src ? src[c] : make_uint4(0u, 0u, 0u, 0u);
-      *reinterpret_cast<uint4*>(smem + C::OFF_Q + C::sw128(kPrefixRows, r, 16 * c)) = v;
+      const uint32_t dst = base + C::OFF_Q + C::sw128(kPrefixRows, r, 16 * c);
+      if (src)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src + 16 * c) : "memory");
+      else
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
     }
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
     fence_proxy_async_smem();
   }
   tc_fence_before();
@@ -490,13 +494,14 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
   constexpr int D = C::D;
 
   const int g = blockIdx.z;
-  const int y = blockIdx.y / p.row_blocks;
-  const int rb = blockIdx.y - y * p.row_blocks;
   const int chunk = blockIdx.x;
   const int first = p.group_start[g], members = p.group_start[g + 1] - first;
   const int pblk = group_prefix_blocks(p, g, first, members);
 
-  if (blockIdx.x == 0 && blockIdx.y == 0) {
+  // The last row of the grid checks the groups (its x = 0 CTA per group),
+  // beside the CTAs that attend over the prefixes.
+  if (blockIdx.y == gridDim.y - 1) {
+    if (blockIdx.x != 0) return;
     // One CTA per group: the group's description, and the suffix offsets of
     // its members (plus those of the sequences before the first group / from
     // the last group's end on, which have no shared prefix).
@@ -531,7 +536,10 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
       const int hi = max(min(first + members, p.num_seqs), 0);
       for (int s = hi + threadIdx.x; s < p.num_seqs; s += blockDim.x) p.seq_skip[s] = 0;
     }
+    return;
   }
+  const int y = blockIdx.y / p.row_blocks;
+  const int rb = blockIdx.y - y * p.row_blocks;
 
   const int kvh = y / p.head_splits;
   const int hs = y - kvh * p.head_splits;
