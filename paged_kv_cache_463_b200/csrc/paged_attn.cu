@@ -147,7 +147,7 @@ template <> struct Tuned<64, __half, __half> {
 };
 template <> struct Tuned<128, __half, __half> {
   using C = DecodeCfg<128, __half, __half, PA_NS_16B_128, 8>;
-  using P = pa::PrefixCfg<128, __half, __half, 8, 4>;
+  using P = pa::PrefixCfg<128, __half, __half, 6, 2>;
 };
 template <> struct Tuned<256, __half, __half> {
   using C = DecodeCfg<256, __half, __half, PA_NS_16B_256, 3>;
@@ -159,7 +159,7 @@ template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> {
 };
 template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128, 8>;
-  using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, 8, 4>;
+  using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, 6, 2>;
 };
 template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_256, 3>;
