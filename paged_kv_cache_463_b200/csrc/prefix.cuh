@@ -407,12 +407,13 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
       }
       tmem_wait_ld();
       const int valid = min(T, lim - u * T);  // keys of this step the row sees
-      float bm = -INFINITY;
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent max chains
 #pragma unroll
       for (int j = 0; j < T; ++j) {
         x[j] = j < valid ? x[j] * scale_log2 : -INFINITY;
-        bm = fmaxf(bm, x[j]);
+        mx[j & 3] = fmaxf(mx[j & 3], x[j]);
       }
+      const float bm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
       // lazy rescaling: move the reference max (and rescale l, O) only when
       // this step's max exceeds it by more than 2^8
       const bool grow = bm > m + 8.f;
@@ -440,19 +441,19 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
       }
       // P row r: token groups of 8 as 16-byte core-matrix rows
       uint8_t* prow = smem + C::OFF_P + cb * C::P_BYTES + (r >> 3) * C::CM_STRIDE + (r & 7) * 16;
-      float sum = 0.f;
+      float sm[4] = {0.f, 0.f, 0.f, 0.f};  // four independent sum chains
 #pragma unroll
       for (int g8 = 0; g8 < T / 8; ++g8) {
         uint32_t pk[4];
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float p0 = ex2(x[8 * g8 + 2 * q] - m), p1 = ex2(x[8 * g8 + 2 * q + 1] - m);
-          sum += p0 + p1;
+          sm[q] += p0 + p1;
           pk[q] = pack2<C::kBf16>(p0, p1);
         }
         *reinterpret_cast<uint4*>(prow + g8 * 128) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
       }
-      l += sum;
+      l += (sm[0] + sm[1]) + (sm[2] + sm[3]);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
