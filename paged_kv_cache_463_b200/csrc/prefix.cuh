@@ -15,19 +15,25 @@
 // S[128 rows x T] = Q K^T, then O[128 x D] += P V.  Both run on the
 // 5th-generation tensor cores (tcgen05.mma, issued by one thread,
 // accumulators in tensor memory), one CTA per (group, KV unit, 128 query
-// rows, chunk of 32 prefix blocks):
-//   warp 8      TMA producer: each block's K/V tiles into an NS-stage ring;
-//   warps 4..7  stage a step's MMA operands: K as a 16-bit 128-byte-swizzled
-//               [T x D] tile (fp8 E4M3 codes converted to f16), V transposed
-//               to V^T [D x T] (tokens contiguous); two step buffers;
+// rows, chunk of 32 prefix blocks).  The core, `stacked_attention`, is shared
+// with the multi-query (prefill) kernel; its roles:
+//   warp 8      TMA producer: each block's K and V tiles into two NS-stage
+//               rings laid out sub-tile-major, so that a step's SB stages
+//               hold its tokens' rows contiguously;
+//   warps 4..7  16-bit caches: the rings are the MMA operands (K K-major, V
+//               MN-major), so these warps only zero V rows past the valid
+//               keys; fp8 caches: they convert each block's K and V rows to
+//               f16 once, into per-step operand buffers;
 //   warp 9      polls the barriers and issues S for a step once its operands
-//               are staged (into one of two TMEM S buffers) and O += P V once
-//               the softmax has written that step's P;
+//               are ready (into one of two TMEM S buffers) and O += P V once
+//               the softmax has written that step's P; for 16-bit caches the
+//               ring stages are released by tcgen05.commit after the step's
+//               P V;
 //   warps 0..3  one query row per thread: read the step's S row from TMEM,
 //               online softmax in the log2 domain (lazy: O is rescaled in
 //               TMEM only when a row's maximum grows by more than 2^8), write
 //               P (16-bit) to shared memory; at the end read O, normalise,
-//               store the partial.
+//               hand the row to the caller's store.
 #pragma once
 
 #include "decode.cuh"
