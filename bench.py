@@ -293,14 +293,15 @@ def run_ours(args, world, rank, local):
         max_group = int(gsizes.max().item())
         max_prefix = int(w.group_prefix_len.max().item())
 
-    def attend(q, bt, lens, o=None):
+    def attend(q, bt, lens, o=None, st=None):
         o = out if o is None else o
+        st = stream if st is None else st
         if shared:
             pa.paged_attention_decode_shared_prefix(o, q, kc, vc, bt, lens, max_len, w.group_start,
                                                     w.group_prefix_len, max_group, max_prefix, w.scale,
-                                                    w.k_scale, w.v_scale, stream)
+                                                    w.k_scale, w.v_scale, st)
         else:
-            pa.paged_attention_decode(o, q, kc, vc, bt, lens, max_len, w.scale, w.k_scale, w.v_scale, stream)
+            pa.paged_attention_decode(o, q, kc, vc, bt, lens, max_len, w.scale, w.k_scale, w.v_scale, st)
 
     def step():
         pa.reshape_and_cache(w.new_key, w.new_value, kc, vc, w.slot_mapping, w.k_scale, w.v_scale, stream)
@@ -313,6 +314,22 @@ def run_ours(args, world, rank, local):
         raise SystemExit("device check fired during warm-up")
 
     # ---- device-timed region: whole steps, plus the decode call inside each
+    # (--graph: each step is one replay of a CUDA graph captured from the same
+    # calls; the decode-call time then comes from a decode-only graph)
+    g_step = g_dec = None
+    if args.graph:
+        side = torch.cuda.Stream(device=dev)
+        side.wait_stream(stream)
+        g_step, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_step, stream=side):
+            pa.reshape_and_cache(w.new_key, w.new_value, kc, vc, w.slot_mapping, w.k_scale, w.v_scale, side)
+            attend(w.query, w.block_tables, w.seq_lens, out, side)
+        with torch.cuda.graph(g_dec, stream=side):
+            attend(w.query, w.block_tables, w.seq_lens, out, side)
+        stream.wait_stream(side)
+        for _ in range(args.warmup):
+            g_step.replay()
+        torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     barrier(world)
@@ -323,6 +340,9 @@ def run_ours(args, world, rank, local):
         t_start.record(stream)
         for i in range(args.steps):
             a, m, e = ev[i]
+            if g_step is not None:
+                g_step.replay()
+                continue
             a.record(stream)
             pa.reshape_and_cache(w.new_key, w.new_value, kc, vc, w.slot_mapping, w.k_scale, w.v_scale, stream)
             m.record(stream)
@@ -332,8 +352,18 @@ def run_ours(args, world, rank, local):
         torch.cuda.synchronize()
     barrier(world)
     total_ms = t_start.elapsed_time(t_end)
-    decode_ms = [m.elapsed_time(e) for (_, m, e) in ev]
-    write_ms = [a.elapsed_time(m) for (a, m, _) in ev]
+    if g_step is None:
+        decode_ms = [m.elapsed_time(e) for (_, m, e) in ev]
+        write_ms = [a.elapsed_time(m) for (a, m, _) in ev]
+    else:
+        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for _ in range(args.steps):
+            g_dec.replay()
+        d1.record(stream)
+        torch.cuda.synchronize()
+        decode_ms = [d0.elapsed_time(d1) / args.steps]
+        write_ms = [max(0.0, total_ms / args.steps - decode_ms[0])]
     total_ms = max_over_ranks(total_ms, world)
     if pa.get_error() != 0:
         raise SystemExit("device check fired during the timed region")
@@ -418,6 +448,7 @@ def run_ours(args, world, rank, local):
                    else chosen_part,
                    "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
                    "shared_prefix": bool(shared),
+                   "launch": "one CUDA graph replay per step" if args.graph else "eager launches",
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
         "seq_steps_per_s": seq_steps,
         "pct_of_nominal_8tbs": 100.0 * value / world / NOMINAL_HBM_GBS,
@@ -698,6 +729,8 @@ def main():
                          "block-manager: host bookkeeping of a decode step; prefill: causal multi-query attention")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=list(wl.SPEC_BY_NAME))
     ap.add_argument("--partition", default="auto", help="auto | none | tokens per partition")
+    ap.add_argument("--eager", dest="graph", action="store_false",
+                    help="launch each step's kernels directly instead of replaying a captured CUDA graph")
     ap.add_argument("--num-seqs", type=int, default=0, help="smaller batch of the same workload (profiling)")
     ap.add_argument("--shared-prefix", choices=["auto", "on", "off"], default="auto",
                     help="shared-prefix decode for workloads with prefix groups (auto: when the workload has them)")
