@@ -233,6 +233,20 @@ struct WarpAttn {
   uint32_t qf[NKT][2];
   float o[NDT][4];
   float m0, m1, l0, l1;
+  // fp8 V rows of the current tile: lane row gid owns dims [D/8*gid,
+  // D/8*gid + D/8) of tokens 2c4, 2c4+1, 2c4+8, 2c4+9; output tile t holds
+  // dims D/8*gid + 2t (MMA row gid) and +1 (row gid+8)
+  uint4 vr[4][FP8 ? D / 128 : 1];
+
+  __device__ __forceinline__ void load_v8(uint32_t vb, int gid, int c4) {
+    constexpr int LB = D / 8;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int row = 2 * c4 + (r & 1) + ((r >> 1) << 3);
+#pragma unroll
+      for (int u = 0; u < LB / 16; ++u) vr[r][u] = lds128(vb + tile_off(row, LB * gid + 16 * u));
+    }
+  }
 
   __device__ __forceinline__ void reset() {
 #pragma unroll
@@ -287,6 +301,7 @@ struct WarpAttn {
         kr[0][u] = lds128(kb + tile_off(gid, LB * c4 + 16 * u));
         kr[1][u] = lds128(kb + tile_off(gid + 8, LB * c4 + 16 * u));
       }
+      load_v8(vb, gid, c4);  // the V loads overlap the S contraction and the softmax
       const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&kr[0][0]);
       const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&kr[1][0]);
 #pragma unroll
@@ -301,23 +316,26 @@ struct WarpAttn {
       }
     }
     // ---- online softmax (log2 domain); rows of S^T are tokens gid, gid+8
-            const float x0 = gid < valid ? (sa[0] + sb[0]) * sl : -INFINITY;
+    const float x0 = gid < valid ? (sa[0] + sb[0]) * sl : -INFINITY;
     const float x1 = gid < valid ? (sa[1] + sb[1]) * sl : -INFINITY;
     const float x2 = gid + 8 < valid ? (sa[2] + sb[2]) * sl : -INFINITY;
     const float x3 = gid + 8 < valid ? (sa[3] + sb[3]) * sl : -INFINITY;
     float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-      bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
-      bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
-    }
     // Lazy rescaling: the reference max only moves (and O, l are
     // rescaled) when some head's block max exceeds it by more than
     // 2^kLazy; otherwise weights up to 2^kLazy are accumulated as they are
-    // (exact in fp32, and well inside the 16-bit P range).
+    // (exact in fp32, and well inside the 16-bit P range).  A head's running
+    // max is the same in all lanes of its column, so "some lane's own
+    // scores exceed it" is the same test as "the block max does": the
+    // column reductions are only needed when it passes.
     constexpr float kLazy = 8.f;
     const bool grow = (bm0 > m0 + kLazy) || (bm1 > m1 + kLazy);
     if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
+        bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
+      }
       const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
       const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
       m0 = mn0;
@@ -357,17 +375,7 @@ struct WarpAttn {
         }
       }
     } else {
-      // lane row gid owns dims [D/8*gid, D/8*gid + D/8) of tokens 2c4, 2c4+1, 2c4+8, 2c4+9;
-      // output tile t holds dims D/8*gid + 2t (MMA row gid) and +1 (row gid+8)
-      constexpr int LB = D / 8;
-      constexpr int LC = LB / 16;
-      uint4 vr[4][LC];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int row = 2 * c4 + (r & 1) + ((r >> 1) << 3);
-#pragma unroll
-        for (int u = 0; u < LC; ++u) vr[r][u] = lds128(vb + tile_off(row, LB * gid + 16 * u));
-      }
+      constexpr int LC = D / 128;
       if (valid < kBS) {
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
