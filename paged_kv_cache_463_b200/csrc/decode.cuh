@@ -33,7 +33,9 @@
 //      O^T[D x 8] += V^T[D x 16 tok] . P^T[16 x 8]       (V via ldmatrix.trans)
 //    fp8 E4M3 tiles are read with 128-bit shared loads and converted in
 //    registers to f16 pairs (exact); the contraction order is permuted so
-//    that every lane's operands are contiguous bytes;
+//    that every lane's operands are contiguous bytes; when an item's next
+//    block has already landed, two fp8 tiles share one step (one softmax
+//    update for 32 tokens);
 //  * at an item's last block the consumer writes the output (one-partition
 //    sequences) or (O / l, m, l) partials; paged_decode_merge_kernel, launched
 //    as a programmatic dependent of this grid, combines split sequences with
@@ -273,6 +275,123 @@ struct WarpAttn {
     }
   }
 
+  // Lazy rescaling with this lane's own maxima bm0 / bm1 of its two columns:
+  // the reference max only moves (and O, l are rescaled) when some head's
+  // new scores exceed it by more than 2^kLazy; otherwise weights up to 2^kLazy
+  // are accumulated as they are (exact in fp32, and well inside the 16-bit P
+  // range).  A head's running max is the same in all lanes of its column, so
+  // "some lane's own scores exceed it" is the same test as "the column max
+  // does": the column reductions are only needed when it passes.
+  __device__ __forceinline__ void update_max(float bm0, float bm1) {
+    constexpr float kLazy = 8.f;
+    const bool grow = (bm0 > m0 + kLazy) || (bm1 > m1 + kLazy);
+    if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
+        bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
+      }
+      const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
+      const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
+      m0 = mn0;
+      m1 = mn1;
+      l0 *= al0;
+      l1 *= al1;
+#pragma unroll
+      for (int t = 0; t < NDT; ++t) {
+        o[t][0] *= al0;
+        o[t][1] *= al1;
+        o[t][2] *= al0;
+        o[t][3] *= al1;
+      }
+    }
+  }
+
+  // fp8: S^T partial sums (two accumulation chains) of the K tile at kb.
+  __device__ __forceinline__ void scores8(uint32_t kb, float (&sa)[4], float (&sb)[4], int gid, int c4) {
+    constexpr int LB = D / 4;  // bytes of a K row owned by one lane
+    constexpr int LC = LB / 16;
+    uint4 kr[2][LC];
+#pragma unroll
+    for (int u = 0; u < LC; ++u) {
+      kr[0][u] = lds128(kb + tile_off(gid, LB * c4 + 16 * u));
+      kr[1][u] = lds128(kb + tile_off(gid + 8, LB * c4 + 16 * u));
+    }
+    const uint32_t* w0 = reinterpret_cast<const uint32_t*>(&kr[0][0]);
+    const uint32_t* w1 = reinterpret_cast<const uint32_t*>(&kr[1][0]);
+#pragma unroll
+    for (int j = 0; j < NKT; ++j) {
+      uint32_t a0, a1, a2, a3;
+      e4m3x4_to_f16x2x2(w0[j], a0, a2);
+      e4m3x4_to_f16x2x2(w1[j], a1, a3);
+      if (j & 1)
+        mma_16816<false>(sb, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+      else
+        mma_16816<false>(sa, a0, a1, a2, a3, qf[j][0], qf[j][1]);
+    }
+  }
+
+  // fp8: O^T += V^T P^T with the V rows held in vr (rows past `valid` zeroed
+  // first: they may hold NaN/Inf).
+  __device__ __forceinline__ void pv8(int valid, uint32_t pb0, uint32_t pb1, int c4) {
+    constexpr int LC = D / 128;
+    if (valid < kBS) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int row = 2 * c4 + (r & 1) + ((r >> 1) << 3);
+        if (row >= valid) {
+#pragma unroll
+          for (int u = 0; u < LC; ++u) vr[r][u] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+    }
+    const uint32_t* r0 = reinterpret_cast<const uint32_t*>(&vr[0][0]);
+    const uint32_t* r1 = reinterpret_cast<const uint32_t*>(&vr[1][0]);
+    const uint32_t* r2 = reinterpret_cast<const uint32_t*>(&vr[2][0]);
+    const uint32_t* r3 = reinterpret_cast<const uint32_t*>(&vr[3][0]);
+#pragma unroll
+    for (int w = 0; w < NDT / 2; ++w) {
+      uint32_t a0, a1, a2, a3;
+      // tile 2w: bytes 0,1 of word w; tile 2w+1: bytes 2,3
+      e4m3x4_to_f16x2x2(prmt(r0[w], r1[w], 0x5140u), a0, a1);
+      e4m3x4_to_f16x2x2(prmt(r2[w], r3[w], 0x5140u), a2, a3);
+      mma_16816<false>(o[2 * w], a0, a1, a2, a3, pb0, pb1);
+      e4m3x4_to_f16x2x2(prmt(r0[w], r1[w], 0x7362u), a0, a1);
+      e4m3x4_to_f16x2x2(prmt(r2[w], r3[w], 0x7362u), a2, a3);
+      mma_16816<false>(o[2 * w + 1], a0, a1, a2, a3, pb0, pb1);
+    }
+  }
+
+  // fp8: two consecutive tiles of one item (the first full, the second with
+  // valid2 tokens) with one softmax step over their 32 tokens.
+  __device__ __forceinline__ void block2(uint32_t kb1, uint32_t vb1, uint32_t kb2, uint32_t vb2, int valid2,
+                                         float sl, int lane) {
+    const int gid = lane >> 2, c4 = lane & 3;
+    float s1a[4] = {0.f, 0.f, 0.f, 0.f}, s1b[4] = {0.f, 0.f, 0.f, 0.f};
+    float s2a[4] = {0.f, 0.f, 0.f, 0.f}, s2b[4] = {0.f, 0.f, 0.f, 0.f};
+    scores8(kb1, s1a, s1b, gid, c4);
+    load_v8(vb1, gid, c4);
+    scores8(kb2, s2a, s2b, gid, c4);
+    const float x0 = (s1a[0] + s1b[0]) * sl, x1 = (s1a[1] + s1b[1]) * sl;
+    const float x2 = (s1a[2] + s1b[2]) * sl, x3 = (s1a[3] + s1b[3]) * sl;
+    const float y0 = gid < valid2 ? (s2a[0] + s2b[0]) * sl : -INFINITY;
+    const float y1 = gid < valid2 ? (s2a[1] + s2b[1]) * sl : -INFINITY;
+    const float y2 = gid + 8 < valid2 ? (s2a[2] + s2b[2]) * sl : -INFINITY;
+    const float y3 = gid + 8 < valid2 ? (s2a[3] + s2b[3]) * sl : -INFINITY;
+    update_max(fmaxf(fmaxf(x0, x2), fmaxf(y0, y2)), fmaxf(fmaxf(x1, x3), fmaxf(y1, y3)));
+    const float p0 = ex2(x0 - m0), p1 = ex2(x1 - m1), p2 = ex2(x2 - m0), p3 = ex2(x3 - m1);
+    const float q0 = ex2(y0 - m0), q1 = ex2(y1 - m1), q2 = ex2(y2 - m0), q3 = ex2(y3 - m1);
+    l0 += (p0 + p2) + (q0 + q2);
+    l1 += (p1 + p3) + (q1 + q3);
+    const uint32_t pb0 = movmatrix_trans(pack2<false>(p0, p1));
+    const uint32_t pb1 = movmatrix_trans(pack2<false>(p2, p3));
+    const uint32_t qb0 = movmatrix_trans(pack2<false>(q0, q1));
+    const uint32_t qb1 = movmatrix_trans(pack2<false>(q2, q3));
+    pv8(kBS, pb0, pb1, c4);
+    load_v8(vb2, gid, c4);
+    pv8(valid2, qb0, qb1, c4);
+  }
+
   // One 16-token tile: K at kb, V at vb (shared addresses, 128-byte swizzled
   // [16 x D] tiles); tokens >= valid are masked out.  sl = softmax scale x log2(e).
   __device__ __forceinline__ void block(uint32_t kb, uint32_t vb, int valid, float sl, int lane) {
@@ -320,36 +439,7 @@ struct WarpAttn {
     const float x1 = gid < valid ? (sa[1] + sb[1]) * sl : -INFINITY;
     const float x2 = gid + 8 < valid ? (sa[2] + sb[2]) * sl : -INFINITY;
     const float x3 = gid + 8 < valid ? (sa[3] + sb[3]) * sl : -INFINITY;
-    float bm0 = fmaxf(x0, x2), bm1 = fmaxf(x1, x3);
-    // Lazy rescaling: the reference max only moves (and O, l are
-    // rescaled) when some head's block max exceeds it by more than
-    // 2^kLazy; otherwise weights up to 2^kLazy are accumulated as they are
-    // (exact in fp32, and well inside the 16-bit P range).  A head's running
-    // max is the same in all lanes of its column, so "some lane's own
-    // scores exceed it" is the same test as "the block max does": the
-    // column reductions are only needed when it passes.
-    constexpr float kLazy = 8.f;
-    const bool grow = (bm0 > m0 + kLazy) || (bm1 > m1 + kLazy);
-    if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        bm0 = fmaxf(bm0, __shfl_xor_sync(0xffffffffu, bm0, off));
-        bm1 = fmaxf(bm1, __shfl_xor_sync(0xffffffffu, bm1, off));
-      }
-      const float mn0 = fmaxf(m0, bm0), mn1 = fmaxf(m1, bm1);
-      const float al0 = ex2(m0 - mn0), al1 = ex2(m1 - mn1);
-      m0 = mn0;
-      m1 = mn1;
-      l0 *= al0;
-      l1 *= al1;
-#pragma unroll
-      for (int t = 0; t < NDT; ++t) {
-        o[t][0] *= al0;
-        o[t][1] *= al1;
-        o[t][2] *= al0;
-        o[t][3] *= al1;
-      }
-    }
+    update_max(fmaxf(x0, x2), fmaxf(x1, x3));
     const float p0 = ex2(x0 - m0), p1 = ex2(x1 - m1), p2 = ex2(x2 - m0), p3 = ex2(x3 - m1);
     l0 += p0 + p2;
     l1 += p1 + p3;
@@ -375,32 +465,7 @@ struct WarpAttn {
         }
       }
     } else {
-      constexpr int LC = D / 128;
-      if (valid < kBS) {
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const int row = 2 * c4 + (r & 1) + ((r >> 1) << 3);
-          if (row >= valid) {
-#pragma unroll
-            for (int u = 0; u < LC; ++u) vr[r][u] = make_uint4(0u, 0u, 0u, 0u);
-          }
-        }
-      }
-      const uint32_t* r0 = reinterpret_cast<const uint32_t*>(&vr[0][0]);
-      const uint32_t* r1 = reinterpret_cast<const uint32_t*>(&vr[1][0]);
-      const uint32_t* r2 = reinterpret_cast<const uint32_t*>(&vr[2][0]);
-      const uint32_t* r3 = reinterpret_cast<const uint32_t*>(&vr[3][0]);
-#pragma unroll
-      for (int w = 0; w < NDT / 2; ++w) {
-        uint32_t a0, a1, a2, a3;
-        // tile 2w: bytes 0,1 of word w; tile 2w+1: bytes 2,3
-        e4m3x4_to_f16x2x2(prmt(r0[w], r1[w], 0x5140u), a0, a1);
-        e4m3x4_to_f16x2x2(prmt(r2[w], r3[w], 0x5140u), a2, a3);
-        mma_16816<false>(o[2 * w], a0, a1, a2, a3, pb0, pb1);
-        e4m3x4_to_f16x2x2(prmt(r0[w], r1[w], 0x7362u), a0, a1);
-        e4m3x4_to_f16x2x2(prmt(r2[w], r3[w], 0x7362u), a2, a3);
-        mma_16816<false>(o[2 * w + 1], a0, a1, a2, a3, pb0, pb1);
-      }
+      pv8(valid, pb0, pb1, c4);
     }
   }
 
@@ -765,16 +830,42 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
         A.reset();
       }
       const int valid = (md.w >> 8) & 0xff;
-      if (valid > 0) {
-        const uint32_t kb = base_u32 + L.ring + st * C::STAGE_BYTES;
-        A.block(kb, kb + C::TILE_BYTES, valid, p.scale_log2, lane);
+      // fp8: when the item's next block is already in the ring, take both
+      // tiles in one step (one softmax update for 32 tokens)
+      bool two = false;
+      int st2 = 0;
+      if constexpr (C::kFp8) {
+        if (!(md.w & kLast)) {
+          st2 = (stage_i + 1) % NS;
+          two = __all_sync(0xffffffffu, mbar_test_wait(full0 + 8 * st2, ((stage_i + 1) / NS) & 1));
+        }
       }
-      fence_proxy_async_smem();  // (the stage's next writer is TMA)
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8 * st);
-      ++stage_i;
+      int last = md.w & kLast;
+      if (two) {
+        const int4 md2 = meta[st2];
+        const uint32_t kb = base_u32 + L.ring + st * C::STAGE_BYTES;
+        const uint32_t kb2 = base_u32 + L.ring + st2 * C::STAGE_BYTES;
+        A.block2(kb, kb + C::TILE_BYTES, kb2, kb2 + C::TILE_BYTES, (md2.w >> 8) & 0xff, p.scale_log2, lane);
+        fence_proxy_async_smem();  // (the stages' next writer is TMA)
+        __syncwarp();
+        if (lane == 0) {
+          mbar_arrive(empty0 + 8 * st);
+          mbar_arrive(empty0 + 8 * st2);
+        }
+        stage_i += 2;
+        last = md2.w & kLast;
+      } else {
+        if (valid > 0) {
+          const uint32_t kb = base_u32 + L.ring + st * C::STAGE_BYTES;
+          A.block(kb, kb + C::TILE_BYTES, valid, p.scale_log2, lane);
+        }
+        fence_proxy_async_smem();  // (the stage's next writer is TMA)
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty0 + 8 * st);
+        ++stage_i;
+      }
 
-      if (md.w & kLast) {
+      if (last) {
         // ---- finish the item straight from registers; lane (gid, c4) holds
         // heads 2c4, 2c4+1 of 2 dims per tile
         float L0, L1;
