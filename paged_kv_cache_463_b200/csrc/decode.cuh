@@ -33,9 +33,8 @@
 //      O^T[D x 8] += V^T[D x 16 tok] . P^T[16 x 8]       (V via ldmatrix.trans)
 //    fp8 E4M3 tiles are read with 128-bit shared loads and converted in
 //    registers to f16 pairs (exact); the contraction order is permuted so
-//    that every lane's operands are contiguous bytes; when an item's next
-//    block has already landed, two fp8 tiles share one step (one softmax
-//    update for 32 tokens);
+//    that every lane's operands are contiguous bytes; an item's fp8 tiles go
+//    two by two through one step (one softmax update for 32 tokens);
 //  * at an item's last block the consumer writes the output (one-partition
 //    sequences) or (O / l, m, l) partials; paged_decode_merge_kernel, launched
 //    as a programmatic dependent of this grid, combines split sequences with
@@ -796,6 +795,7 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
     WarpAttn<D, C::kFp8, C::kBf16> A;
     A.reset();
     int stage_i = 0, item_i = 0;
+    int blk = 0;  // block of the current item (fp8 pairing)
     int cur_s = 0, cur_head0 = 0, cur_nheads = 0, cur_part = 0, cur_np = 1;
 
     while (true) {
@@ -830,16 +830,23 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
         A.reset();
       }
       const int valid = (md.w >> 8) & 0xff;
-      // fp8: when the item's next block is already in the ring, take both
-      // tiles in one step (one softmax update for 32 tokens)
+      if (md.w & kFirst) blk = 0;
+      // fp8: blocks 2k and 2k+1 of an item go through one step (one softmax
+      // update for 32 tokens).  The pairing depends only on the block's
+      // position in its item, so results do not depend on timing.
       bool two = false;
       int st2 = 0;
       if constexpr (C::kFp8) {
-        if (!(md.w & kLast)) {
+        if (!(md.w & kLast) && !(blk & 1)) {
           st2 = (stage_i + 1) % NS;
-          two = __all_sync(0xffffffffu, mbar_test_wait(full0 + 8 * st2, ((stage_i + 1) / NS) & 1));
+          if (!mbar_wait(full0 + 8 * st2, ((stage_i + 1) / NS) & 1)) {
+            atomicOr(p.err, kCheckWaitTimeout);
+            break;
+          }
+          two = true;
         }
       }
+      blk += two ? 2 : 1;
       int last = md.w & kLast;
       if (two) {
         const int4 md2 = meta[st2];
