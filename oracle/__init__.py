@@ -19,10 +19,16 @@ pages it cites:
 * ``attention``   -- decode attention softmax(scale * q K^T) V in fp64, computed
                      directly over the re-assembled K/V in two explicit passes
                      (max, then exp/sum).  It does NOT use the online-softmax
-                     recurrence that the GPU path uses.
+                     recurrence that the GPU path uses.  ``prefill_attention``:
+                     the same for several causal query rows per sequence
+                     (prefill, chunked prefill).
 * ``cache_write`` -- the per-token slot write (reshape_and_cache).
 * ``block_copy``  -- whole-block copies (copy-on-write fork, CPU swap).
 * ``prefix_sharing`` -- the whole blocks a group of forked sequences shares.
+* ``block_manager`` -- the host allocator: free list, reference counts,
+                     append / fork with copy-on-write, prefix cache, LRU release
+                     (page "5.KV Cache 管理 & PagedAttention", Q9, Q10, Q12, Q18,
+                     Q20).
 * ``fp8_e4m3``    -- an OCP FP8 E4M3 codec written from the format definition.
 * ``dtypes``      -- raw 16-bit / 8-bit storage -> fp64 values.
 * ``kv_size``     -- the pages' closed-form KV-cache size.
