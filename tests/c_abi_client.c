@@ -11,6 +11,7 @@
  * "<what> <values...>"; the test compares the lines with the oracle's.
  */
 #include <stdio.h>
+#include <string.h>
 
 #include "block_manager.h"
 #include "paged_attn.h"
@@ -117,8 +118,9 @@ int main(void) {
 
   /* the attention context rejects a configuration whose head counts do not divide */
   {
-    pa_config cfg = {0};
+    pa_config cfg;
     pa_ctx* ctx = NULL;
+    memset(&cfg, 0, sizeof cfg);
     cfg.num_heads = 32;
     cfg.num_kv_heads = 5;
     cfg.head_dim = 128;

@@ -81,6 +81,16 @@ def client(tmp_path_factory):
     return exe
 
 
+def test_headers_compile_as_cxx():
+    """The same client compiles as C++ too (the headers' extern "C" guards)."""
+    if shutil.which("g++") is None:
+        pytest.skip("g++ not available")
+    r = subprocess.run(["g++", "-x", "c++", "-std=c++17", "-Wall", "-Wextra", "-Werror", "-fsyntax-only", "-I",
+                        os.path.join(ROOT, "include"), os.path.join(HERE, "c_abi_client.c")],
+                       capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
 def test_c_client_matches_the_oracle(client):
     r = subprocess.run([client], capture_output=True, text=True, timeout=60)
     assert r.returncode == 0, r.stdout + r.stderr
