@@ -251,6 +251,294 @@ def run_reference(args, world, rank):
     return 0
 
 
+class DecodeBench:
+    """One workload on one GPU: its seeded inputs in HBM, a library context,
+    and CUDA graphs of one whole step (cache write + decode call) and of the
+    decode call alone."""
+
+    def __init__(self, spec: wl.WorkloadSpec, args, local: int, shared_opt: str = "auto"):
+        self.spec, self.args, self.local = spec, args, local
+        self.dev = dev = f"cuda:{local}"
+        self.w = w = wl.make_workload(spec, dev)
+        part = {"auto": pab.PA_PARTITION_AUTO, "none": pab.PA_PARTITION_NONE}.get(args.partition)
+        part = int(args.partition) if part is None else part
+        self.shared = shared = w.group_start is not None and shared_opt != "off"
+        if shared_opt == "on" and not shared:
+            raise SystemExit(f"workload {spec.name} has no shared-prefix groups")
+        self.pa = pa = pab.PagedAttention(spec.num_heads, spec.num_kv_heads, spec.head_dim, w.num_blocks,
+                                          block_size=spec.block_size, q_dtype=spec.q_dtype, kv_dtype=spec.kv_dtype,
+                                          max_num_seqs=spec.num_seqs, max_blocks_per_seq=w.block_tables.shape[1],
+                                          partition_tokens=part, device=local, shared_prefix=shared)
+        if spec.kv_dtype == "fp8_e4m3":  # the pool quantised once by the library's own cache write
+            NB, bs, Hkv, D = w.key_src.shape
+            self.kc = torch.empty((NB, bs, Hkv, D), dtype=torch.float8_e4m3fn, device=dev)
+            self.vc = torch.empty_like(self.kc)
+            pa.reshape_and_cache(w.key_src.view(-1, Hkv, D), w.value_src.view(-1, Hkv, D), self.kc, self.vc,
+                                 torch.arange(NB * bs, dtype=torch.int64, device=dev), w.k_scale, w.v_scale)
+            w.key_src = w.value_src = None
+        else:
+            self.kc, self.vc = w.key_cache, w.value_cache
+        self.out = torch.empty_like(w.query)
+        self.stream = torch.cuda.current_stream()
+        self.max_len = w.max_seq_len
+        self.chosen_part = pa.get_partition_tokens()
+        # cache write + decode, + the merge kernel (auto partitioning or a split),
+        # + the prefix pass (shared-prefix decode)
+        self.launches_per_step = 2 + (1 if (self.chosen_part < 0 or shared or 0 < self.chosen_part < self.max_len)
+                                      else 0) + (1 if shared else 0)
+        if shared:
+            gsizes = (w.group_start[1:] - w.group_start[:-1]).cpu()
+            self.max_group = int(gsizes.max().item())
+            self.max_prefix = int(w.group_prefix_len.max().item())
+        self.dec_bytes = wl.decode_bytes(w)
+        # bytes the call must move: with shared prefixes, each group's prefix once
+        self.alg_bytes = wl.shared_decode_bytes(w) if shared else self.dec_bytes
+        self.g_step = self.g_dec = None
+
+    def attend(self, q, bt, lens, o=None, st=None):
+        w, pa = self.w, self.pa
+        o = self.out if o is None else o
+        st = self.stream if st is None else st
+        if self.shared:
+            pa.paged_attention_decode_shared_prefix(o, q, self.kc, self.vc, bt, lens, self.max_len, w.group_start,
+                                                    w.group_prefix_len, self.max_group, self.max_prefix, w.scale,
+                                                    w.k_scale, w.v_scale, st)
+        else:
+            pa.paged_attention_decode(o, q, self.kc, self.vc, bt, lens, self.max_len, w.scale, w.k_scale,
+                                      w.v_scale, st)
+
+    def write(self, k, v, slots, st=None):
+        w = self.w
+        self.pa.reshape_and_cache(k, v, self.kc, self.vc, slots, w.k_scale, w.v_scale,
+                                  self.stream if st is None else st)
+
+    def step(self):
+        w = self.w
+        self.write(w.new_key, w.new_value, w.slot_mapping)
+        self.attend(w.query, w.block_tables, w.seq_lens)
+
+    def warm_and_capture(self, warmup: int, graph: bool):
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize()
+        if self.pa.get_error() != 0:
+            raise SystemExit("device check fired during warm-up")
+        if graph:
+            w = self.w
+            side = torch.cuda.Stream(device=self.dev)
+            side.wait_stream(self.stream)
+            self.g_step, self.g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+            with torch.cuda.graph(self.g_step, stream=side):
+                self.write(w.new_key, w.new_value, w.slot_mapping, side)
+                self.attend(w.query, w.block_tables, w.seq_lens, self.out, side)
+            with torch.cuda.graph(self.g_dec, stream=side):
+                self.attend(w.query, w.block_tables, w.seq_lens, self.out, side)
+            self.stream.wait_stream(side)
+            for _ in range(warmup):
+                self.g_step.replay()
+            torch.cuda.synchronize()
+
+    def timed_steps(self, steps: int, world: int):
+        """K whole steps between a barrier + synchronize on each side; returns
+        (total ms max over ranks, per-step cache-write ms list or None, decode ms list or None, clocks)."""
+        w, st = self.w, self.stream
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        with ClockSampler(self.local) as clk:
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            t0.record(st)
+            for i in range(steps):
+                if self.g_step is not None:
+                    self.g_step.replay()
+                    continue
+                a, m, e = ev[i]
+                a.record(st)
+                self.write(w.new_key, w.new_value, w.slot_mapping)
+                m.record(st)
+                self.attend(w.query, w.block_tables, w.seq_lens)
+                e.record(st)
+            t1.record(st)
+            torch.cuda.synchronize()
+        barrier(world)
+        total = max_over_ranks(t0.elapsed_time(t1), world)
+        if self.pa.get_error() != 0:
+            raise SystemExit("device check fired during the timed region")
+        if self.g_step is None:
+            return total, [a.elapsed_time(m) for a, m, _ in ev], [m.elapsed_time(e) for _, m, e in ev], clk.summary()
+        return total, None, None, clk.summary()
+
+    def decode_loop(self, min_seconds: float):
+        """The decode call alone (its graph, or direct launches), replayed back
+        to back for at least ``min_seconds``; CUDA events on the launching
+        stream around the whole loop, NVML clocks sampled during it.
+        Returns (ms per call, calls, clocks)."""
+        st = self.stream
+        w = self.w
+
+        def once():
+            if self.g_dec is not None:
+                self.g_dec.replay()
+            else:
+                self.attend(w.query, w.block_tables, w.seq_lens)
+
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(st)
+        for _ in range(10):
+            once()
+        e1.record(st)
+        torch.cuda.synchronize()
+        est = max(1e-3, e0.elapsed_time(e1) / 10)
+        n = int(min(200000, max(50, math.ceil(min_seconds * 1e3 / est))))
+        with ClockSampler(self.local) as clk:
+            e0.record(st)
+            for _ in range(n):
+                once()
+            e1.record(st)
+            torch.cuda.synchronize()
+        if self.pa.get_error() != 0:
+            raise SystemExit("device check fired during the decode loop")
+        return e0.elapsed_time(e1) / n, n, clk.summary()
+
+    def end_to_end(self, steps: int, warmup: int, world: int):
+        """The same step through the public API from pinned host buffers:
+        every step uploads its inputs (new K/V, query, slot mapping, block
+        tables, lengths) and reads its output back.  Uploads run on one copy
+        stream and read-backs on another (the two directions of the host link
+        in parallel), into double-buffered device tensors, so step i+1's
+        upload and step i-1's read-back overlap step i's kernels, as in a
+        serving loop.  Returns (ms per step max over ranks, h2d bytes, d2h bytes)."""
+        w, st, dev = self.w, self.stream, self.dev
+        names = ("new_key", "new_value", "query", "slot_mapping", "block_tables", "seq_lens")
+        host = {k: getattr(w, k).cpu().pin_memory() for k in names}
+        dev_in = [{k: torch.empty_like(getattr(w, k)) for k in host} for _ in range(2)]
+        outs = [torch.empty_like(self.out) for _ in range(2)]
+        out_host = [torch.empty(self.out.shape, dtype=self.out.dtype).pin_memory() for _ in range(2)]
+        h2d = sum(t.numel() * t.element_size() for t in host.values())
+        d2h = out_host[0].numel() * out_host[0].element_size()
+        up, down = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_read = [torch.cuda.Event() for _ in range(2)]
+        for e in ev_done + ev_read:
+            e.record(st)
+
+        def upload(i):
+            b = i % 2
+            up.wait_event(ev_done[b])  # step i - 2's kernels are done with these inputs
+            with torch.cuda.stream(up):
+                for k, t in host.items():
+                    dev_in[b][k].copy_(t, non_blocking=True)
+            ev_in[b].record(up)
+
+        def compute_and_read_back(i):
+            b = i % 2
+            st.wait_event(ev_in[b])
+            st.wait_event(ev_read[b])  # step i - 2's output has been read back
+            d = dev_in[b]
+            self.write(d["new_key"], d["new_value"], d["slot_mapping"])
+            self.attend(d["query"], d["block_tables"], d["seq_lens"], outs[b])
+            ev_done[b].record(st)
+            down.wait_event(ev_done[b])
+            with torch.cuda.stream(down):
+                out_host[b].copy_(outs[b], non_blocking=True)
+            ev_read[b].record(down)
+
+        def run(n):
+            upload(0)
+            for i in range(n):
+                if i + 1 < n:
+                    upload(i + 1)
+                compute_and_read_back(i)
+            tail = torch.cuda.Event()
+            tail.record(down)
+            st.wait_event(tail)  # the last read-back is inside the timed region
+
+        run(warmup)
+        barrier(world)
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s0.record(st)
+        run(steps)
+        s1.record(st)
+        torch.cuda.synchronize()
+        ms = max_over_ranks(s0.elapsed_time(s1), world)
+        if self.pa.get_error() != 0:
+            raise SystemExit("device check fired during the end-to-end steps")
+        return ms / steps, h2d, d2h
+
+    def close(self):
+        self.g_step = self.g_dec = None
+        self.pa.close()
+
+
+def _workload_config(b: DecodeBench, graph: bool, world: int) -> dict:
+    spec, w = b.spec, b.w
+    return {"workload": spec.name, "description": spec.description, "num_seqs": spec.num_seqs,
+            "num_heads": spec.num_heads, "num_kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim,
+            "block_size": spec.block_size, "kv_dtype": spec.kv_dtype, "q_dtype": spec.q_dtype,
+            "sum_seq_len": int(w.seq_lens.sum().item()),
+            "partition_tokens": "auto (chosen by the decode kernel from the lengths)" if b.chosen_part < 0
+            else b.chosen_part,
+            "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
+            "shared_prefix": bool(b.shared),
+            "launch": "one CUDA graph replay per step" if graph else "eager launches",
+            "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"}
+
+
+def _roofline(b: DecodeBench, dec_ms: float, peak: float, peak_kind: str, traffic):
+    achieved = b.alg_bytes / (dec_ms * 1e-3) / 1e9
+    r = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+         "traffic": traffic,
+         "kernel": ("paged_prefix_kernel + paged_decode_kernel + merge (the whole call)" if b.shared
+                    else "paged_decode_kernel"),
+         "algorithmic_bytes": b.alg_bytes,
+         "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+         if peak_kind == "measured" else "fallback 6.65 TB/s"}
+    if traffic is not None:
+        r["traffic_note"] = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of the decode kernel on the "
+                             "16-sequence case of this workload, scaled x4 to the 64-sequence launch")
+    return r
+
+
+def workload_entry(spec: wl.WorkloadSpec, args, local: int, shared_opt: str, peak: float, peak_kind: str) -> dict:
+    """Device-timed decode call (>= 1 s of back-to-back graph replays), the
+    whole step and the end-to-end step of one more workload (1 GPU)."""
+    b = DecodeBench(spec, args, local, shared_opt)
+    try:
+        b.warm_and_capture(args.warmup, args.graph)
+        total_ms, _, _, _ = b.timed_steps(args.steps, 1)
+        dec_ms, calls, clocks = b.decode_loop(args.decode_seconds)
+        e2e_ms, h2d, d2h = b.end_to_end(args.steps, args.warmup, 1)
+        S = spec.num_seqs
+        gbs = b.dec_bytes / (dec_ms * 1e-3) / 1e9
+        e = {"workload": spec.name, "config": _workload_config(b, args.graph, 1),
+             "decode_ms": dec_ms, "decode_calls_timed": calls,
+             "gbs": gbs, "unit": "GB/s (the metric's byte formula: every sequence's whole length)",
+             "pct_of_nominal_8tbs": 100.0 * gbs / NOMINAL_HBM_GBS, "pct_of_measured_copy": 100.0 * gbs / peak,
+             "seq_steps_per_s": S / (dec_ms * 1e-3), "bytes_per_call": b.dec_bytes,
+             "step_ms": total_ms / args.steps, "step_gbs": b.dec_bytes / (total_ms / args.steps * 1e-3) / 1e9,
+             "roofline": _roofline(b, dec_ms, peak, peak_kind, None),
+             "e2e": {"gbs": b.dec_bytes / (e2e_ms * 1e-3) / 1e9, "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d,
+                     "d2h_bytes_per_step": d2h},
+             "gpu_launches_per_step": b.launches_per_step, "clocks": clocks}
+        if spec.prefix_groups:
+            e["unique_bytes_per_call"] = b.alg_bytes
+            e["unique_gbs"] = b.alg_bytes / (dec_ms * 1e-3) / 1e9
+            e["unique_note"] = ("bytes the call must read: each group's shared prefix once plus every private "
+                                "suffix, q and out")
+        return e
+    finally:
+        b.close()
+
+
+# The bench line's extra workloads: the other full-size configurations of the
+# hot path, each timed on the same GPU after the headline one.
+EXTRA_WORKLOADS = [("gqa-70b-like", "auto"), ("long-context-split-kv", "auto"), ("shared-prefix-fp8", "off"),
+                   ("shared-prefix-fp8", "on")]
+
+
 def run_ours(args, world, rank, local):
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA GPU (the product path has no CPU fallback)")
@@ -260,224 +548,78 @@ def run_ours(args, world, rank, local):
     if args.num_seqs:
         spec = wl.scaled(spec, num_seqs=args.num_seqs, pool_blocks=None,
                          prefix_groups=min(spec.prefix_groups, args.num_seqs) if spec.prefix_groups else 0)
-    dev = f"cuda:{local}"
-    w = wl.make_workload(spec, dev)
-    part = {"auto": pab.PA_PARTITION_AUTO, "none": pab.PA_PARTITION_NONE}.get(args.partition)
-    part = int(args.partition) if part is None else part
-    shared = w.group_start is not None and args.shared_prefix != "off"
-    if args.shared_prefix == "on" and not shared:
-        raise SystemExit(f"workload {spec.name} has no shared-prefix groups")
-    pa = pab.PagedAttention(spec.num_heads, spec.num_kv_heads, spec.head_dim, w.num_blocks,
-                            block_size=spec.block_size, q_dtype=spec.q_dtype, kv_dtype=spec.kv_dtype,
-                            max_num_seqs=spec.num_seqs, max_blocks_per_seq=w.block_tables.shape[1],
-                            partition_tokens=part, device=local, shared_prefix=shared)
-    if spec.kv_dtype == "fp8_e4m3":
-        NB, bs, Hkv, D = w.key_src.shape
-        kc = torch.empty((NB, bs, Hkv, D), dtype=torch.float8_e4m3fn, device=dev)
-        vc = torch.empty_like(kc)
-        pa.reshape_and_cache(w.key_src.view(-1, Hkv, D), w.value_src.view(-1, Hkv, D), kc, vc,
-                             torch.arange(NB * bs, dtype=torch.int64, device=dev), w.k_scale, w.v_scale)
-        w.key_src = w.value_src = None
+    peak, peak_kind = measured_hbm_peak()
+    b = DecodeBench(spec, args, local, args.shared_prefix)
+    b.warm_and_capture(args.warmup, args.graph)
+    # ---- device-timed region: K whole steps (each one graph replay of the
+    # cache write + decode call, or direct launches with --eager)
+    total_ms, write_ms, decode_ms, clocks = b.timed_steps(args.steps, world)
+    # ---- the decode call alone, >= decode_seconds of back-to-back replays
+    dec_ms, calls, dec_clocks = b.decode_loop(args.decode_seconds)
+    dec_ms = max_over_ranks(dec_ms, world)
+    if decode_ms is not None:  # eager: the calls inside the timed steps are timed one by one too
+        write_ms = sum(write_ms) / len(write_ms)
     else:
-        kc, vc = w.key_cache, w.value_cache
-    out = torch.empty_like(w.query)
-    stream = torch.cuda.current_stream()
-    max_len = w.max_seq_len
-    chosen_part = pa.get_partition_tokens()
-    # cache write + decode, + the merge kernel (auto partitioning or a split),
-    # + the prefix pass (shared-prefix decode)
-    launches_per_step = 2 + (1 if (chosen_part < 0 or shared or 0 < chosen_part < max_len) else 0) + \
-        (1 if shared else 0)
-    if shared:
-        gsizes = (w.group_start[1:] - w.group_start[:-1]).cpu()
-        max_group = int(gsizes.max().item())
-        max_prefix = int(w.group_prefix_len.max().item())
+        write_ms = max(0.0, total_ms / args.steps - dec_ms)
+    # ---- end to end through the public API, host buffers every step
+    e2e_step_ms, h2d, d2h = b.end_to_end(args.steps, args.warmup, world)
 
-    def attend(q, bt, lens, o=None, st=None):
-        o = out if o is None else o
-        st = stream if st is None else st
-        if shared:
-            pa.paged_attention_decode_shared_prefix(o, q, kc, vc, bt, lens, max_len, w.group_start,
-                                                    w.group_prefix_len, max_group, max_prefix, w.scale,
-                                                    w.k_scale, w.v_scale, st)
-        else:
-            pa.paged_attention_decode(o, q, kc, vc, bt, lens, max_len, w.scale, w.k_scale, w.v_scale, st)
-
-    def step():
-        pa.reshape_and_cache(w.new_key, w.new_value, kc, vc, w.slot_mapping, w.k_scale, w.v_scale, stream)
-        attend(w.query, w.block_tables, w.seq_lens)
-
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
-    if pa.get_error() != 0:
-        raise SystemExit("device check fired during warm-up")
-
-    # ---- device-timed region: whole steps, plus the decode call inside each
-    # (--graph: each step is one replay of a CUDA graph captured from the same
-    # calls; the decode-call time then comes from a decode-only graph)
-    g_step = g_dec = None
-    if args.graph:
-        side = torch.cuda.Stream(device=dev)
-        side.wait_stream(stream)
-        g_step, g_dec = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_step, stream=side):
-            pa.reshape_and_cache(w.new_key, w.new_value, kc, vc, w.slot_mapping, w.k_scale, w.v_scale, side)
-            attend(w.query, w.block_tables, w.seq_lens, out, side)
-        with torch.cuda.graph(g_dec, stream=side):
-            attend(w.query, w.block_tables, w.seq_lens, out, side)
-        stream.wait_stream(side)
-        for _ in range(args.warmup):
-            g_step.replay()
-        torch.cuda.synchronize()
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
-           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    barrier(world)
-    torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
-        t_start = torch.cuda.Event(enable_timing=True)
-        t_end = torch.cuda.Event(enable_timing=True)
-        t_start.record(stream)
-        for i in range(args.steps):
-            a, m, e = ev[i]
-            if g_step is not None:
-                g_step.replay()
-                continue
-            a.record(stream)
-            pa.reshape_and_cache(w.new_key, w.new_value, kc, vc, w.slot_mapping, w.k_scale, w.v_scale, stream)
-            m.record(stream)
-            attend(w.query, w.block_tables, w.seq_lens)
-            e.record(stream)
-        t_end.record(stream)
-        torch.cuda.synchronize()
-    barrier(world)
-    total_ms = t_start.elapsed_time(t_end)
-    if g_step is None:
-        decode_ms = [m.elapsed_time(e) for (_, m, e) in ev]
-        write_ms = [a.elapsed_time(m) for (a, m, _) in ev]
-    else:
-        d0, d1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        d0.record(stream)
-        for _ in range(args.steps):
-            g_dec.replay()
-        d1.record(stream)
-        torch.cuda.synchronize()
-        decode_ms = [d0.elapsed_time(d1) / args.steps]
-        write_ms = [max(0.0, total_ms / args.steps - decode_ms[0])]
-    total_ms = max_over_ranks(total_ms, world)
-    if pa.get_error() != 0:
-        raise SystemExit("device check fired during the timed region")
-
-    dec_bytes = wl.decode_bytes(w)
     S = spec.num_seqs
     ms_per_step = total_ms / args.steps
-    value = world * dec_bytes * args.steps / (total_ms * 1e-3) / 1e9
+    value = world * b.dec_bytes * args.steps / (total_ms * 1e-3) / 1e9
     seq_steps = world * S * args.steps / (total_ms * 1e-3)
-
-    # ---- end to end through the public API: every step copies its inputs
-    # from pinned host memory to the device and reads its output back.  The
-    # copies run on a second stream into double-buffered device inputs, so
-    # step i+1's upload overlaps step i's kernels (as a serving loop would).
-    host = {k: getattr(w, k).cpu().pin_memory() for k in ("new_key", "new_value", "query", "slot_mapping",
-                                                          "block_tables", "seq_lens")}
-    dev_in = [{k: torch.empty_like(getattr(w, k)) for k in host} for _ in range(2)]
-    outs = [torch.empty_like(out) for _ in range(2)]
-    out_host = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
-    h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = out_host[0].numel() * out_host[0].element_size()
-    copy = torch.cuda.Stream(device=dev)
-    ev_in = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-
-    def upload(i):
-        b = i % 2
-        copy.wait_event(ev_done[b])  # step i - 2's kernels are done with these buffers
-        with torch.cuda.stream(copy):
-            for k, t in host.items():
-                dev_in[b][k].copy_(t, non_blocking=True)
-        ev_in[b].record(copy)
-
-    def compute_and_download(i):
-        b = i % 2
-        stream.wait_event(ev_in[b])
-        d = dev_in[b]
-        pa.reshape_and_cache(d["new_key"], d["new_value"], kc, vc, d["slot_mapping"], w.k_scale, w.v_scale, stream)
-        attend(d["query"], d["block_tables"], d["seq_lens"], outs[b])
-        ev_done[b].record(stream)
-        copy.wait_event(ev_done[b])
-        with torch.cuda.stream(copy):
-            out_host[b].copy_(outs[b], non_blocking=True)
-
-    def e2e_run(n):
-        upload(0)
-        for i in range(n):
-            if i + 1 < n:
-                upload(i + 1)
-            compute_and_download(i)
-        tail = torch.cuda.Event()
-        tail.record(copy)
-        stream.wait_event(tail)  # the last read-back is inside the timed region
-
-    e2e_run(args.warmup)
-    barrier(world)
-    torch.cuda.synchronize()
-    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s0.record(stream)
-    e2e_run(args.steps)
-    s1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(s0.elapsed_time(s1), world)
-    e2e_value = world * dec_bytes * args.steps / (e2e_ms * 1e-3) / 1e9
-
-    peak, peak_kind = measured_hbm_peak()
-    dec_avg_ms = sum(decode_ms) / len(decode_ms)
-    # bytes the call must move: with shared prefixes, each group's prefix once
-    alg_bytes = wl.shared_decode_bytes(w) if shared else dec_bytes
-    achieved = alg_bytes / (dec_avg_ms * 1e-3) / 1e9
-    traffic = None if shared else traffic_record("paged_decode_kernel", spec.name)
+    e2e_value = world * b.dec_bytes / (e2e_step_ms * 1e-3) / 1e9
+    traffic = None if b.shared else traffic_record("paged_decode_kernel", spec.name)
     result = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": {"f16": "f16", "bf16": "bf16", "fp8_e4m3": "fp8_e4m3"}[spec.kv_dtype],
         "data": "synthetic",
-        "config": {"workload": spec.name, "description": spec.description, "num_seqs": S,
-                   "num_heads": spec.num_heads, "num_kv_heads": spec.num_kv_heads, "head_dim": spec.head_dim,
-                   "block_size": spec.block_size, "kv_dtype": spec.kv_dtype, "q_dtype": spec.q_dtype,
-                   "sum_seq_len": int(w.seq_lens.sum().item()),
-                   "partition_tokens": "auto (chosen by the decode kernel from the lengths)" if chosen_part < 0
-                   else chosen_part,
-                   "l2": "inputs larger than L2 (KV read per step >> 126 MB), no flush",
-                   "shared_prefix": bool(shared),
-                   "launch": "one CUDA graph replay per step" if args.graph else "eager launches",
-                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU"},
+        "config": _workload_config(b, args.graph, world),
         "seq_steps_per_s": seq_steps,
         "pct_of_nominal_8tbs": 100.0 * value / world / NOMINAL_HBM_GBS,
         "pct_of_measured_copy": 100.0 * value / world / peak,
-        "bytes_per_step": dec_bytes,
+        "bytes_per_step": b.dec_bytes,
         "bytes_note": ("value counts every sequence's prefix (the metric's byte formula); the roofline counts "
-                       "each group's shared prefix once (the bytes the call must read)") if shared else None,
-        "decode_ms": dec_avg_ms, "cache_write_ms": sum(write_ms) / len(write_ms),
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic,
-                     "kernel": ("paged_prefix_kernel + paged_decode_kernel + merge (the whole call)" if shared
-                                else "paged_decode_kernel"),
-                     "algorithmic_bytes": alg_bytes,
-                     "peak_kind": f"{peak_kind} copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
-                     if peak_kind == "measured" else "fallback 6.65 TB/s"},
+                       "each group's shared prefix once (the bytes the call must read)") if b.shared else None,
+        "decode_ms": dec_ms, "decode_calls_timed": calls,
+        "decode_timing": (f"{calls} back-to-back replays of the decode call's CUDA graph" if args.graph
+                          else f"{calls} back-to-back direct decode calls") +
+                         ", CUDA events on the launching stream around the loop; NVML clocks in decode_clocks",
+        "decode_clocks": dec_clocks,
+        "cache_write_ms": write_ms,
+        "roofline": _roofline(b, dec_ms, peak, peak_kind, traffic),
         "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "ms_per_step": e2e_ms / args.steps,
-                "how": "pinned host inputs -> device (copy stream, double-buffered) -> cache write + decode -> "
-                       "output -> pinned host, every step; uploads overlap the previous step's kernels"},
-        "gpu_launches": launches_per_step * args.steps,
-        "clocks": clk.summary(),
+                "ms_per_step": e2e_step_ms,
+                "how": "pinned host inputs -> device (upload stream, double-buffered) -> cache write + decode -> "
+                       "output -> pinned host (read-back stream), every step; uploads and read-backs overlap "
+                       "the neighbouring steps' kernels"},
+        "gpu_launches": b.launches_per_step * args.steps,
+        "clocks": clocks,
     }
+    b.close()
+    del b
+    torch.cuda.empty_cache()
+    if world == 1 and args.workload == DEFAULT_WORKLOAD and not args.num_seqs and not args.no_extra:
+        per = []
+        for name, sp_opt in EXTRA_WORKLOADS:
+            per.append(workload_entry(wl.SPEC_BY_NAME[name], args, local, sp_opt, peak, peak_kind))
+            torch.cuda.empty_cache()
+        result["per_workload"] = per
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         gbs, sps, desc, threads, el = oracle_sample(spec, args.cpu_budget)
         result["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
                                   "sample": desc, "seq_steps_per_s": sps, "seconds": el}
+        try:
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                g1, s1, d1, _, e1 = oracle_sample(spec, args.cpu_budget / 2)
+            result["cpu_baseline"]["one_core"] = {"value": g1, "unit": "GB/s", "cores": 1, "sample": d1,
+                                                  "seq_steps_per_s": s1, "seconds": e1}
+        except ImportError:
+            pass
     if rank == 0:
         print(json.dumps(result), flush=True)
-    pa.close()
     return 0
 
 
@@ -736,6 +878,10 @@ def main():
                     help="shared-prefix decode for workloads with prefix groups (auto: when the workload has them)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for cpu_baseline")
+    ap.add_argument("--decode-seconds", type=float, default=1.0,
+                    help="minimum length of the back-to-back decode-call loop behind decode_ms and the roofline")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other full-size workloads (per_workload) of the default run")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

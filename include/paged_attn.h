@@ -246,6 +246,22 @@ int paged_attention_prefill(pa_ctx* ctx, void* out, const void* query, const voi
  */
 int paged_attn_get_error(pa_ctx* ctx, void* stream);
 
+/*
+ * Failure-path test hook (the pages describe no counterpart; it exists so
+ * that the device-side timeout exit can be exercised without any GPU fault).
+ * The next paged_attention_decode or paged_attention_decode_shared_prefix on
+ * this context runs its decode kernel with every pipeline wait bounded by
+ * wait_limit_cycles SM clock cycles instead of the default (~2 s), and with
+ * the first wait of each consumer warp aimed at a barrier that nothing ever
+ * completes.  Every CTA of that launch therefore gives up after about
+ * wait_limit_cycles, waits (with the default bound) for the copies it has in
+ * flight, and exits; the call's output is invalid and paged_attn_get_error()
+ * reports PA_CHECK_WAIT_TIMEOUT.  Later calls run normally.  One-shot.
+ * wait_limit_cycles: [1000, the default limit].  Returns PA_OK or
+ * PA_ERR_INVALID_ARG.
+ */
+int paged_attn_test_wait_timeout(pa_ctx* ctx, long long wait_limit_cycles);
+
 /* Check bits seen by the last paged_attn_get_error (PA_CHECK_*). */
 int paged_attn_last_check_bits(const pa_ctx* ctx);
 
@@ -303,8 +319,10 @@ int paged_copy_blocks(pa_ctx* ctx, void* dst_key_cache, void* dst_value_cache, i
 /*
  * Decode attention that allocates nothing (the pages describe no counterpart:
  * it exists for callers of this library that cannot allocate device memory,
- * e.g. code running while its stream is being captured into a CUDA graph, or
- * hosts that own every device allocation through their own pool).
+ * e.g. hosts that hand out every byte of device memory from their own pool or
+ * arena and forbid outside allocations, or serving loops that must not risk
+ * an allocation failure, or the allocator's implicit device synchronisation,
+ * in the middle of a step).
  *
  * Same computation, layouts and argument meanings as paged_attention_decode,
  * but without a context: the cache shape is passed directly (num_heads,
@@ -320,8 +338,13 @@ int paged_copy_blocks(pa_ctx* ctx, void* dst_key_cache, void* dst_value_cache, i
  * check_bits: optional device int that receives PA_CHECK_* bits (or-ed in;
  * the caller clears it); NULL sends them to a word inside the array.
  * Runs on the calling thread's current CUDA device.  The first call on each
- * device looks up the array's device address and raises the decode kernel's
- * shared-memory limit; make that first call before any stream capture.
+ * device does a one-time set-up there: it looks up the array's device
+ * address, raises the shared-memory limit of every decode kernel the library
+ * holds (all head_dim / dtype combinations), and clears the array's 256-byte
+ * header (check word and work counters) with an asynchronous memset on
+ * `stream`, ordered before that call's kernels on any kind of stream.  A
+ * caller that captures streams into CUDA graphs should make this first call
+ * before any capture.  Later calls change no host or device setting.
  * Every call on a device shares the array and finds it as the previous call
  * left it; calls whose kernels may overlap on the GPU (other streams or host
  * threads on the same device) race on it and must be serialised by the caller.

@@ -96,7 +96,7 @@ class BlockManager:
 
     def allocate(self) -> int:
         if not self.free_blocks and not self._evict_one_cached():
-            raise OutOfBlocks(f"All {self.num_blocks} blocks are in use.")
+            raise OutOfBlocks(f"no free block left in a pool of {self.num_blocks}")
         blk = self.free_blocks.pop()
         self.ref_counts[blk] = 1
         return blk

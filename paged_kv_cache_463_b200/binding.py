@@ -70,6 +70,7 @@ def load_library(path: str | None = None) -> ctypes.CDLL:
                                                      _P]),
         "paged_attention_prefill": (i, [_P, _P, _P, _P, _P, _P, i, _P, _P, i, i, i, i, f, f, f, _P]),
         "paged_attn_get_error": (i, [_P, _P]),
+        "paged_attn_test_wait_timeout": (i, [_P, ctypes.c_longlong]),
         "paged_attn_last_check_bits": (i, [_P]),
         "paged_attn_status_string": (ctypes.c_char_p, [i]),
         "paged_attn_last_error": (ctypes.c_char_p, [_P]),
@@ -250,6 +251,13 @@ class PagedAttention:
             return self.lib.paged_attn_last_check_bits(self.ctx)
         self._check(st, "paged_attn_get_error")
         return 0
+
+    def test_wait_timeout(self, wait_limit_cycles: int) -> None:
+        """Failure-path test hook: the next decode call's waits are bounded by
+        ``wait_limit_cycles`` and its consumers wait on a barrier nothing
+        completes, so the call must take the timeout exit (one-shot)."""
+        self._check(self.lib.paged_attn_test_wait_timeout(self.ctx, int(wait_limit_cycles)),
+                    "paged_attn_test_wait_timeout")
 
     def set_partition_tokens(self, n: int) -> None:
         self._check(self.lib.paged_attn_set_partition_tokens(self.ctx, int(n)), "paged_attn_set_partition_tokens")

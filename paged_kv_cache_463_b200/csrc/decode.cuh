@@ -93,6 +93,11 @@ struct DecodeParams {
   const float* pre_o = nullptr;   // [S, Hq, max_chunks, D]
   const float* pre_ml = nullptr;  // [S, Hq, max_chunks, 2]
   int max_chunks = 0;
+  // failure-path test hook: every pipeline wait of the launch is bounded by
+  // wait_limit cycles, and with debug_stall the consumer's first wait targets
+  // a barrier that nothing completes, so the launch must take its timeout exit
+  long long wait_limit = kWaitLimitCycles;
+  int debug_stall = 0;
 };
 
 constexpr int kPrefixChunkBlocks = 32;  // blocks per partial of the prefix pass
@@ -140,14 +145,19 @@ __device__ __forceinline__ Pieces unit_pieces(int a, int nblk, int per_group) {
 }
 
 // Shared-memory layout of a decode CTA (offsets from a 1024-aligned base):
-// ring[NS stages] | query slots[2] | mbarriers | stage metadata | prefix[S+1], lens[S]
+// ring[NS stages] | query slots[2] | mbarriers | exit record | stage metadata | prefix[S+1], lens[S]
+// mbarriers: full[NS], empty[NS], qfull[2], qempty[2], and one that nothing
+// completes (the target of the failure-path test hook).  Exit record: stages
+// and query slots the consumer took, and a flag set by a wait that ran out.
+__host__ __device__ constexpr int kDecodeBarriers(int ns) { return 2 * ns + 5; }
 struct DecodeLayout {
-  int ring, q, bar, meta, prefix;
+  int ring, q, bar, exitrec, meta, prefix;
   __host__ __device__ DecodeLayout(int ns, int stage_bytes, int q_slot_bytes) {
     ring = 0;
     q = ns * stage_bytes;
     bar = q + 2 * q_slot_bytes;
-    meta = (bar + (2 * ns + 4) * 8 + 15) & ~15;
+    exitrec = (bar + kDecodeBarriers(ns) * 8 + 15) & ~15;
+    meta = exitrec + 16;
     prefix = meta + ns * 16;
   }
   // bytes of dynamic shared memory for up to `max_seqs` sequences (+ alignment slack)
@@ -503,6 +513,9 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
   const DecodeLayout L(NS, C::STAGE_BYTES, p.q_slot_bytes);
   const uint32_t base_u32 = smem_u32(smem);
   const uint32_t full0 = base_u32 + L.bar, empty0 = full0 + NS * 8, qfull0 = full0 + 2 * NS * 8, qempty0 = qfull0 + 16;
+  const uint32_t never = qempty0 + 16;  // no thread ever arrives on it
+  volatile int* exitrec = reinterpret_cast<volatile int*>(smem + L.exitrec);  // [0] stages, [1] q slots, [2] timed out
+  const long long wl = p.wait_limit;
   int4* meta = reinterpret_cast<int4*>(smem + L.meta);
   int* prefix = reinterpret_cast<int*>(smem + L.prefix);  // [S + 1]
   int* lens = prefix + (S + 1);                             // [S], clamped
@@ -588,11 +601,16 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
     }
   }
   if (threadIdx.x == 0) {
-    for (int i = 0; i < 2 * NS + 4; ++i) mbar_init(full0 + 8 * i, 1);
+    for (int i = 0; i < kDecodeBarriers(NS); ++i) mbar_init(full0 + 8 * i, 1);
     fence_mbar_init();
+    exitrec[0] = exitrec[1] = exitrec[2] = 0;
   }
   __syncthreads();
   const int total = prefix[S];  // items (ticket mode) or blocks (stream-K mode)
+  // Copies this CTA's producer has issued (lane 0 counts): ring stages armed
+  // and query slots filled, in order.  After a wait runs out, the ones the
+  // consumer did not take are waited for before the CTA exits.
+  int armed = 0, q_armed = 0;
 
   if (warp == 1) {
     // ---------------------------------------------------------------- producer
@@ -604,8 +622,9 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
     // Claim stage `stage_i` (lane 0): wait until the consumer released its last use.
     auto claim = [&](int& st) -> bool {
       st = stage_i % NS;
-      if (stage_i >= NS && !mbar_wait(empty0 + 8 * st, ((stage_i / NS) - 1) & 1)) {
+      if (stage_i >= NS && !mbar_wait(empty0 + 8 * st, ((stage_i / NS) - 1) & 1, wl)) {
         atomicOr(p.err, kCheckWaitTimeout);
+        exitrec[2] = 1;
         return false;
       }
       return true;
@@ -715,8 +734,9 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
       };
       if (lane == 0) {  // this item's query rows -> q slot
         const int qs = item_i & 1;
-        if (item_i >= 2 && !mbar_wait(qempty0 + 8 * qs, ((item_i >> 1) - 1) & 1)) {
+        if (item_i >= 2 && !mbar_wait(qempty0 + 8 * qs, ((item_i >> 1) - 1) & 1, wl)) {
           atomicOr(p.err, kCheckWaitTimeout);
+          exitrec[2] = 1;
           stop = 1;
         } else {
           const uint32_t bytes = nheads * D * 2;
@@ -724,6 +744,7 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
           bulk_load(base_u32 + L.q + qs * p.q_slot_bytes,
                     reinterpret_cast<const uint8_t*>(p.query) + ((size_t)cur.s * p.num_heads + head0) * D * 2, bytes,
                     qfull0 + 8 * qs);
+          ++q_armed;
         }
       }
       stop = __shfl_sync(0xffffffffu, stop, 0);
@@ -737,6 +758,7 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
           } else {
             meta[st] = make_int4(cur.s, cur.y, meta_z, kFirst | kLast);
             mbar_arrive(full0 + 8 * st);
+            ++armed;
           }
         }
         ++stage_i;
@@ -768,6 +790,7 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
                 tma_load_2d(kdst + sub * kBS * 128, &tmK, x, yy, fb);
                 tma_load_2d(vdst + sub * kBS * 128, &tmV, x, yy, fb);
               }
+              ++armed;
             }
           }
           ++stage_i;
@@ -787,6 +810,7 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
       if (claim(st)) {
         meta[st] = make_int4(0, 0, 0, kEnd);
         mbar_arrive(full0 + 8 * st);
+        ++armed;
       }
     }
   } else {
@@ -800,8 +824,14 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
 
     while (true) {
       const int st = stage_i % NS;
-      if (!mbar_wait(full0 + 8 * st, (stage_i / NS) & 1)) {
+      // (test hook: the first wait targets the barrier nothing completes)
+      const bool stall = p.debug_stall && stage_i == 0;
+      // (all lanes wait; the warp leaves together even if the limit ran out
+      // for some lanes only)
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(stall ? never : full0 + 8 * st, stall ? 0u : (uint32_t)((stage_i / NS) & 1), wl))) {
         atomicOr(p.err, kCheckWaitTimeout);
+        exitrec[2] = 1;
         break;
       }
       const int4 md = meta[st];
@@ -816,8 +846,9 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
         cur_part = md.z & 0xffff;
         cur_np = md.z >> 16;
         const int qs = item_i & 1;
-        if (!mbar_wait(qfull0 + 8 * qs, (item_i >> 1) & 1)) {
+        if (!__all_sync(0xffffffffu, mbar_wait(qfull0 + 8 * qs, (item_i >> 1) & 1, wl))) {
           atomicOr(p.err, kCheckWaitTimeout);
+          exitrec[2] = 1;
           break;
         }
         A.load_q(gid < cur_nheads ? smem + L.q + qs * p.q_slot_bytes + gid * D * 2 : nullptr, c4);
@@ -839,8 +870,9 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
       if constexpr (C::kFp8) {
         if (!(md.w & kLast) && !(blk & 1)) {
           st2 = (stage_i + 1) % NS;
-          if (!mbar_wait(full0 + 8 * st2, ((stage_i + 1) / NS) & 1)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(full0 + 8 * st2, ((stage_i + 1) / NS) & 1, wl))) {
             atomicOr(p.err, kCheckWaitTimeout);
+            exitrec[2] = 1;
             break;
           }
           two = true;
@@ -903,8 +935,22 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
         }
       }
     }
+    if (lane == 0) {  // what this warp took, for the timeout exit below
+      exitrec[0] = stage_i;
+      exitrec[1] = item_i;
+    }
   }
 
+  __syncthreads();
+  // After a wait ran out, the consumer stopped taking stages while TMA and
+  // bulk copies the producer issued may still be landing in this CTA's shared
+  // memory: wait (bounded by the default limit) for every stage and query slot
+  // armed but not taken, so that no copy outlives the CTA.  At most NS stages
+  // and 2 slots are outstanding, each in its own ring position.
+  if (warp == 1 && lane == 0 && exitrec[2]) {
+    for (int k = exitrec[0]; k < armed; ++k) mbar_wait(full0 + 8 * (k % NS), (k / NS) & 1);
+    for (int i = exitrec[1]; i < q_armed; ++i) mbar_wait(qfull0 + 8 * (i & 1), (i >> 1) & 1);
+  }
   // the last CTA to finish resets the counters for the next launch
   __syncthreads();
   if (threadIdx.x == 0) {

@@ -230,6 +230,7 @@ struct pa_ctx {
   int* err_host = nullptr;      // pinned
   int grid = 0;                 // persistent grid: SMs x resident CTAs
   int last_bits = 0;
+  long long test_wait_limit = 0;  // > 0: the next decode launch takes the failure path (test hook)
   KernelSet ks;
   std::unordered_map<const void*, CUtensorMap> maps;
   std::string msg;
@@ -643,6 +644,12 @@ int decode_impl(pa_ctx* ctx, void* out, const void* query, const void* key_cache
     p.max_chunks = ctx->max_chunks;
   }
 
+  if (ctx->test_wait_limit > 0) {  // one-shot failure-path test hook
+    p.wait_limit = ctx->test_wait_limit;
+    p.debug_stall = 1;
+    ctx->test_wait_limit = 0;
+  }
+
   merge_shape(c.head_dim, parts + prefix_chunks, c.num_heads, &p.merge_hpc, &p.merge_slices);
   void* args[] = {&mk, &mv, &p};
   cudaError_t e = cudaLaunchKernel(ctx->ks.decode, dim3(ctx->grid), dim3(ctx->ks.threads), args,
@@ -748,6 +755,14 @@ PA_API int paged_attn_get_error(pa_ctx* ctx, void* stream) {
   return ctx->last_bits ? PA_ERR_DEVICE_CHECK : PA_OK;
 }
 
+PA_API int paged_attn_test_wait_timeout(pa_ctx* ctx, long long wait_limit_cycles) {
+  if (!ctx) return PA_ERR_INVALID_ARG;
+  if (wait_limit_cycles < 1000 || wait_limit_cycles > pa::kWaitLimitCycles)
+    return fail(ctx, PA_ERR_INVALID_ARG, "wait_limit_cycles outside [1000, default limit]");
+  ctx->test_wait_limit = wait_limit_cycles;
+  return PA_OK;
+}
+
 PA_API int paged_gather_kv(pa_ctx* ctx, void* k_out, void* v_out, const void* key_cache, const void* value_cache,
                            const int32_t* block_table_row, int seq_len, void* stream) {
   if (!ctx) return PA_ERR_INVALID_ARG;
@@ -781,19 +796,22 @@ PA_API int paged_gather_kv(pa_ctx* ctx, void* k_out, void* v_out, const void* ke
 // ---------------------------------------------------------------------------
 // Decode without any allocation.
 //
-// Some callers cannot call cudaMalloc at all: code that runs while a CUDA
-// graph is being captured on its stream, hosts that hand out device memory
-// from their own pool and forbid outside allocations, or callers that must not
-// risk an allocation failure (or an allocator's implicit synchronisation) in
-// the middle of a serving step.  For them this entry point needs no context:
-// the split-KV partials live in one file-scope device array of fixed size,
-// which every GPU that loads this library holds until the process exits.
+// Some callers cannot call cudaMalloc at all: hosts that hand out device
+// memory only from their own pool or arena and forbid outside allocations
+// (an inference server that budgets every byte of HBM up front), or callers
+// that must not risk an allocation failure, or the allocator's implicit
+// device synchronisation, in the middle of a serving step.  For them this
+// entry point needs no context: the split-KV partials live in one file-scope
+// device array of fixed size, which every GPU that loads this library holds
+// until the process exits.
 //
 // The array is shared by every call on a device and keeps whatever the last
-// call left in it.  Only the decode kernel's two work-ticket counters must
-// start at zero: the first call on a device clears the whole array, and every
-// launch leaves them at zero again.  Every partial that the merge reads is
-// written earlier in the same call; the check word is only ever or-ed into.  Two calls whose kernels overlap on the GPU (different
+// call left in it.  Only its 256-byte header (the check word and the decode
+// kernel's work-ticket counters) must start at zero: the first call on a
+// device clears it on the caller's stream, ahead of its own kernels, and
+// every launch leaves the counters at zero again.  Every partial that the
+// merge reads is written earlier in the same call; the check word is only
+// ever or-ed into.  Two calls whose kernels overlap on the GPU (different
 // streams, or different host threads, on one device) race on the array.
 // ---------------------------------------------------------------------------
 namespace {
@@ -801,56 +819,52 @@ namespace {
 static __device__ __align__(256) unsigned char g_noalloc_scratch[PA_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxNoallocDevices = 64;
-constexpr size_t kNoallocHeader = 256;  // bytes reserved at the front (check word)
+constexpr size_t kNoallocHeader = 256;  // bytes reserved at the front (check word, work counters)
 
 struct NoallocDevice {
   bool ready = false;
   unsigned char* scratch = nullptr;  // device address of g_noalloc_scratch on this device
   int num_sms = 0;
   int smem_optin = 0;
-  const void* kernel_ready[16] = {};  // decode kernels whose shared-memory limit was raised here
 };
 NoallocDevice g_noalloc_dev[kMaxNoallocDevices];
 std::mutex g_noalloc_mu;
 
-// Device address of the scratch array on `dev` (the current device).  The
-// array's name in host code is only a host-side handle; kernels must be given
-// the address cudaGetSymbolAddress returns with the device current.
-int noalloc_setup(int dev, const void* kernel, const void* merge, unsigned char** scratch, int* num_sms,
-                  int* smem_optin) {
+// Every (head_dim, q_dtype, kv_dtype) the library has decode kernels for.
+constexpr int kDecodeCombos[][3] = {{64, PA_F16, PA_F16},        {128, PA_F16, PA_F16},
+                                    {256, PA_F16, PA_F16},       {64, PA_BF16, PA_BF16},
+                                    {128, PA_BF16, PA_BF16},     {256, PA_BF16, PA_BF16},
+                                    {128, PA_F16, PA_FP8_E4M3},  {256, PA_F16, PA_FP8_E4M3}};
+
+// First call on `dev` (the current device): the device address of the
+// scratch array (its name in host code is only a host-side handle; kernels
+// must be given the address cudaGetSymbolAddress returns with the device
+// current), the shared-memory limit and carve-out of every decode and merge
+// kernel, and the header cleared on `stream`, so that the caller's first
+// kernels, queued after it on the same stream, see zero counters whatever
+// kind of stream it is.  Later calls only read the cached record.
+int noalloc_setup(int dev, cudaStream_t stream, NoallocDevice* out) {
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   NoallocDevice& d = g_noalloc_dev[dev];
   if (!d.ready) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return PA_ERR_CUDA;
-    // the decode kernel's work counters must start at zero (each launch
-    // leaves the ones it used at zero again); clear the whole array once
-    if (cudaMemset(p, 0, PA_NOALLOC_SCRATCH_BYTES) != cudaSuccess) return PA_ERR_CUDA;
     if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
       return PA_ERR_CUDA;
+    for (const auto& c : kDecodeCombos) {
+      KernelSet ks;
+      if (!select_kernels(c[0], c[1], c[2], &ks)) return PA_ERR_CUDA;
+      if (cudaFuncSetAttribute(ks.decode, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) !=
+              cudaSuccess ||
+          pin_carveout(ks.decode) != cudaSuccess || pin_carveout(ks.merge) != cudaSuccess)
+        return PA_ERR_CUDA;
+    }
+    if (cudaMemsetAsync(p, 0, kNoallocHeader, stream) != cudaSuccess) return PA_ERR_CUDA;
     d.scratch = static_cast<unsigned char*>(p);
     d.ready = true;
   }
-  int slot = -1;
-  for (int i = 0; i < 16; ++i) {
-    if (d.kernel_ready[i] == kernel) {
-      slot = i;
-      break;
-    }
-    if (d.kernel_ready[i] == nullptr) {
-      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) != cudaSuccess ||
-          pin_carveout(kernel) != cudaSuccess || pin_carveout(merge) != cudaSuccess)
-        return PA_ERR_CUDA;
-      d.kernel_ready[i] = kernel;
-      slot = i;
-      break;
-    }
-  }
-  if (slot < 0) return PA_ERR_CUDA;
-  *scratch = d.scratch;
-  *num_sms = d.num_sms;
-  *smem_optin = d.smem_optin;
+  *out = d;
   return PA_OK;
 }
 
@@ -908,12 +922,14 @@ PA_API int paged_attention_decode_noalloc(void* out, const void* query, const vo
 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxNoallocDevices) return PA_ERR_CUDA;
-  unsigned char* scratch = nullptr;
-  int num_sms = 0, smem_optin = 0;
-  int st = noalloc_setup(dev, ks.decode, ks.merge, &scratch, &num_sms, &smem_optin);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  NoallocDevice nd;
+  int st = noalloc_setup(dev, s, &nd);
   if (st != PA_OK) return st;
+  unsigned char* scratch = nd.scratch;
+  const int num_sms = nd.num_sms;
   const size_t smem = ks.smem(q_slot_bytes(num_heads, num_kv_heads, head_dim), num_seqs);
-  if (smem > (size_t)smem_optin) return PA_ERR_UNSUPPORTED;
+  if (smem > (size_t)nd.smem_optin) return PA_ERR_UNSUPPORTED;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ks.decode, ks.threads, smem) != cudaSuccess ||
       per_sm < 1)
@@ -951,7 +967,6 @@ PA_API int paged_attention_decode_noalloc(void* out, const void* query, const vo
   p.v_scale = fp8 ? v_scale : 1.0f;
 
   merge_shape(head_dim, parts, num_heads, &p.merge_hpc, &p.merge_slices);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   void* args[] = {&mk, &mv, &p};
   if (cudaLaunchKernel(ks.decode, dim3(num_sms * per_sm), dim3(ks.threads), args, smem, s) != cudaSuccess)
     return PA_ERR_CUDA;

@@ -103,7 +103,7 @@ class RefCountAllocator:
 
     def allocate(self) -> int:
         if not self.free_blocks:
-            raise MemoryError(f"All {self.total} blocks are in use.")
+            raise MemoryError(f"free list empty: pool of {self.total} blocks exhausted")
         blk = self.free_blocks.pop()
         self.ref_counts[blk] = 1
         return blk
