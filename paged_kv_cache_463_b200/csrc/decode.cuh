@@ -497,6 +497,161 @@ struct WarpAttn {
   }
 };
 
+// The launch's work hand-out, computed by one warp of every CTA (all 32
+// lanes call this) from the clamped lengths: lens[S] and the exclusive prefix
+// prefix[S+1] of items (ticket mode) or blocks (stream-K mode) in shared
+// memory.  In auto mode the hand-out is chosen from the lengths: near-uniform
+// lengths (all within 10 %) -> tickets with large partitions (items finish
+// together; the memory system stays saturated), varying lengths -> stream-K
+// ranges (no stragglers).  A zero-length sequence is one item with no blocks
+// in ticket mode (so its zero output gets written) and has no blocks in
+// stream-K mode (the merge kernel writes its zero output).  CTA 0 records the
+// choice for the merge kernel.
+struct HandOut {
+  int pb;       // ticket mode: blocks per partition
+  int per_cta;  // stream-K mode: blocks per CTA group
+  bool sk;
+};
+__device__ __forceinline__ HandOut decode_hand_out(const DecodeParams& p, int* prefix, int* lens, int lane) {
+  const int S = p.num_seqs;
+  int pb = p.partition_blocks, per_cta = 0;
+  bool sk = false;
+
+  bool bad = false;
+  long long sum_len = 0;
+  int min_len = 0x7fffffff, max_len = 0;
+  for (int b = 0; b < S; b += 32) {
+    const int s = b + lane;
+    if (s < S) {
+      const int raw = p.seq_lens[s];
+      int len = clamp_len(raw, p);
+      bad |= raw != len;
+      if (p.seq_skip) len = max(0, len - p.seq_skip[s] * kBS);  // the private suffix
+      lens[s] = len;
+      sum_len += len;
+      min_len = min(min_len, len);
+      max_len = max(max_len, len);
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    sum_len += __shfl_xor_sync(0xffffffffu, sum_len, off);
+    min_len = min(min_len, __shfl_xor_sync(0xffffffffu, min_len, off));
+    max_len = max(max_len, __shfl_xor_sync(0xffffffffu, max_len, off));
+  }
+  if (p.auto_mode) {
+    const bool uniform = (long long)min_len * 10 >= (long long)max_len * 9;
+    sk = !uniform && (int)gridDim.x >= p.kv_units;
+    if (!sk) pb = uniform_partition_blocks(p, sum_len, max_len, gridDim.x);
+  }
+  __syncwarp();
+  int carry = 0;
+  for (int b = 0; b < S; b += 32) {
+    const int s = b + lane;
+    int n = 0;
+    if (s < S) {
+      const int len = lens[s];
+      const int nblk = (len + kBS - 1) / kBS;
+      if (sk) {
+        n = nblk;
+      } else {
+        bad |= (nblk + pb - 1) / pb > p.max_parts;
+        n = max(1, num_partitions(len, pb, p)) * p.kv_units;
+      }
+    }
+    int x = n;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, x, off);
+      if (lane >= off) x += y;
+    }
+    if (s < S) prefix[s + 1] = carry + x;
+    carry += __shfl_sync(0xffffffffu, x, 31);
+  }
+  if (lane == 0) prefix[0] = 0;
+  if (blockIdx.x == 0 && __any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, kCheckSeqTooLong);
+  if (sk) {
+    const int groups = max(1, (int)gridDim.x / p.kv_units);
+    per_cta = max(p.min_piece_blocks, (carry + groups - 1) / groups);  // blocks per CTA group
+  }
+  if (blockIdx.x == 0) {  // what this launch used, for the merge kernel
+    __syncwarp();
+    if (sk)
+      for (int i = lane; i <= S; i += 32) p.seq_prefix[i] = prefix[i];
+    if (lane == 0) {
+      p.counters[2] = sk ? per_cta : pb;
+      p.counters[3] = sk ? 1 : 0;
+    }
+  }
+  return {pb, per_cta, sk};
+}
+
+// A work item: sequence, partition (piece) index and count, KV unit, block range.
+struct Item {
+  int s, y, part, np, len, b0, nb, off;  // off: table entries before the suffix
+};
+
+// Items of a launch's hand-out (decode_hand_out), as the producer warp of a
+// CTA enumerates them.
+struct WorkItems {
+  const DecodeParams& p;
+  const int* prefix;  // [S + 1] (shared memory)
+  const int* lens;    // [S]
+  int pb, per_cta, sk_group;
+
+  __device__ int last_seq_at(int v) const {  // last s with prefix[s] <= v (skips empty sequences)
+    int lo = 0, hi = p.num_seqs - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (prefix[mid] <= v) lo = mid; else hi = mid - 1;
+    }
+    return lo;
+  }
+  // ticket mode: item t of the (sequence, partition, KV unit) enumeration
+  __device__ Item ticket(int t) const {
+    Item it;
+    it.s = last_seq_at(t);
+    const int r = t - prefix[it.s];
+    it.part = r / p.kv_units;
+    it.y = r - it.part * p.kv_units;
+    it.len = lens[it.s];
+    it.np = max(1, num_partitions(it.len, pb, p));
+    const int nblk = (it.len + kBS - 1) / kBS;
+    it.b0 = it.part * pb;
+    it.nb = max(0, min(nblk, it.b0 + pb) - it.b0);
+    it.off = p.seq_skip ? __ldg(p.seq_skip + it.s) : 0;
+    return it;
+  }
+  // stream-K mode: this CTA's KV unit of the sequence under global block g, up to `end`
+  __device__ Item streamk(int g, int end) const {
+    Item it;
+    it.s = last_seq_at(g);
+    it.len = lens[it.s];
+    const int nblk = (it.len + kBS - 1) / kBS;
+    it.y = (int)blockIdx.x - sk_group * p.kv_units;
+    it.b0 = g - prefix[it.s];
+    it.nb = min(nblk - it.b0, end - g);
+    const Pieces pc = unit_pieces(prefix[it.s], nblk, per_cta);
+    it.part = sk_group - pc.c0;
+    it.np = pc.count;
+    it.off = p.seq_skip ? __ldg(p.seq_skip + it.s) : 0;
+    return it;
+  }
+  // Lane j's block-table entry of chunk c (blocks 32c + j) of an item; out-of-pool ids are flagged.
+  __device__ int table_chunk(const Item& it, int c, int lane) const {
+    const int i = 32 * c + lane;
+    int b = 0;
+    if (i < it.nb) {
+      b = __ldg(p.block_tables + (size_t)it.s * p.bt_stride + it.off + it.b0 + i);
+      if (b < 0 || b >= p.num_blocks) {
+        atomicOr(p.err, kCheckBadBlock);
+        b = 0;
+      }
+    }
+    return b;
+  }
+};
+
 template <class C>
 __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                           const __grid_constant__ CUtensorMap tmV,
@@ -521,84 +676,13 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
   int* lens = prefix + (S + 1);                             // [S], clamped
 
 
-  // Clamped lengths and their statistics; in auto mode the work hand-out is
-  // chosen from them: near-uniform lengths (all within 10 %) -> tickets with
-  // large partitions (items finish together; the memory system stays
-  // saturated), varying lengths -> stream-K ranges (no stragglers).  Then an
-  // exclusive prefix over the sequences of
-  //  ticket mode:    items (partitions x KV units; a zero-length sequence is
-  //                  one item with no blocks, so its zero output gets written)
-  //  stream-K mode:  blocks (a zero-length sequence has none; the merge
-  //                  kernel writes its zero output)
   int pb = p.partition_blocks, per_cta = 0;
   bool sk = false;
   if (warp == 1) {
-    bool bad = false;
-    long long sum_len = 0;
-    int min_len = 0x7fffffff, max_len = 0;
-    for (int b = 0; b < S; b += 32) {
-      const int s = b + lane;
-      if (s < S) {
-        const int raw = p.seq_lens[s];
-        int len = clamp_len(raw, p);
-        bad |= raw != len;
-        if (p.seq_skip) len = max(0, len - p.seq_skip[s] * kBS);  // the private suffix
-        lens[s] = len;
-        sum_len += len;
-        min_len = min(min_len, len);
-        max_len = max(max_len, len);
-      }
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      sum_len += __shfl_xor_sync(0xffffffffu, sum_len, off);
-      min_len = min(min_len, __shfl_xor_sync(0xffffffffu, min_len, off));
-      max_len = max(max_len, __shfl_xor_sync(0xffffffffu, max_len, off));
-    }
-    if (p.auto_mode) {
-      const bool uniform = (long long)min_len * 10 >= (long long)max_len * 9;
-      sk = !uniform && (int)gridDim.x >= p.kv_units;
-      if (!sk) pb = uniform_partition_blocks(p, sum_len, max_len, gridDim.x);
-    }
-    __syncwarp();
-    int carry = 0;
-    for (int b = 0; b < S; b += 32) {
-      const int s = b + lane;
-      int n = 0;
-      if (s < S) {
-        const int len = lens[s];
-        const int nblk = (len + kBS - 1) / kBS;
-        if (sk) {
-          n = nblk;
-        } else {
-          bad |= (nblk + pb - 1) / pb > p.max_parts;
-          n = max(1, num_partitions(len, pb, p)) * p.kv_units;
-        }
-      }
-      int x = n;
-#pragma unroll
-      for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, x, off);
-        if (lane >= off) x += y;
-      }
-      if (s < S) prefix[s + 1] = carry + x;
-      carry += __shfl_sync(0xffffffffu, x, 31);
-    }
-    if (lane == 0) prefix[0] = 0;
-    if (blockIdx.x == 0 && __any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, kCheckSeqTooLong);
-    if (sk) {
-      const int groups = max(1, (int)gridDim.x / p.kv_units);
-      per_cta = max(p.min_piece_blocks, (carry + groups - 1) / groups);  // blocks per CTA group
-    }
-    if (blockIdx.x == 0) {  // what this launch used, for the merge kernel
-      __syncwarp();
-      if (sk)
-        for (int i = lane; i <= S; i += 32) p.seq_prefix[i] = prefix[i];
-      if (lane == 0) {
-        p.counters[2] = sk ? per_cta : pb;
-        p.counters[3] = sk ? 1 : 0;
-      }
-    }
+    const HandOut h = decode_hand_out(p, prefix, lens, lane);
+    pb = h.pb;
+    per_cta = h.per_cta;
+    sk = h.sk;
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < kDecodeBarriers(NS); ++i) mbar_init(full0 + 8 * i, 1);
@@ -629,62 +713,11 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
       }
       return true;
     };
-    // A work item: sequence, partition (piece) index and count, KV unit, block range.
-    struct Item {
-      int s, y, part, np, len, b0, nb, off;  // off: table entries before the suffix
-    };
-    auto last_seq_at = [&](int v) {  // last s with prefix[s] <= v (skips empty sequences)
-      int lo = 0, hi = S - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (prefix[mid] <= v) lo = mid; else hi = mid - 1;
-      }
-      return lo;
-    };
-    // ticket mode: item t of the (sequence, partition, KV unit) enumeration
-    auto decode = [&](int t) -> Item {
-      Item it;
-      it.s = last_seq_at(t);
-      const int r = t - prefix[it.s];
-      it.part = r / p.kv_units;
-      it.y = r - it.part * p.kv_units;
-      it.len = lens[it.s];
-      it.np = max(1, num_partitions(it.len, pb, p));
-      const int nblk = (it.len + kBS - 1) / kBS;
-      it.b0 = it.part * pb;
-      it.nb = max(0, min(nblk, it.b0 + pb) - it.b0);
-      it.off = p.seq_skip ? __ldg(p.seq_skip + it.s) : 0;
-      return it;
-    };
-    // stream-K mode: this CTA's KV unit of the sequence under global block g, up to `end`
-    const int sk_group = (int)blockIdx.x / p.kv_units;
-    auto decode_sk = [&](int g, int end) -> Item {
-      Item it;
-      it.s = last_seq_at(g);
-      it.len = lens[it.s];
-      const int nblk = (it.len + kBS - 1) / kBS;
-      it.y = (int)blockIdx.x - sk_group * p.kv_units;
-      it.b0 = g - prefix[it.s];
-      it.nb = min(nblk - it.b0, end - g);
-      const Pieces pc = unit_pieces(prefix[it.s], nblk, per_cta);
-      it.part = sk_group - pc.c0;
-      it.np = pc.count;
-      it.off = p.seq_skip ? __ldg(p.seq_skip + it.s) : 0;
-      return it;
-    };
-    // Lane j's block-table entry of chunk c (blocks 32c + j) of an item; out-of-pool ids are flagged.
-    auto load_chunk = [&](const Item& it, int c) -> int {
-      const int i = 32 * c + lane;
-      int b = 0;
-      if (i < it.nb) {
-        b = __ldg(p.block_tables + (size_t)it.s * p.bt_stride + it.off + it.b0 + i);
-        if (b < 0 || b >= p.num_blocks) {
-          atomicOr(p.err, kCheckBadBlock);
-          b = 0;
-        }
-      }
-      return b;
-    };
+    const WorkItems items{p, prefix, lens, pb, per_cta, (int)blockIdx.x / p.kv_units};
+    const int sk_group = items.sk_group;
+    auto decode = [&](int t) { return items.ticket(t); };
+    auto decode_sk = [&](int g, int end) { return items.streamk(g, end); };
+    auto load_chunk = [&](const Item& it, int c) { return items.table_chunk(it, c, lane); };
     // Work cursor: a ticket (ticket mode) or a global block index (stream-K
     // mode, over this CTA's range [blockIdx.x * per_cta, g_end)).
     // Software pipeline: the next item's ticket is claimed four blocks before
