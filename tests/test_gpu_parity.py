@@ -216,6 +216,37 @@ def test_split_matches_unsplit_and_len1_exact():
         assert torch.equal(o_512[0, h], v0[h // G]), h
 
 
+@pytest.mark.parametrize("q_dtype,kv_dtype", [("bf16", "bf16"), ("f16", "fp8_e4m3")])
+def test_mixed_split_counts_in_one_call(q_dtype, kv_dtype):
+    """One call whose sequences are split into 1, 2, 3, 6, 7 and 16 partitions
+    of 512 tokens, repeated three times: every element against the oracle, and
+    the calls bit-identical (the launch counters are left at zero)."""
+    base = wl.SPEC_BY_NAME["long-context-split-kv"]
+    spec = wl.scaled(base, num_seqs=6, q_dtype=q_dtype, kv_dtype=kv_dtype, pool_blocks=None)
+    # at 512-token partitions: 2, 6, 7, 16, 1 and 3 partitions
+    lens = [1000, 3072, 3073, 8192, 300, 1100]
+    w = wl.make_workload(spec, DEV, seq_lens=lens)
+    pa = _ctx(spec, w.num_blocks, w.block_tables.shape[1], partition=512)
+    if kv_dtype == "fp8_e4m3":
+        kh, vh = _oracle_fp8_pool(w)
+        kc = torch.from_numpy(kh).to(DEV).view(torch.float8_e4m3fn)
+        vc = torch.from_numpy(vh).to(DEV).view(torch.float8_e4m3fn)
+    else:
+        kh, vh = raw(w.key_cache), raw(w.value_cache)
+        kc, vc = w.key_cache, w.value_cache
+    ref = attention.decode_attention(raw(w.query), kh, vh, raw(w.block_tables), raw(w.seq_lens), w.scale,
+                                     q_dtype=q_dtype, kv_dtype=kv_dtype, k_scale=w.k_scale, v_scale=w.v_scale)
+    outs = []
+    for _ in range(3):
+        outs.append(pa.decode(w.query, kc, vc, w.block_tables, w.seq_lens, w.max_seq_len, w.scale, w.k_scale,
+                              w.v_scale))
+        assert pa.get_error() == 0
+    tol = TOL[kv_dtype] if kv_dtype == "fp8_e4m3" else TOL[q_dtype]
+    assert_out_close(outs[0], ref, tol, q_dtype, "mixed splits")
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2])
+    pa.close()
+
+
 def test_garbage_in_unused_slots_and_blocks_is_ignored():
     spec = wl.scaled(wl.SPEC_BY_NAME["gqa-70b-like"], num_seqs=6, seq_len_min=17, seq_len_max=700)
     w = wl.make_workload(spec, DEV)
