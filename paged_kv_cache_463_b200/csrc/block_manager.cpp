@@ -9,10 +9,22 @@
 #include <unordered_map>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "block_manager.h"
 #include "paged_attn.h"
 
 #define PA_API extern "C" __attribute__((visibility("default")))
+
+// An NVTX range around each block-manager call that changes its state or
+// exports tables (no-ops unless a profiling tool is attached).
+struct BmTraceRange {
+  explicit BmTraceRange(const char* name) { nvtxRangePushA(name); }
+  ~BmTraceRange() { nvtxRangePop(); }
+  BmTraceRange(const BmTraceRange&) = delete;
+  BmTraceRange& operator=(const BmTraceRange&) = delete;
+};
+#define BM_TRACE(name) const BmTraceRange bm_trace_range_(name)
 
 namespace {
 
@@ -105,6 +117,7 @@ struct pa_block_manager {
   std::lock_guard<std::mutex> lock_((bm)->mu)
 
 PA_API int pa_bm_create(int num_blocks, int block_size, pa_block_manager** out) {
+  BM_TRACE("pa_bm_create");
   if (!out) return PA_ERR_INVALID_ARG;
   *out = nullptr;
   if (num_blocks <= 0 || block_size <= 0) return PA_ERR_INVALID_ARG;
@@ -125,6 +138,7 @@ PA_API int pa_bm_create(int num_blocks, int block_size, pa_block_manager** out) 
 }
 
 PA_API int pa_bm_destroy(pa_block_manager* bm) {
+  BM_TRACE("pa_bm_destroy");
   if (!bm) return PA_ERR_INVALID_ARG;
   delete bm;
   return PA_OK;
@@ -152,6 +166,7 @@ PA_API int pa_bm_cached_blocks(pa_block_manager* bm, int* out) {
 }
 
 PA_API int pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id) {
+  BM_TRACE("pa_bm_add_sequence");
   BM_GUARD(bm);
   if (bm->seqs.count(seq_id)) return PA_ERR_INVALID_ARG;
   try {
@@ -164,6 +179,7 @@ PA_API int pa_bm_add_sequence(pa_block_manager* bm, int64_t seq_id) {
 }
 
 PA_API int pa_bm_free_sequence(pa_block_manager* bm, int64_t seq_id) {
+  BM_TRACE("pa_bm_free_sequence");
   BM_GUARD(bm);
   Seq* s = bm->use(seq_id);
   if (!s) return PA_ERR_INVALID_ARG;
@@ -173,6 +189,7 @@ PA_API int pa_bm_free_sequence(pa_block_manager* bm, int64_t seq_id) {
 }
 
 PA_API int pa_bm_ensure_capacity(pa_block_manager* bm, int64_t seq_id, int64_t required_tokens) {
+  BM_TRACE("pa_bm_ensure_capacity");
   BM_GUARD(bm);
   if (required_tokens < 0) return PA_ERR_INVALID_ARG;
   Seq* s = bm->use(seq_id);
@@ -190,6 +207,7 @@ PA_API int pa_bm_ensure_capacity(pa_block_manager* bm, int64_t seq_id, int64_t r
 
 PA_API int pa_bm_append_tokens(pa_block_manager* bm, int64_t seq_id, int num_tokens, int64_t* slots,
                                int64_t* copy_pairs, int* num_copies, int* num_appended) {
+  BM_TRACE("pa_bm_append_tokens");
   BM_GUARD(bm);
   if (num_tokens < 0 || (num_tokens > 0 && (!slots || !copy_pairs)) || !num_copies || !num_appended)
     return PA_ERR_INVALID_ARG;
@@ -229,6 +247,7 @@ PA_API int pa_bm_append_tokens(pa_block_manager* bm, int64_t seq_id, int num_tok
 
 PA_API int pa_bm_append_batch(pa_block_manager* bm, const int64_t* seq_ids, int n, int64_t* slots, int64_t* copy_pairs,
                               int* num_copies, int* num_appended) {
+  BM_TRACE("pa_bm_append_batch");
   BM_GUARD(bm);
   if (n < 0 || (n > 0 && (!seq_ids || !slots || !copy_pairs)) || !num_copies || !num_appended)
     return PA_ERR_INVALID_ARG;
@@ -267,6 +286,7 @@ PA_API int pa_bm_append_batch(pa_block_manager* bm, const int64_t* seq_ids, int 
 }
 
 PA_API int pa_bm_fork(pa_block_manager* bm, int64_t parent_id, int64_t child_id) {
+  BM_TRACE("pa_bm_fork");
   BM_GUARD(bm);
   Seq* p = bm->use(parent_id);
   if (!p || bm->seqs.count(child_id)) return PA_ERR_INVALID_ARG;
@@ -305,6 +325,7 @@ PA_API int pa_bm_block_table(pa_block_manager* bm, int64_t seq_id, int32_t* out,
 
 PA_API int pa_bm_build_batch(pa_block_manager* bm, const int64_t* seq_ids, int n, int32_t* block_tables, int bt_stride,
                              int32_t* seq_lens) {
+  BM_TRACE("pa_bm_build_batch");
   BM_GUARD(bm);
   if (n < 0 || bt_stride < 1 || (n > 0 && (!seq_ids || !block_tables || !seq_lens))) return PA_ERR_INVALID_ARG;
   for (int i = 0; i < n; ++i) {
@@ -319,6 +340,7 @@ PA_API int pa_bm_build_batch(pa_block_manager* bm, const int64_t* seq_ids, int n
 }
 
 PA_API int pa_bm_evict_lru_sequence(pa_block_manager* bm, int64_t exclude_id, int has_exclude, int64_t* victim) {
+  BM_TRACE("pa_bm_evict_lru_sequence");
   BM_GUARD(bm);
   if (!victim) return PA_ERR_INVALID_ARG;
   bool found = false;
@@ -341,6 +363,7 @@ PA_API int pa_bm_evict_lru_sequence(pa_block_manager* bm, int64_t exclude_id, in
 
 PA_API int pa_bm_allocate_with_prefix(pa_block_manager* bm, int64_t seq_id, const int32_t* tokens, int num_tokens,
                                       int* matched_tokens, int64_t* slots, int* num_slots) {
+  BM_TRACE("pa_bm_allocate_with_prefix");
   BM_GUARD(bm);
   if (num_tokens < 0 || (num_tokens > 0 && (!tokens || !slots)) || !matched_tokens || !num_slots)
     return PA_ERR_INVALID_ARG;

@@ -12,6 +12,8 @@
 #include <string>
 #include <unordered_map>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "paged_attn.h"
 #include "cache_ops.cuh"
 #include "decode.cuh"
@@ -19,6 +21,18 @@
 #include "prefix.cuh"
 
 #define PA_API extern "C" __attribute__((visibility("default")))
+
+// An NVTX range around each C-ABI call that touches the GPU, named after the
+// call (seen by Nsight Systems and by ncu --nvtx; without a tool attached the
+// push and pop do nothing).  The allocation-free entry point has none: it
+// leaves every host-side resource alone too.
+struct PaTraceRange {
+  explicit PaTraceRange(const char* name) { nvtxRangePushA(name); }
+  ~PaTraceRange() { nvtxRangePop(); }
+  PaTraceRange(const PaTraceRange&) = delete;
+  PaTraceRange& operator=(const PaTraceRange&) = delete;
+};
+#define PA_TRACE(name) const PaTraceRange pa_trace_range_(name)
 
 namespace {
 
@@ -305,6 +319,7 @@ PA_API const char* paged_attn_last_error(const pa_ctx* ctx) { return ctx ? ctx->
 PA_API int paged_attn_last_check_bits(const pa_ctx* ctx) { return ctx ? ctx->last_bits : 0; }
 
 PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
+  PA_TRACE("paged_attn_create");
   if (!out) return PA_ERR_INVALID_ARG;
   *out = nullptr;
   if (!cfg) return PA_ERR_INVALID_ARG;
@@ -415,6 +430,7 @@ PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
 }
 
 PA_API int paged_attn_destroy(pa_ctx* ctx) {
+  PA_TRACE("paged_attn_destroy");
   if (!ctx) return PA_ERR_INVALID_ARG;
   cudaSetDevice(ctx->device);
   if (ctx->part_o) cudaFree(ctx->part_o);
@@ -451,6 +467,7 @@ PA_API int reshape_and_cache(pa_ctx* ctx, const void* key, const void* value, in
                              int64_t value_token_stride, void* key_cache, void* value_cache,
                              const int64_t* slot_mapping, int num_tokens, float k_scale, float v_scale,
                              void* stream) {
+  PA_TRACE("reshape_and_cache");
   if (!ctx) return PA_ERR_INVALID_ARG;
   const pa_config& c = ctx->cfg;
   if (num_tokens < 0) return fail(ctx, PA_ERR_INVALID_ARG, "num_tokens < 0");
@@ -666,6 +683,7 @@ PA_API int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, con
                                   const void* value_cache, const int32_t* block_tables, int bt_stride,
                                   const int32_t* seq_lens, int num_seqs, int max_seq_len, float scale,
                                   float k_scale, float v_scale, void* stream) {
+  PA_TRACE("paged_attention_decode");
   return decode_impl(ctx, out, query, key_cache, value_cache, block_tables, bt_stride, seq_lens, num_seqs,
                      max_seq_len, scale, k_scale, v_scale, stream, nullptr);
 }
@@ -677,6 +695,7 @@ PA_API int paged_attention_decode_shared_prefix(pa_ctx* ctx, void* out, const vo
                                                 const int32_t* group_prefix_len, int num_groups,
                                                 int max_group_size, int max_prefix_len, float scale,
                                                 float k_scale, float v_scale, void* stream) {
+  PA_TRACE("paged_attention_decode_shared_prefix");
   const PrefixArgs pre = {group_start, group_prefix_len, num_groups, max_group_size, max_prefix_len};
   return decode_impl(ctx, out, query, key_cache, value_cache, block_tables, bt_stride, seq_lens, num_seqs,
                      max_seq_len, scale, k_scale, v_scale, stream, &pre);
@@ -687,6 +706,7 @@ PA_API int paged_attention_prefill(pa_ctx* ctx, void* out, const void* query, co
                                    const int32_t* seq_lens, const int32_t* query_start, int num_seqs, int num_tokens,
                                    int max_query_len, int max_seq_len, float scale, float k_scale, float v_scale,
                                    void* stream) {
+  PA_TRACE("paged_attention_prefill");
   if (!ctx) return PA_ERR_INVALID_ARG;
   const pa_config& c = ctx->cfg;
   if (num_seqs < 0 || num_seqs > 65535) return fail(ctx, PA_ERR_INVALID_ARG, "num_seqs outside [0, 65535]");
@@ -738,6 +758,7 @@ PA_API int paged_attention_prefill(pa_ctx* ctx, void* out, const void* query, co
 }
 
 PA_API int paged_attn_get_error(pa_ctx* ctx, void* stream) {
+  PA_TRACE("paged_attn_get_error");
   if (!ctx) return PA_ERR_INVALID_ARG;
   cudaSetDevice(ctx->device);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -765,6 +786,7 @@ PA_API int paged_attn_test_wait_timeout(pa_ctx* ctx, long long wait_limit_cycles
 
 PA_API int paged_gather_kv(pa_ctx* ctx, void* k_out, void* v_out, const void* key_cache, const void* value_cache,
                            const int32_t* block_table_row, int seq_len, void* stream) {
+  PA_TRACE("paged_gather_kv");
   if (!ctx) return PA_ERR_INVALID_ARG;
   const pa_config& c = ctx->cfg;
   if (seq_len < 0 || seq_len > c.max_blocks_per_seq * c.block_size)
@@ -977,6 +999,7 @@ PA_API int paged_attention_decode_noalloc(void* out, const void* query, const vo
 PA_API int paged_copy_blocks(pa_ctx* ctx, void* dst_key_cache, void* dst_value_cache, int64_t dst_num_blocks,
                              const void* src_key_cache, const void* src_value_cache, int64_t src_num_blocks,
                              const int64_t* block_pairs, int num_pairs, void* stream) {
+  PA_TRACE("paged_copy_blocks");
   if (!ctx) return PA_ERR_INVALID_ARG;
   const pa_config& c = ctx->cfg;
   if (num_pairs < 0) return fail(ctx, PA_ERR_INVALID_ARG, "num_pairs < 0");
