@@ -159,8 +159,12 @@ int reshape_and_cache(pa_ctx* ctx, const void* key, const void* value, int64_t k
  * truncated and flagged (PA_CHECK_SEQ_TOO_LONG).
  * bt_stride: row stride of block_tables in entries (>= 1).
  * Pointers: out/query 16-byte aligned, caches 16-byte aligned.
- * Launches one partition kernel, plus one merge kernel when a sequence spans
- * several partitions.
+ * Launches the decode kernel and then, as a programmatic dependent launch
+ * on the same stream, the merge kernel whenever the call may split a
+ * sequence: always with PA_PARTITION_AUTO (the split is chosen on the device,
+ * and the merge kernel's CTAs for unsplit sequences exit at once), and with a
+ * fixed partition shorter than max_seq_len.  PA_PARTITION_NONE, or a fixed
+ * partition of at least max_seq_len tokens, launches the decode kernel alone.
  */
 int paged_attention_decode(pa_ctx* ctx, void* out, const void* query, const void* key_cache,
                            const void* value_cache, const int32_t* block_tables, int bt_stride,
