@@ -336,8 +336,9 @@ int paged_copy_blocks(pa_ctx* ctx, void* dst_key_cache, void* dst_value_cache, i
  * on that GPU until the process exits.  The caller passes inputs and outputs.
  *
  * partition_tokens: 0 = one partition per sequence (needs no partials), else a
- * multiple of 16.  A split whose partials (num_seqs * num_heads * partitions *
- * (head_dim + 2) floats, plus 256 bytes) do not fit the array is refused with
+ * multiple of 16.  A call whose partials (num_seqs * num_heads * partitions *
+ * (head_dim + 2) floats, with no split none), plus num_seqs ints rounded up
+ * to 256 bytes and a 256-byte header, do not fit the array is refused with
  * PA_ERR_SCRATCH_TOO_SMALL before anything is launched.
  * check_bits: optional device int that receives PA_CHECK_* bits (or-ed in;
  * the caller clears it); NULL sends them to a word inside the array.

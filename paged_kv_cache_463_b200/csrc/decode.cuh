@@ -64,9 +64,7 @@ struct DecodeParams {
   float* part_o;                // [S, Hq, max_parts, D]
   float* part_ml;               // [S, Hq, max_parts, 2]  (m in log2 units, l)
   int* err;                     // device check bits
-  int* counters;                // [0] ticket, [1] finished CTAs (zero between launches),
-                                // [2] partition blocks or stream-K blocks per group, [3] 1 if stream-K
-                                // (both: what the last launch used, for the merge kernel)
+  int* counters;                // [0] ticket, [1] finished CTAs (zero between launches)
   int num_seqs;
   int bt_stride;
   int num_heads;
@@ -79,7 +77,7 @@ struct DecodeParams {
   int partition_blocks;  // ticket mode: blocks per partition
   int auto_mode;         // 1: the kernel chooses tickets or stream-K (and the partition) from the lengths
   int min_piece_blocks;  // stream-K mode: shortest range a CTA group is given
-  int* seq_prefix;       // stream-K mode: [S + 1] block offsets of the sequences, for the merge
+  int* seq_merge;        // [S]: each sequence's merge work, written by CTA 0 for the merge kernel
   int max_parts;    // partitions a sequence may have (workspace extent)
   int q_slot_bytes; // min(group, 8) * head_dim * 2: one item's query rows
   int merge_hpc;    // merge kernel: query heads per CTA
@@ -101,6 +99,10 @@ struct DecodeParams {
 };
 
 constexpr int kPrefixChunkBlocks = 32;  // blocks per partial of the prefix pass
+// DecodeParams::seq_merge values: >= 0 = the decode partials to fold (plus
+// the prefix pass's chunks in shared-prefix decode); or
+constexpr int kMergeNone = -2;  // the decode kernel wrote the row (one unsplit item)
+constexpr int kMergeZero = -1;  // no decode item covered the sequence: zero rows
 
 // Clamp a sequence length to what its table row can address and to the
 // call's max_seq_len bound (which sizes the partial workspace).
@@ -574,13 +576,15 @@ __device__ __forceinline__ HandOut decode_hand_out(const DecodeParams& p, int* p
     const int groups = max(1, (int)gridDim.x / p.kv_units);
     per_cta = max(p.min_piece_blocks, (carry + groups - 1) / groups);  // blocks per CTA group
   }
-  if (blockIdx.x == 0) {  // what this launch used, for the merge kernel
+  if (blockIdx.x == 0) {  // each sequence's merge work under this launch's hand-out
     __syncwarp();
-    if (sk)
-      for (int i = lane; i <= S; i += 32) p.seq_prefix[i] = prefix[i];
-    if (lane == 0) {
-      p.counters[2] = sk ? per_cta : pb;
-      p.counters[3] = sk ? 1 : 0;
+    const bool shared = p.seq_skip != nullptr;
+    for (int s = lane; s < S; s += 32) {
+      const int len = lens[s];
+      const int nblk = (len + kBS - 1) / kBS;
+      // decode partials: stream-K pieces, or fixed partitions
+      const int np = sk ? (nblk == 0 ? 0 : unit_pieces(prefix[s], nblk, per_cta).count) : num_partitions(len, pb, p);
+      p.seq_merge[s] = (!shared && sk && nblk == 0) ? kMergeZero : (shared || np > 1) ? np : kMergeNone;
     }
   }
   return {pb, per_cta, sk};
@@ -1001,16 +1005,20 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
 // `merge_hpc` consecutive query heads of one sequence; its threads are
 // (head, partition slice, 4-dim chunk) triples, `merge_slices` slices taking
 // every merge_slices-th partial.  Each thread folds its partials into a
-// running (max M, weight sum W, weighted sum) in one pass, 8 partials' loads
-// in flight, and the slices are folded together in shared memory with the
-// same rule; out = weighted sum / W.  A head's partials are the decode pass's
-// np partitions, followed, in shared-prefix decode, by the prefix pass's
-// chunks.  Launched as a programmatic dependent of the decode kernel: it may
-// be scheduled early and waits for the decode grid to finish before reading.
+// running (max M, weight sum W, weighted sum) in one pass, four partials'
+// loads in flight (few registers, so that a whole batch's merge CTAs are
+// resident at once), and the slices are folded together in shared memory
+// with the same rule; out = weighted sum / W.  A head's partials are the
+// decode pass's np partitions, followed, in shared-prefix decode, by the
+// prefix pass's chunks; np comes from the decode kernel (seq_merge), read in
+// one load.  Launched as a programmatic dependent of the decode kernel: it
+// may be scheduled early and waits for the decode grid to finish before
+// reading.
 template <typename Q, int D, bool BF16>
-__global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(256, 4) paged_decode_merge_kernel(const DecodeParams p) {
   asm volatile("griddepcontrol.wait;" ::: "memory");
   constexpr int CH = D / 4;  // float4 chunks per head
+  constexpr int B = 4;       // partials per batch
   __shared__ float4 red[256];
   __shared__ float2 redm[256];
   const int hpc = p.merge_hpc, slices = p.merge_slices;
@@ -1018,28 +1026,19 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
   const int s = blockIdx.x / hblocks;
   const int h0 = (blockIdx.x - s * hblocks) * hpc;
   const bool shared = p.seq_skip != nullptr;
+  const int code = p.seq_merge[s];
   const int skip = shared ? p.seq_skip[s] : 0;
-  const int len = shared ? max(0, clamp_len(p.seq_lens[s], p) - skip * kBS) : clamp_len(p.seq_lens[s], p);
-  const int nblk = (len + kBS - 1) / kBS;
-  const int nc = shared ? (skip + kPrefixChunkBlocks - 1) / kPrefixChunkBlocks : 0;  // prefix partials
-  // the decode launch's hand-out: stream-K or tickets with pb blocks per partition
-  const bool sk = p.auto_mode && p.counters[3] != 0;
-  const int param = p.auto_mode ? p.counters[2] : p.partition_blocks;
-  // decode-pass partitions (the same for every head of a sequence)
-  int np;
-  if (!sk) np = num_partitions(len, param, p);
-  else np = nblk == 0 ? 0 : unit_pieces(p.seq_prefix[s], nblk, param).count;
-  if (!shared && sk && nblk == 0) {  // empty sequence: zero rows (no decode item covered it)
+  if (code == kMergeNone) return;  // written by the decode kernel
+  if (code == kMergeZero) {        // empty sequence: zero rows (no decode item covered it)
     for (int i = threadIdx.x; i < hpc * D; i += blockDim.x) {
       const int h = h0 + i / D;
       if (h < p.num_heads) reinterpret_cast<Q*>(p.out)[((size_t)s * p.num_heads + h) * D + i % D] = Q(0.0f);
     }
     return;
   }
-  // without a prefix pass, a single partition was written by the decode kernel
-  const bool merged = shared || np > 1;
+  const int np = code;
+  const int nc = shared ? (skip + kPrefixChunkBlocks - 1) / kPrefixChunkBlocks : 0;  // prefix partials
   const int nt = np + nc;
-  if (!merged) return;
   // partial q of head h: decode partition q < np, else prefix chunk q - np
   auto ml_of = [&](int h, int q) -> const float* {
     return q < np ? p.part_ml + (((size_t)s * p.num_heads + h) * p.max_parts + q) * 2
@@ -1049,9 +1048,6 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
     return q < np ? p.part_o + (((size_t)s * p.num_heads + h) * p.max_parts + q) * D
                   : p.pre_o + (((size_t)s * p.num_heads + h) * p.max_chunks + (q - np)) * D;
   };
-  // One pass: each thread keeps a running (max, weight sum, weighted sum of
-  // its 4 dims) over its partials, loading 8 partials at a time; slices are
-  // then combined with the same rule.
   const int c = threadIdx.x % CH;
   const int rest = threadIdx.x / CH;
   const int slice = rest % slices, hl = rest / slices;
@@ -1072,18 +1068,18 @@ __global__ void __launch_bounds__(256) paged_decode_merge_kernel(const DecodePar
     M = mn;
   };
   if (active) {
-    for (int q0 = slice; q0 < nt; q0 += 8 * slices) {
-      float2 mlq[8];
-      float4 v[8];
+    for (int q0 = slice; q0 < nt; q0 += B * slices) {
+      float2 mlq[B];
+      float4 v[B];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {
+      for (int u = 0; u < B; ++u) {
         const int q = q0 + u * slices;
         const bool ok = q < nt;
         mlq[u] = ok ? *reinterpret_cast<const float2*>(ml_of(h, q)) : make_float2(-INFINITY, 0.f);
         v[u] = ok ? *reinterpret_cast<const float4*>(o_of(h, q) + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) {  // a partial (o, m, l) is the summary (m, l, l o)
+      for (int u = 0; u < B; ++u) {  // a partial (o, m, l) is the summary (m, l, l o)
         const float l = mlq[u].y;
         combine(mlq[u].x, l, make_float4(l * v[u].x, l * v[u].y, l * v[u].z, l * v[u].w));
       }

@@ -234,8 +234,8 @@ struct pa_ctx {
   int partition_tokens = 0;     // current setting (PA_PARTITION_* or > 0)
   float* part_o = nullptr;
   float* part_ml = nullptr;
-  int* err = nullptr;           // [0] check word, [1..4] decode kernel counters (DecodeParams::counters)
-  int* seq_prefix = nullptr;    // [max_num_seqs + 1] stream-K block offsets (decode -> merge)
+  int* err = nullptr;           // [0] check word, [1..2] decode kernel counters (DecodeParams::counters)
+  int* seq_merge = nullptr;     // [max_num_seqs] each sequence's merge work (decode -> merge)
   // shared-prefix decode (PA_FLAG_SHARED_PREFIX)
   int max_chunks = 0;           // prefix partials per (seq, head)
   float* pre_o = nullptr;
@@ -394,7 +394,7 @@ PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
       break;
     }
     ctx->grid = ctx->num_sms * ctx->ctas_per_sm;
-    if ((e = cudaMalloc(&ctx->seq_prefix, (c.max_num_seqs + 1) * sizeof(int))) != cudaSuccess) {
+    if ((e = cudaMalloc(&ctx->seq_merge, c.max_num_seqs * sizeof(int))) != cudaSuccess) {
       cudaGetLastError();
       st = PA_ERR_NO_MEMORY;
       break;
@@ -436,7 +436,7 @@ PA_API int paged_attn_destroy(pa_ctx* ctx) {
   if (ctx->part_o) cudaFree(ctx->part_o);
   if (ctx->part_ml) cudaFree(ctx->part_ml);
   if (ctx->err) cudaFree(ctx->err);
-  if (ctx->seq_prefix) cudaFree(ctx->seq_prefix);
+  if (ctx->seq_merge) cudaFree(ctx->seq_merge);
   if (ctx->pre_o) cudaFree(ctx->pre_o);
   if (ctx->pre_ml) cudaFree(ctx->pre_ml);
   if (ctx->seq_skip) cudaFree(ctx->seq_skip);
@@ -650,7 +650,7 @@ int decode_impl(pa_ctx* ctx, void* out, const void* query, const void* key_cache
   p.partition_blocks = part_blocks;
   p.auto_mode = is_auto ? 1 : 0;
   p.min_piece_blocks = kMinPieceBlocks;
-  p.seq_prefix = ctx->seq_prefix;
+  p.seq_merge = ctx->seq_merge;
   p.max_parts = ctx->max_parts;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
   p.v_scale = fp8 ? v_scale : 1.0f;
@@ -769,7 +769,7 @@ PA_API int paged_attn_get_error(pa_ctx* ctx, void* stream) {
   ctx->last_bits = *ctx->err_host;
   if (ctx->last_bits & PA_CHECK_WAIT_TIMEOUT) {
     // a launch that gave up may have left its work counters non-zero
-    if ((e = cudaMemsetAsync(ctx->err + 1, 0, 3 * sizeof(int), s)) != cudaSuccess ||
+    if ((e = cudaMemsetAsync(ctx->err + 1, 0, 2 * sizeof(int), s)) != cudaSuccess ||
         (e = cudaStreamSynchronize(s)) != cudaSuccess)
       return cuda_fail(ctx, e, "paged_attn_get_error(counter reset)");
   }
@@ -938,8 +938,9 @@ PA_API int paged_attention_decode_noalloc(void* out, const void* query, const vo
   int parts = (max_blocks + part_blocks - 1) / part_blocks;
   if (parts < 1) parts = 1;
   const size_t rows = (size_t)num_seqs * num_heads * parts;
+  const size_t codes = ((size_t)num_seqs * sizeof(int) + 255) / 256 * 256;  // the merge's per-sequence work
   const size_t ml_bytes = (rows * 2 * sizeof(float) + 255) / 256 * 256;
-  const size_t need = kNoallocHeader + (parts > 1 ? ml_bytes + rows * head_dim * sizeof(float) : 0);
+  const size_t need = kNoallocHeader + codes + (parts > 1 ? ml_bytes + rows * head_dim * sizeof(float) : 0);
   if (need > PA_NOALLOC_SCRATCH_BYTES) return PA_ERR_SCRATCH_TOO_SMALL;
 
   int dev = 0;
@@ -966,8 +967,9 @@ PA_API int paged_attention_decode_noalloc(void* out, const void* query, const vo
   p.query = query;
   p.block_tables = block_tables;
   p.seq_lens = seq_lens;
-  p.part_ml = reinterpret_cast<float*>(scratch + kNoallocHeader);
-  p.part_o = reinterpret_cast<float*>(scratch + kNoallocHeader + ml_bytes);
+  p.seq_merge = reinterpret_cast<int*>(scratch + kNoallocHeader);
+  p.part_ml = reinterpret_cast<float*>(scratch + kNoallocHeader + codes);
+  p.part_o = reinterpret_cast<float*>(scratch + kNoallocHeader + codes + ml_bytes);
   p.err = check_bits ? check_bits : reinterpret_cast<int*>(scratch);
   p.counters = reinterpret_cast<int*>(scratch) + 4;
   p.num_seqs = num_seqs;
@@ -983,7 +985,6 @@ PA_API int paged_attention_decode_noalloc(void* out, const void* query, const vo
   p.partition_blocks = part_blocks;
   p.auto_mode = 0;
   p.min_piece_blocks = kMinPieceBlocks;
-  p.seq_prefix = nullptr;
   p.max_parts = parts;
   p.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
   p.v_scale = fp8 ? v_scale : 1.0f;
