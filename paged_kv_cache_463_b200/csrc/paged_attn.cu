@@ -154,14 +154,24 @@ struct Tuned;
 #ifndef PA_MIN_CTAS_FP8_128
 #define PA_MIN_CTAS_FP8_128 8
 #endif
-// The shared-prefix pass: ring stages (blocks) and blocks per tensor-core step.
+// The tensor-core passes (shared prefixes, prefill): ring stages (blocks)
+// and blocks per step.  16-bit head_dim 64 / 128: 32-key steps, which leave
+// room (tensor and shared memory) for two CTAs per SM, so that two softmax
+// warps share each scheduler; longer steps with one CTA per SM measured
+// slower (the softmax warps, not the tensor core, set the pace).
+#ifndef PA_PF_NS_16B
+#define PA_PF_NS_16B 6
+#endif
+#ifndef PA_PF_SB_16B
+#define PA_PF_SB_16B 2
+#endif
 template <> struct Tuned<64, __half, __half> {
   using C = DecodeCfg<64, __half, __half, PA_NS_16B_64, 8>;
-  using P = pa::PrefixCfg<64, __half, __half, 8, 4>;
+  using P = pa::PrefixCfg<64, __half, __half, PA_PF_NS_16B, PA_PF_SB_16B>;
 };
 template <> struct Tuned<128, __half, __half> {
   using C = DecodeCfg<128, __half, __half, PA_NS_16B_128, 8>;
-  using P = pa::PrefixCfg<128, __half, __half, 6, 2>;
+  using P = pa::PrefixCfg<128, __half, __half, PA_PF_NS_16B, PA_PF_SB_16B>;
 };
 template <> struct Tuned<256, __half, __half> {
   using C = DecodeCfg<256, __half, __half, PA_NS_16B_256, 3>;
@@ -169,11 +179,11 @@ template <> struct Tuned<256, __half, __half> {
 };
 template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<64, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_64, 8>;
-  using P = pa::PrefixCfg<64, __nv_bfloat16, __nv_bfloat16, 8, 4>;
+  using P = pa::PrefixCfg<64, __nv_bfloat16, __nv_bfloat16, PA_PF_NS_16B, PA_PF_SB_16B>;
 };
 template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128, 8>;
-  using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, 6, 2>;
+  using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, PA_PF_NS_16B, PA_PF_SB_16B>;
 };
 template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_256, 3>;

@@ -26,14 +26,15 @@
 //               f16 once, into per-step operand buffers;
 //   warp 9      polls the barriers and issues S for a step once its operands
 //               are ready (into one of two TMEM S buffers) and O += P V once
-//               the softmax has written that step's P; for 16-bit caches the
-//               ring stages are released by tcgen05.commit after the step's
-//               P V;
+//               the softmax has written that step's P, with P read from
+//               tensor memory as the A operand; for 16-bit caches the ring
+//               stages are released by tcgen05.commit after the step's P V;
 //   warps 0..3  one query row per thread: read the step's S row from TMEM,
 //               online softmax in the log2 domain (lazy: O is rescaled in
 //               TMEM only when a row's maximum grows by more than 2^8), write
-//               P (16-bit) to shared memory; at the end read O, normalise,
-//               hand the row to the caller's store.
+//               P (16-bit pairs) back over the first T/2 columns of the same
+//               S buffer; at the end read O, normalise, hand the row to the
+//               caller's store.
 #pragma once
 
 #include "decode.cuh"
@@ -96,30 +97,32 @@ struct PrefixCfg {
   static constexpr int RING_SUB = NS * kBS * 128;      // bytes between a ring's sub-tiles
   static constexpr int Q_BYTES = kPrefixRows * D * 2;  // 128-byte swizzled, D/64 sub-tiles of 128 rows
   static constexpr int F_BYTES = kFp8 ? T * D * 2 : 0;  // fp8 only: a step's K or V as f16, D/64 sub-tiles of T rows
-  static constexpr int P_BYTES = kPrefixRows * T * 2;  // no swizzle: (8 rows x 8 tokens) core matrices
-  static constexpr int CM_STRIDE = T * 16;             // bytes between 8-row groups of P
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_RING_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_RING_V = OFF_RING_K + NS * TILE_BYTES;
   static constexpr int OFF_KF = OFF_RING_V + NS * TILE_BYTES;  // [B] (fp8)
   static constexpr int OFF_VF = OFF_KF + B * F_BYTES;          // [B] (fp8)
-  static constexpr int OFF_P = OFF_VF + B * F_BYTES;           // [B]
-  static constexpr int OFF_BAR = OFF_P + B * P_BYTES;
+  static constexpr int OFF_BAR = OFF_VF + B * F_BYTES;
   // full[NS] empty[NS] conv_full[B] s_full[B] p_full[B] pv_done[B] fin
   static constexpr int NBARS = 2 * NS + 4 * B + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem base, dead flag, blocks converted
   static constexpr int TMEM_COLS = D + B * T <= 128 ? 128 : (D + B * T <= 256 ? 256 : 512);
-  static constexpr int O_COL = 0, S_COL = D;  // O: D columns; S buffers: T columns each
+  // O: D columns; S buffers: T columns each, a step's P over the first T/2 of its buffer
+  static constexpr int O_COL = 0, S_COL = D;
   static constexpr int MAX_CTAS = 512 / TMEM_COLS;  // CTAs whose TMEM fits one SM
   static constexpr int LAYOUT_BYTES = 1024 + OFF_MISC + 16;
   // at least this much shared memory, so that no more than MAX_CTAS CTAs are resident
   static constexpr int MIN_BYTES = kSmemPerSM / (MAX_CTAS + 1) + 1024;
   static constexpr int SMEM_BYTES = LAYOUT_BYTES > MIN_BYTES ? LAYOUT_BYTES : MIN_BYTES;
   static constexpr int THREADS = 320;
-  static constexpr int REG_CTAS = 1;  // register budget hint (shared memory allows one CTA per SM)
+  // register budget: as many CTAs per SM as tensor and shared memory allow,
+  // up to two (~100 registers a thread: the softmax keeps a step's T scores)
+  static constexpr int SMEM_CTAS = kSmemPerSM / (SMEM_BYTES + 1024);
+  static constexpr int FIT_CTAS = MAX_CTAS < SMEM_CTAS ? MAX_CTAS : SMEM_CTAS;
+  static constexpr int REG_CTAS = FIT_CTAS < 2 ? FIT_CTAS : 2;
   static_assert(ROW_BYTES % 128 == 0, "rows must be whole 128-byte swizzle spans");
   static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
-  static_assert(T % 16 == 0 && T <= 256, "step tokens");
+  static_assert(T % 32 == 0 && T <= 256, "step tokens (P is stored 16 columns at a time)");
   static_assert(NS % SB == 0, "a step's blocks occupy consecutive ring stages");
   static_assert(!kFp8 || std::is_same<Q, __half>::value, "fp8 caches pair with fp16 queries");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -361,7 +364,7 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
         if (npv < ns_ && mbar_test_wait(pfull0 + 8 * (npv % B), (npv / B) & 1)) {
           tc_fence_after();
           const int cb = npv % B;
-          const uint32_t pa_ = base + C::OFF_P + cb * C::P_BYTES;
+          const uint32_t pt = tmem + C::S_COL + cb * T;  // P: T/2 columns of 16-bit pairs
           // V operand, MN-major (dims contiguous in 128-byte rows, one row per
           // token): the f16 copy (fp8) or the ring stages of the step (16-bit)
           const uint32_t va = C::kFp8 ? base + C::OFF_VF + cb * C::F_BYTES
@@ -369,9 +372,8 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
           constexpr int VSUB = C::kFp8 ? T * 128 : C::RING_SUB;  // bytes between 64-dim sub-tiles
 #pragma unroll
           for (int k = 0; k < T / 16; ++k) {  // O += P V over 16-token slices (one block each)
-            const uint64_t a = umma_desc(pa_ + k * 256, 128, C::CM_STRIDE, kUmmaNoSwizzle);
             const uint64_t b = umma_desc(va + k * (kBS * 128), VSUB, 1024, kUmmaSwizzle128);
-            umma_f16(tmem + C::O_COL, a, b, idO, (npv > 0 || k > 0) ? 1 : 0);
+            umma_f16_ts(tmem + C::O_COL, pt + 8 * k, b, idO, (npv > 0 || k > 0) ? 1 : 0);
           }
           umma_commit(pvdone0 + 8 * cb);
           if constexpr (!C::kFp8) {  // the step's ring stages are free once these MMAs complete
@@ -385,6 +387,8 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
         } else if (clock64() - idle_since > kWaitLimitCycles) {
           atomicOr(err, kCheckWaitTimeout);
           *dead = 1;
+        } else {
+          __nanosleep(32);  // (leave the issue slots to the softmax warp sharing this scheduler)
         }
       }
       // every MMA issued has completed before the CTA releases tensor memory
@@ -414,12 +418,24 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
       tmem_wait_ld();
       const int valid = min(T, lim - u * T);  // keys of this step the row sees
       float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent max chains
+      // Steps before the diagonal, where every row of the warp sees every key
+      // and the scale is positive, take the max of the raw scores and fold
+      // the scale into the exponent's FMA; the others scale and mask first.
+      const bool plain = scale_log2 > 0.f && __all_sync(0xffffffffu, valid >= T);
+      float xs;  // exponent = x * xs - m
+      if (plain) {
 #pragma unroll
-      for (int j = 0; j < T; ++j) {
-        x[j] = j < valid ? x[j] * scale_log2 : -INFINITY;
-        mx[j & 3] = fmaxf(mx[j & 3], x[j]);
+        for (int j = 0; j < T; ++j) mx[j & 3] = fmaxf(mx[j & 3], x[j]);
+        xs = scale_log2;
+      } else {
+#pragma unroll
+        for (int j = 0; j < T; ++j) {
+          x[j] = j < valid ? x[j] * scale_log2 : -INFINITY;
+          mx[j & 3] = fmaxf(mx[j & 3], x[j]);
+        }
+        xs = 1.f;
       }
-      const float bm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3]));
+      const float bm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * xs;
       // lazy rescaling: move the reference max (and rescale l, O) only when
       // this step's max exceeds it by more than 2^8
       const bool grow = bm > m + 8.f;
@@ -441,26 +457,23 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
         l *= al;
       }
       if (grow) m = bm;
-      if (u >= B) {
-        ok = wait(pvdone0 + 8 * cb, ((u - B) / B) & 1);  // P buffer cb free
-        if (!ok) break;
-      }
-      // P row r: token groups of 8 as 16-byte core-matrix rows
-      uint8_t* prow = smem + C::OFF_P + cb * C::P_BYTES + (r >> 3) * C::CM_STRIDE + (r & 7) * 16;
+      // P of row r as 16-bit pairs over the first T/2 columns of this S
+      // buffer (its S values are all in registers by now): the A operand of
+      // the step's P V.  The buffer's next S is issued only after that P V.
       float sm[4] = {0.f, 0.f, 0.f, 0.f};  // four independent sum chains
 #pragma unroll
-      for (int g8 = 0; g8 < T / 8; ++g8) {
-        uint32_t pk[4];
+      for (int c0 = 0; c0 < T / 2; c0 += 16) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float p0 = ex2(x[8 * g8 + 2 * q] - m), p1 = ex2(x[8 * g8 + 2 * q + 1] - m);
-          sm[q] += p0 + p1;
+        for (int q = 0; q < 16; ++q) {
+          const float p0 = ex2(fmaf(x[2 * (c0 + q)], xs, -m)), p1 = ex2(fmaf(x[2 * (c0 + q) + 1], xs, -m));
+          sm[q & 3] += p0 + p1;
           pk[q] = pack2<C::kBf16>(p0, p1);
         }
-        *reinterpret_cast<uint4*>(prow + g8 * 128) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        tmem_st16(trow + C::S_COL + cb * T + c0, pk);
       }
       l += (sm[0] + sm[1]) + (sm[2] + sm[3]);
-      fence_proxy_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(pfull0 + 8 * cb);

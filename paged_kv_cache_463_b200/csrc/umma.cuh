@@ -1,5 +1,6 @@
 // Blackwell (sm_100a) 5th-generation tensor-core helpers: tcgen05.mma with
-// operands in shared memory and the accumulator in tensor memory (TMEM).
+// operands in shared memory (or A in tensor memory) and the accumulator in
+// tensor memory (TMEM).
 //
 // Shared-memory matrix descriptor (64 bits): start address >> 4 in bits
 // [0,14), leading-dimension byte offset >> 4 in [16,30), stride-dimension
@@ -43,6 +44,18 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b
       "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A[tmem] . B[smem]^T, issued by one thread: A (M rows x 16 K
+// elements, 16-bit) is read from tensor memory, row m in lane m, K elements
+// 2c and 2c+1 packed in column c (low half first), 8 columns per instruction.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                            int accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(accumulate)
       : "memory");
 }
 
