@@ -98,7 +98,10 @@ struct DecodeParams {
   int debug_stall = 0;
 };
 
-constexpr int kPrefixChunkBlocks = 32;  // blocks per partial of the prefix pass
+#ifndef PA_PREFIX_CHUNK_BLOCKS
+#define PA_PREFIX_CHUNK_BLOCKS 32
+#endif
+constexpr int kPrefixChunkBlocks = PA_PREFIX_CHUNK_BLOCKS;  // blocks per partial of the prefix pass
 // DecodeParams::seq_merge values: >= 0 = the decode partials to fold (plus
 // the prefix pass's chunks in shared-prefix decode); or
 constexpr int kMergeNone = -2;  // the decode kernel wrote the row (one unsplit item)

@@ -159,6 +159,12 @@ struct Tuned;
 // room (tensor and shared memory) for two CTAs per SM, so that two softmax
 // warps share each scheduler; longer steps with one CTA per SM measured
 // slower (the softmax warps, not the tensor core, set the pace).
+#ifndef PA_PX_NS_FP8
+#define PA_PX_NS_FP8 8
+#endif
+#ifndef PA_PX_SB_FP8
+#define PA_PX_SB_FP8 4
+#endif
 #ifndef PA_PF_NS_16B
 #define PA_PF_NS_16B 6
 #endif
@@ -191,7 +197,7 @@ template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> {
 };
 template <> struct Tuned<128, __nv_fp8_e4m3, __half> {
   using C = DecodeCfg<128, __nv_fp8_e4m3, __half, PA_NS_FP8_128, PA_MIN_CTAS_FP8_128>;
-  using P = pa::PrefixCfg<128, __nv_fp8_e4m3, __half, 8, 4>;
+  using P = pa::PrefixCfg<128, __nv_fp8_e4m3, __half, PA_PX_NS_FP8, PA_PX_SB_FP8>;
 };
 template <> struct Tuned<256, __nv_fp8_e4m3, __half> {
   using C = DecodeCfg<256, __nv_fp8_e4m3, __half, PA_NS_FP8_256, 4>;
