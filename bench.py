@@ -629,6 +629,10 @@ def run_ours(args, world, rank, local):
                 g1, s1, d1, _, e1 = oracle_sample(spec, args.cpu_budget / 2)
             result["cpu_baseline"]["one_core"] = {"value": g1, "unit": "GB/s", "cores": 1, "sample": d1,
                                                   "seq_steps_per_s": s1, "seconds": e1}
+            result["cpu_baseline"]["cores_note"] = (
+                f"cores = the BLAS thread pool the oracle ran with; its per-(sequence, head) matrix-vector "
+                f"products are too small to spread over it, so the pool run is {gbs / g1:.2f}x the one-thread "
+                f"run (effective parallelism about 1)")
         except ImportError:
             pass
     if rank == 0:

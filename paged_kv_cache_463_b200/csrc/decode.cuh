@@ -153,7 +153,8 @@ __device__ __forceinline__ Pieces unit_pieces(int a, int nblk, int per_group) {
 // ring[NS stages] | query slots[2] | mbarriers | exit record | stage metadata | prefix[S+1], lens[S]
 // mbarriers: full[NS], empty[NS], qfull[2], qempty[2], and one that nothing
 // completes (the target of the failure-path test hook).  Exit record: stages
-// and query slots the consumer took, and a flag set by a wait that ran out.
+// and query slots the consumer took, a flag set by a wait that ran out, and
+// the two warps' scheduler slots.
 __host__ __device__ constexpr int kDecodeBarriers(int ns) { return 2 * ns + 5; }
 struct DecodeLayout {
   int ring, q, bar, exitrec, meta, prefix;
@@ -162,7 +163,7 @@ struct DecodeLayout {
     q = ns * stage_bytes;
     bar = q + 2 * q_slot_bytes;
     exitrec = (bar + kDecodeBarriers(ns) * 8 + 15) & ~15;
-    meta = exitrec + 16;
+    meta = exitrec + 32;
     prefix = meta + ns * 16;
   }
   // bytes of dynamic shared memory for up to `max_seqs` sequences (+ alignment slack)
@@ -676,16 +677,34 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
   const uint32_t base_u32 = smem_u32(smem);
   const uint32_t full0 = base_u32 + L.bar, empty0 = full0 + NS * 8, qfull0 = full0 + 2 * NS * 8, qempty0 = qfull0 + 16;
   const uint32_t never = qempty0 + 16;  // no thread ever arrives on it
-  volatile int* exitrec = reinterpret_cast<volatile int*>(smem + L.exitrec);  // [0] stages, [1] q slots, [2] timed out
+  // [0] stages, [1] q slots, [2] timed out, [4] [5] the warps' slots
+  volatile int* exitrec = reinterpret_cast<volatile int*>(smem + L.exitrec);
   const long long wl = p.wait_limit;
   int4* meta = reinterpret_cast<int4*>(smem + L.meta);
   int* prefix = reinterpret_cast<int*>(smem + L.prefix);  // [S + 1]
   int* lens = prefix + (S + 1);                             // [S], clamped
 
+  // Roles by scheduler.  The SM gives each warp a slot, slot w is issued
+  // from by scheduler w % 4, and the two warps of a CTA take adjacent slots:
+  // with warp 0 as the consumer everywhere, all of an SM's consumer warps
+  // (the ones doing the math) end up on two of its four schedulers.  The
+  // consumer is instead the warp whose slot has bit 0 equal to bit 2, which
+  // puts the consumers of four consecutive CTAs on schedulers 0, 2, 1, 3
+  // (warp 0 if the rule does not pick exactly one).  Either choice computes
+  // the same; only the speed depends on it.
+  if (lane == 0) {
+    unsigned int w;
+    asm volatile("mov.u32 %0, %%warpid;" : "=r"(w));
+    exitrec[4 + warp] = (int)w;
+  }
+  __syncthreads();
+  const int slot0 = exitrec[4], slot1 = exitrec[5];
+  const bool pick0 = (slot0 & 1) == ((slot0 >> 2) & 1), pick1 = (slot1 & 1) == ((slot1 >> 2) & 1);
+  const bool producer = warp != ((pick1 && !pick0) ? 1 : 0);
 
   int pb = p.partition_blocks, per_cta = 0;
   bool sk = false;
-  if (warp == 1) {
+  if (producer) {
     const HandOut h = decode_hand_out(p, prefix, lens, lane);
     pb = h.pb;
     per_cta = h.per_cta;
@@ -703,7 +722,7 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
   // consumer did not take are waited for before the CTA exits.
   int armed = 0, q_armed = 0;
 
-  if (warp == 1) {
+  if (producer) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
@@ -987,7 +1006,7 @@ __global__ void __launch_bounds__(64, C::MIN_CTAS) paged_decode_kernel(const __g
   // memory: wait (bounded by the default limit) for every stage and query slot
   // armed but not taken, so that no copy outlives the CTA.  At most NS stages
   // and 2 slots are outstanding, each in its own ring position.
-  if (warp == 1 && lane == 0 && exitrec[2]) {
+  if (producer && lane == 0 && exitrec[2]) {
     for (int k = exitrec[0]; k < armed; ++k) mbar_wait(full0 + 8 * (k % NS), (k / NS) & 1);
     for (int i = exitrec[1]; i < q_armed; ++i) mbar_wait(qfull0 + 8 * (i & 1), (i >> 1) & 1);
   }
