@@ -154,11 +154,12 @@ struct Tuned;
 #ifndef PA_MIN_CTAS_FP8_128
 #define PA_MIN_CTAS_FP8_128 8
 #endif
-// The tensor-core passes (shared prefixes, prefill): ring stages (blocks)
-// and blocks per step.  16-bit head_dim 64 / 128: 32-key steps, which leave
-// room (tensor and shared memory) for two CTAs per SM, so that two softmax
-// warps share each scheduler; longer steps with one CTA per SM measured
-// slower (the softmax warps, not the tensor core, set the pace).
+// The tensor-core passes (shared prefixes, prefill): ring stages (blocks),
+// blocks per step and step buffers.  16-bit head_dim 64 / 128: 32-key steps
+// with four S buffers (the MMAs run up to three steps ahead of the softmax),
+// which still leave room (tensor and shared memory) for two CTAs per SM, so
+// that two softmax warps share each scheduler; longer steps with one CTA per
+// SM measured slower (the softmax warps, not the tensor core, set the pace).
 #ifndef PA_PX_NS_FP8
 #define PA_PX_NS_FP8 8
 #endif
@@ -166,18 +167,21 @@ struct Tuned;
 #define PA_PX_SB_FP8 4
 #endif
 #ifndef PA_PF_NS_16B
-#define PA_PF_NS_16B 6
+#define PA_PF_NS_16B 8
 #endif
 #ifndef PA_PF_SB_16B
 #define PA_PF_SB_16B 2
 #endif
+#ifndef PA_PF_B_16B
+#define PA_PF_B_16B 4
+#endif
 template <> struct Tuned<64, __half, __half> {
   using C = DecodeCfg<64, __half, __half, PA_NS_16B_64, 8>;
-  using P = pa::PrefixCfg<64, __half, __half, PA_PF_NS_16B, PA_PF_SB_16B>;
+  using P = pa::PrefixCfg<64, __half, __half, PA_PF_NS_16B, PA_PF_SB_16B, PA_PF_B_16B>;
 };
 template <> struct Tuned<128, __half, __half> {
   using C = DecodeCfg<128, __half, __half, PA_NS_16B_128, 8>;
-  using P = pa::PrefixCfg<128, __half, __half, PA_PF_NS_16B, PA_PF_SB_16B>;
+  using P = pa::PrefixCfg<128, __half, __half, PA_PF_NS_16B, PA_PF_SB_16B, PA_PF_B_16B>;
 };
 template <> struct Tuned<256, __half, __half> {
   using C = DecodeCfg<256, __half, __half, PA_NS_16B_256, 3>;
@@ -185,11 +189,11 @@ template <> struct Tuned<256, __half, __half> {
 };
 template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<64, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_64, 8>;
-  using P = pa::PrefixCfg<64, __nv_bfloat16, __nv_bfloat16, PA_PF_NS_16B, PA_PF_SB_16B>;
+  using P = pa::PrefixCfg<64, __nv_bfloat16, __nv_bfloat16, PA_PF_NS_16B, PA_PF_SB_16B, PA_PF_B_16B>;
 };
 template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128, 8>;
-  using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, PA_PF_NS_16B, PA_PF_SB_16B>;
+  using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, PA_PF_NS_16B, PA_PF_SB_16B, PA_PF_B_16B>;
 };
 template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_256, 3>;

@@ -75,7 +75,7 @@ constexpr int kPrefixRows = 128;  // query rows per CTA (the MMA M)
 // Shared memory per SM, for capping residency.
 constexpr int kSmemPerSM = 233472;
 
-template <int D_, typename KV_, typename Q_, int NS_, int SB_>
+template <int D_, typename KV_, typename Q_, int NS_, int SB_, int B_ = 2>
 struct PrefixCfg {
   static constexpr int D = D_;
   using KV = KV_;
@@ -83,7 +83,7 @@ struct PrefixCfg {
   static constexpr int NS = NS_;   // ring stages (blocks)
   static constexpr int SB = SB_;   // blocks per step
   static constexpr int T = SB * kBS;  // tokens per step (the S MMA's N, the P V MMA's K)
-  static constexpr int B = 2;      // step buffers (S, P, and the fp8 operands)
+  static constexpr int B = B_;     // step buffers (S and P, and the fp8 operands): how far the MMAs may run ahead
   static constexpr bool kFp8 = sizeof(KV) == 1;
   static constexpr bool kBf16 = std::is_same<Q, __nv_bfloat16>::value;
   static constexpr int ROW_BYTES = D * (int)sizeof(KV);
