@@ -41,6 +41,10 @@ using pa::DecodeParams;
 
 struct KernelSet {
   const void* decode = nullptr;
+  // the same decode kernel with a one-stage-shallower ring (16-bit head_dim
+  // 128), used where it fits more CTAs per SM (choose_decode)
+  const void* decode_shallow = nullptr;
+  int ns_shallow = 0;
   const void* merge = nullptr;
   const void* prefix = nullptr;   // shared-prefix pass
   const void* prefill = nullptr;  // multi-query (prefill) attention, same CTA shape as the prefix pass
@@ -52,10 +56,16 @@ struct KernelSet {
   }
 };
 
-template <class C, class P>
+// CS: the shallower-ring decode configuration, or void.
+template <class C, class P, class CS>
 KernelSet make_set() {
   KernelSet k;
   k.decode = reinterpret_cast<const void*>(&pa::paged_decode_kernel<C>);
+  if constexpr (!std::is_void<CS>::value) {
+    static_assert(CS::STAGE_BYTES == C::STAGE_BYTES && CS::THREADS == C::THREADS, "same ring stages and CTA");
+    k.decode_shallow = reinterpret_cast<const void*>(&pa::paged_decode_kernel<CS>);
+    k.ns_shallow = CS::NS;
+  }
   k.merge = reinterpret_cast<const void*>(&pa::paged_decode_merge_kernel<typename C::Q, C::D, C::kBf16>);
   k.prefix = reinterpret_cast<const void*>(&pa::paged_prefix_kernel<P>);
   k.prefill = reinterpret_cast<const void*>(&pa::paged_prefill_kernel<P>);
@@ -67,6 +77,27 @@ KernelSet make_set() {
   return k;
 }
 
+// Resident decode CTAs per SM for a call shape; with a shallower-ring
+// variant, take it when more of its CTAs fit (bytes in flight per SM: CTAs x
+// stages).  Results do not depend on the ring depth.  Both kernels' shared
+// memory limits must have been raised.
+cudaError_t choose_decode(KernelSet* ks, int q_slot, int max_seqs, int* per_sm) {
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, ks->decode, ks->threads,
+                                                                ks->smem(q_slot, max_seqs));
+  if (e != cudaSuccess || !ks->decode_shallow) return e;
+  KernelSet alt = *ks;
+  alt.decode = ks->decode_shallow;
+  alt.ns = ks->ns_shallow;
+  int n = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, alt.decode, alt.threads, alt.smem(q_slot, max_seqs));
+  if (e != cudaSuccess) return e;
+  if (n > *per_sm) {
+    *ks = alt;
+    *per_sm = n;
+  }
+  return cudaSuccess;
+}
+
 // Every kernel of the library asks for the same (maximum shared-memory)
 // L1/shared split, so consecutive launches (cache write -> decode -> merge)
 // never make the SMs switch configuration between kernels.
@@ -75,7 +106,8 @@ cudaError_t pin_carveout(const void* fn) {
 }
 
 cudaError_t pin_all_carveouts(const KernelSet& ks) {
-  const void* fns[] = {ks.decode, ks.merge, ks.prefix, ks.prefill, reinterpret_cast<const void*>(&pa::reshape_and_cache_copy_kernel),
+  const void* fns[] = {ks.decode, ks.decode_shallow ? ks.decode_shallow : ks.decode, ks.merge, ks.prefix, ks.prefill,
+                       reinterpret_cast<const void*>(&pa::reshape_and_cache_copy_kernel),
                        reinterpret_cast<const void*>(&pa::reshape_and_cache_fp8_kernel<true>),
                        reinterpret_cast<const void*>(&pa::reshape_and_cache_fp8_kernel<false>),
                        reinterpret_cast<const void*>(&pa::paged_gather_kernel),
@@ -177,39 +209,49 @@ struct Tuned;
 #endif
 template <> struct Tuned<64, __half, __half> {
   using C = DecodeCfg<64, __half, __half, PA_NS_16B_64, 8>;
+  using CS = void;
   using P = pa::PrefixCfg<64, __half, __half, PA_PF_NS_16B, PA_PF_SB_16B, PA_PF_B_16B>;
 };
 template <> struct Tuned<128, __half, __half> {
   using C = DecodeCfg<128, __half, __half, PA_NS_16B_128, 8>;
+  using CS = DecodeCfg<128, __half, __half, PA_NS_16B_128 - 1, 8>;
   using P = pa::PrefixCfg<128, __half, __half, PA_PF_NS_16B, PA_PF_SB_16B, PA_PF_B_16B>;
 };
 template <> struct Tuned<256, __half, __half> {
   using C = DecodeCfg<256, __half, __half, PA_NS_16B_256, 3>;
+  using CS = void;
   using P = pa::PrefixCfg<256, __half, __half, 4, 2>;
 };
 template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<64, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_64, 8>;
+  using CS = void;
   using P = pa::PrefixCfg<64, __nv_bfloat16, __nv_bfloat16, PA_PF_NS_16B, PA_PF_SB_16B, PA_PF_B_16B>;
 };
 template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128, 8>;
+  using CS = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128 - 1, 8>;
   using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, PA_PF_NS_16B, PA_PF_SB_16B, PA_PF_B_16B>;
 };
 template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_256, 3>;
+  using CS = void;
   using P = pa::PrefixCfg<256, __nv_bfloat16, __nv_bfloat16, 4, 2>;
 };
 template <> struct Tuned<128, __nv_fp8_e4m3, __half> {
   using C = DecodeCfg<128, __nv_fp8_e4m3, __half, PA_NS_FP8_128, PA_MIN_CTAS_FP8_128>;
+  using CS = void;
   using P = pa::PrefixCfg<128, __nv_fp8_e4m3, __half, PA_PX_NS_FP8, PA_PX_SB_FP8>;
 };
 template <> struct Tuned<256, __nv_fp8_e4m3, __half> {
   using C = DecodeCfg<256, __nv_fp8_e4m3, __half, PA_NS_FP8_256, 4>;
+  using CS = void;
   using P = pa::PrefixCfg<256, __nv_fp8_e4m3, __half, 4, 2>;
 };
 
 bool select_kernels(int head_dim, int q_dtype, int kv_dtype, KernelSet* ks) {
-#define PA_CASE(D, KVT, QT) *ks = make_set<typename Tuned<D, KVT, QT>::C, typename Tuned<D, KVT, QT>::P>(); return true
+#define PA_CASE(D, KVT, QT) \
+  *ks = make_set<typename Tuned<D, KVT, QT>::C, typename Tuned<D, KVT, QT>::P, typename Tuned<D, KVT, QT>::CS>(); \
+  return true
   if (kv_dtype == PA_F16 && q_dtype == PA_F16) {
     if (head_dim == 64) { PA_CASE(64, __half, __half); }
     if (head_dim == 128) { PA_CASE(128, __half, __half); }
@@ -389,6 +431,9 @@ PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
       break;
     }
     if ((e = cudaFuncSetAttribute(ks.decode, cudaFuncAttributeMaxDynamicSharedMemorySize, optin)) != cudaSuccess ||
+        (ks.decode_shallow &&
+         (e = cudaFuncSetAttribute(ks.decode_shallow, cudaFuncAttributeMaxDynamicSharedMemorySize, optin)) !=
+             cudaSuccess) ||
         (e = cudaFuncSetAttribute(ks.prefix, cudaFuncAttributeMaxDynamicSharedMemorySize, ks.prefix_smem)) !=
             cudaSuccess ||
         (e = cudaFuncSetAttribute(ks.prefill, cudaFuncAttributeMaxDynamicSharedMemorySize, ks.prefix_smem)) !=
@@ -397,8 +442,8 @@ PA_API int paged_attn_create(const pa_config* cfg, pa_ctx** out) {
       st = cuda_fail(ctx, e, "cudaFuncSetAttribute");
       break;
     }
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ctx->ctas_per_sm, ks.decode, ks.threads,
-                                                           ks.smem(q_slot_bytes(c.num_heads, c.num_kv_heads, c.head_dim), c.max_num_seqs))) != cudaSuccess) {
+    if ((e = choose_decode(&ctx->ks, q_slot_bytes(c.num_heads, c.num_kv_heads, c.head_dim), c.max_num_seqs,
+                           &ctx->ctas_per_sm)) != cudaSuccess) {
       st = cuda_fail(ctx, e, "cudaOccupancyMaxActiveBlocksPerMultiprocessor");
       break;
     }
@@ -901,6 +946,11 @@ int noalloc_setup(int dev, cudaStream_t stream, NoallocDevice* out) {
               cudaSuccess ||
           pin_carveout(ks.decode) != cudaSuccess || pin_carveout(ks.merge) != cudaSuccess)
         return PA_ERR_CUDA;
+      if (ks.decode_shallow &&
+          (cudaFuncSetAttribute(ks.decode_shallow, cudaFuncAttributeMaxDynamicSharedMemorySize, d.smem_optin) !=
+               cudaSuccess ||
+           pin_carveout(ks.decode_shallow) != cudaSuccess))
+        return PA_ERR_CUDA;
     }
     if (cudaMemsetAsync(p, 0, kNoallocHeader, stream) != cudaSuccess) return PA_ERR_CUDA;
     d.scratch = static_cast<unsigned char*>(p);
@@ -971,12 +1021,13 @@ PA_API int paged_attention_decode_noalloc(void* out, const void* query, const vo
   if (st != PA_OK) return st;
   unsigned char* scratch = nd.scratch;
   const int num_sms = nd.num_sms;
-  const size_t smem = ks.smem(q_slot_bytes(num_heads, num_kv_heads, head_dim), num_seqs);
-  if (smem > (size_t)nd.smem_optin) return PA_ERR_UNSUPPORTED;
+  if (ks.smem(q_slot_bytes(num_heads, num_kv_heads, head_dim), num_seqs) > (size_t)nd.smem_optin)
+    return PA_ERR_UNSUPPORTED;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ks.decode, ks.threads, smem) != cudaSuccess ||
+  if (choose_decode(&ks, q_slot_bytes(num_heads, num_kv_heads, head_dim), num_seqs, &per_sm) != cudaSuccess ||
       per_sm < 1)
     return PA_ERR_CUDA;
+  const size_t smem = ks.smem(q_slot_bytes(num_heads, num_kv_heads, head_dim), num_seqs);
 
   CUtensorMap mk, mv;
   if ((st = encode_cache_map(key_cache, kv_dtype, num_kv_heads, head_dim, num_blocks, &mk)) != PA_OK) return st;
