@@ -233,6 +233,12 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
     *dead = 1;
     return false;
   };
+  // The same, voted across the warp, for waits that all 32 lanes make: the
+  // warp takes the failure path together even if the limit ran out for some
+  // lanes only (they meet again at warp-wide operations further on).
+  auto wait_all = [&](uint32_t bar, uint32_t parity) -> bool {
+    return __all_sync(0xffffffffu, wait(bar, parity));
+  };
 
   if (warp == 8) {
     // ---------------------------------------------------------------- TMA producer
@@ -253,10 +259,15 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
         }
       }
       const int phys = __shfl_sync(0xffffffffu, my, i & 31);
+      const int st = i % NS;
+      int ok = 1;
       if (lane == 0) {
-        const int st = i % NS;
-        if (i >= NS && !wait(empty0 + 8 * st, ((i / NS) - 1) & 1)) break;
-        mbar_arrive_expect_tx(full0 + 8 * st, C::STAGE_BYTES);
+        if (i >= NS) ok = wait(empty0 + 8 * st, ((i / NS) - 1) & 1);
+        if (ok) mbar_arrive_expect_tx(full0 + 8 * st, C::STAGE_BYTES);
+      }
+      // (the whole warp leaves together: the lanes meet again at the next shuffle)
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+      if (lane == 0) {
 #pragma unroll
         for (int sub = 0; sub < C::SUBTILES; ++sub) {
           const int x = job.kvh * D + sub * (128 / (int)sizeof(typename C::KV));
@@ -264,8 +275,8 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
           tma_load_2d(base + C::OFF_RING_K + off, &tmK, x, phys * kBS, full0 + 8 * st);
           tma_load_2d(base + C::OFF_RING_V + off, &tmV, x, phys * kBS, full0 + 8 * st);
         }
-        ++issued;
       }
+      ++issued;
     }
     // copies still in flight after a failure: wait for them (bounded) before the CTA exits
     if (lane == 0)
@@ -280,14 +291,14 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
     const int t = threadIdx.x - 128;
     for (int u = 0; u < nsteps; ++u) {
       const int cb = u % B;
-      if (u >= B && !wait(pvdone0 + 8 * cb, ((u - B) / B) & 1)) break;  // step u - B's operands are free
+      if (u >= B && !wait_all(pvdone0 + 8 * cb, ((u - B) / B) & 1)) break;  // step u - B's operands are free
       bool stop = false;
 #pragma unroll 1
       for (int j = 0; j < SB; ++j) {
         const int i = u * SB + j;  // block of the range
         const int st = i % NS;
         const int valid = min(kBS, max(0, job.kv_valid - i * kBS));  // tokens of this block that exist
-        if (i < nb && !wait(full0 + 8 * st, (i / NS) & 1)) {
+        if (i < nb && !wait_all(full0 + 8 * st, (i / NS) & 1)) {
           stop = true;
           break;
         }
@@ -404,7 +415,7 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
     bool ok = true;
     for (int u = 0; u < nsteps && ok; ++u) {
       const int cb = u % B;
-      ok = wait(sfull0 + 8 * cb, (u / B) & 1);
+      ok = wait_all(sfull0 + 8 * cb, (u / B) & 1);
       if (!ok) break;
       tc_fence_after();
       float x[T];
@@ -440,7 +451,7 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
       // this step's max exceeds it by more than 2^8
       const bool grow = bm > m + 8.f;
       if (u > 0 && __any_sync(0xffffffffu, grow)) {
-        ok = wait(pvdone0 + 8 * ((u - 1) % B), ((u - 1) / B) & 1);  // O holds every earlier step
+        ok = wait_all(pvdone0 + 8 * ((u - 1) % B), ((u - 1) / B) & 1);  // O holds every earlier step
         if (!ok) break;
         tc_fence_after();
         const float al = grow ? ex2(m - bm) : 1.f;
@@ -478,7 +489,7 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
       __syncwarp();
       if (lane == 0) mbar_arrive(pfull0 + 8 * cb);
     }
-    if (ok) ok = wait(pvdone0 + 8 * ((nsteps - 1) % B), ((nsteps - 1) / B) & 1);  // the last P V
+    if (ok) ok = wait_all(pvdone0 + 8 * ((nsteps - 1) % B), ((nsteps - 1) / B) & 1);  // the last P V
     if (ok) {
       tc_fence_after();
       const float inv = l > 0.f ? v_scale / l : 0.f;
