@@ -642,6 +642,8 @@ int decode_impl(pa_ctx* ctx, void* out, const void* query, const void* key_cache
   if (pre) {  // shared blocks first: their partials, and each sequence's suffix offset
     pa::PrefixParams q;
     q.query = query;
+    q.k_cache = key_cache;
+    q.v_cache = value_cache;
     q.block_tables = block_tables;
     q.seq_lens = seq_lens;
     q.group_start = pre->group_start;
@@ -798,6 +800,8 @@ PA_API int paged_attention_prefill(pa_ctx* ctx, void* out, const void* query, co
   pa::PrefillParams p;
   p.out = out;
   p.query = query;
+  p.k_cache = key_cache;
+  p.v_cache = value_cache;
   p.block_tables = block_tables;
   p.seq_lens = seq_lens;
   p.query_start = query_start;

@@ -24,6 +24,8 @@ namespace pa {
 struct PrefillParams {
   void* out;                    // [T, Hq, D] query dtype
   const void* query;            // [T, Hq, D]
+  const void* k_cache;          // [num_blocks, 16, Hkv, D]
+  const void* v_cache;
   const int32_t* block_tables;  // [S, bt_stride]
   const int32_t* seq_lens;      // [S]
   const int32_t* query_start;   // [S + 1]
@@ -100,8 +102,10 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
     __device__ void store_ml(int, float, float) const {}
   };
   const Rows rw{&p, rb, tpb, hpu, head0, q_len, qs, len - q_len};
+  const size_t row_stride = (size_t)(p.num_heads / p.group) * C::ROW_BYTES;
   const StackedJob job{p.block_tables + (size_t)s * p.bt_stride, (kv_valid + kBS - 1) / kBS, kv_valid, kvh,
-                       p.num_blocks};
+                       p.num_blocks, static_cast<const uint8_t*>(p.k_cache) + (size_t)kvh * C::ROW_BYTES,
+                       static_cast<const uint8_t*>(p.v_cache) + (size_t)kvh * C::ROW_BYTES, row_stride};
   stacked_attention<C>(tmK, tmV, job, rw, p.scale_log2, p.v_scale, p.err);
 }
 

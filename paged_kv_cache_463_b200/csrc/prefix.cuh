@@ -17,18 +17,23 @@
 // accumulators in tensor memory), one CTA per (group, KV unit, 128 query
 // rows, chunk of 32 prefix blocks).  The core, `stacked_attention`, is shared
 // with the multi-query (prefill) kernel; its roles:
-//   warp 8      TMA producer: each block's K and V tiles into two NS-stage
-//               rings laid out sub-tile-major, so that a step's SB stages
-//               hold its tokens' rows contiguously;
-//   warps 4..7  16-bit caches: the rings are the MMA operands (K K-major, V
-//               MN-major), so these warps only zero V rows past the valid
-//               keys; fp8 caches: they convert each block's K and V rows to
-//               f16 once, into per-step operand buffers;
-//   warp 9      polls the barriers and issues S for a step once its operands
-//               are ready (into one of two TMEM S buffers) and O += P V once
-//               the softmax has written that step's P, with P read from
-//               tensor memory as the A operand; for 16-bit caches the ring
-//               stages are released by tcgen05.commit after the step's P V;
+//   warps 4..7  16-bit caches: copy each step's K and V rows from the cache
+//               into the step's ring stages with 16-byte cp.async (one warp
+//               per step buffer, refilling it as soon as the P V that last
+//               read it completes); the rings, laid out sub-tile-
+//               major so that a step's SB stages hold its tokens' rows
+//               contiguously, are themselves the MMA operands (K K-major, V
+//               MN-major); V rows past the valid keys are written as zeros.
+//               fp8 caches: convert each block's K and V rows to f16 once,
+//               into per-step operand buffers;
+//   warp 8      16-bit caches: issues O += P V for a step once the softmax
+//               has written its P (P read from tensor memory as the A
+//               operand).  fp8 caches: TMA producer of the two NS-stage rings
+//               the converting warps read;
+//   warp 9      issues S for a step into one of B TMEM S buffers once its
+//               operands are ready (16-bit caches: and the buffer's previous
+//               P V has completed).  fp8 caches: also P V, both from one
+//               polling loop;
 //   warps 0..3  one query row per thread: read the step's S row from TMEM,
 //               online softmax in the log2 domain (lazy: O is rescaled in
 //               TMEM only when a row's maximum grows by more than 2^8), write
@@ -46,6 +51,8 @@ enum : int { kCheckBadPrefix = 16 };
 
 struct PrefixParams {
   const void* query;               // [S, Hq, D]
+  const void* k_cache;             // [num_blocks, 16, Hkv, D]
+  const void* v_cache;
   const int32_t* block_tables;     // [S, bt_stride]
   const int32_t* seq_lens;         // [S]
   const int32_t* group_start;      // [num_groups + 1]: group g = sequences [start[g], start[g+1])
@@ -165,6 +172,9 @@ struct StackedJob {
   int kv_valid;          // tokens 0..kv_valid-1 of the range exist
   int kvh;
   int num_blocks;        // physical pool size (ids outside it are flagged and replaced by block 0)
+  const uint8_t* k_head;  // 16-bit caches: this KV head's row of token 0 of block 0, K and V
+  const uint8_t* v_head;
+  size_t row_stride;      // bytes between consecutive token rows of the cache
 };
 
 template <class C, class Rows>
@@ -191,16 +201,15 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
   if (threadIdx.x == 0) {
     for (int i = 0; i < NS; ++i) {
       mbar_init(full0 + 8 * i, 1);
-      // released by the four converting warps (fp8) or by the tensor core (16-bit: tcgen05.commit after P V)
-      mbar_init(empty0 + 8 * i, C::kFp8 ? 4 : 1);
+      mbar_init(empty0 + 8 * i, 4);  // fp8: released by the four converting warps
     }
     for (int i = 0; i < B; ++i) {
-      mbar_init(convf0 + 8 * i, 4);
+      mbar_init(convf0 + 8 * i, C::kFp8 ? 4 : 1);  // fp8: the four converting warps; 16-bit: the loading warp
       mbar_init(sfull0 + 8 * i, 1);  // tcgen05.commit
       mbar_init(pfull0 + 8 * i, 4);  // the four softmax warps
       mbar_init(pvdone0 + 8 * i, 1);
     }
-    mbar_init(fin, 1);
+    mbar_init(fin, C::kFp8 ? 1 : 2);  // the MMA-issuing threads (16-bit: S and P V from two warps)
     *dead = 0;
     *converted = 0;
     fence_mbar_init();
@@ -225,8 +234,10 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  // A failed (timed-out) wait marks the CTA dead: every role then stops.
+  // A failed (timed-out) wait marks the CTA dead: every role then stops at
+  // its next wait that does not complete at once.
   auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+    if (mbar_try_wait(bar, parity)) return true;
     if (*dead) return false;
     if (mbar_wait(bar, parity)) return true;
     atomicOr(err, kCheckWaitTimeout);
@@ -241,7 +252,8 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
   };
 
   if (warp == 8) {
-    // ---------------------------------------------------------------- TMA producer
+    // ---------------------------------------------------------------- TMA producer (fp8)
+    if constexpr (C::kFp8) {
     int issued = 0, my = 0;
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
@@ -281,13 +293,98 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
     // copies still in flight after a failure: wait for them (bounded) before the CTA exits
     if (lane == 0)
       for (int i = *converted; i < issued; ++i) mbar_wait(full0 + 8 * (i % NS), (i / NS) & 1);
+    } else if (lane == 0) {
+      // ---------------------------------------------------------------- 16-bit: P V issue
+      // O += P V for each step once the softmax has written its P (P read
+      // from tensor memory as the A operand, V MN-major from the step's ring
+      // stages); the commit frees the step's S buffer and ring stages.
+      constexpr uint32_t idO = umma_idesc_f16(kPrefixRows, D, C::kBf16, /*b_mn_major=*/true);
+#pragma unroll 1
+      for (int u = 0; u < nsteps; ++u) {
+        const int cb = u % B;
+        if (!wait(pfull0 + 8 * cb, (u / B) & 1)) break;
+        tc_fence_after();
+        const uint32_t pt = tmem + C::S_COL + cb * T;
+        const uint32_t va = base + C::OFF_RING_V + cb * SB * (kBS * 128);
+#pragma unroll
+        for (int k = 0; k < T / 16; ++k) {  // 16-token slices (one block each)
+          const uint64_t b = umma_desc(va + k * (kBS * 128), C::RING_SUB, 1024, kUmmaSwizzle128);
+          umma_f16_ts(tmem + C::O_COL, pt + 8 * k, b, idO, (u > 0 || k > 0) ? 1 : 0);
+        }
+        umma_commit(pvdone0 + 8 * cb);
+      }
+      umma_commit(fin);  // every MMA this thread issued has completed before tensor memory is released
+      mbar_wait(fin, 0);
+    }
+  } else if (warp >= 4 && warp < 8 && !C::kFp8) {
+    // ---------------------------------------------------------------- 16-bit loads
+    // Step u's tokens go to ring stages (u % B) * SB .. + SB - 1, which step
+    // u - B used: its P V must have completed, which also frees S buffer
+    // u % B, so the signal that step u's K and V have landed (`convf`) is
+    // all that S of step u waits for.  Staging warp w < NW loads the steps
+    // u = w mod NW, one at a time (copy, wait for its own copies, then
+    // signal), so that the step buffers refill independently of each other;
+    // every buffer has one loading warp, which therefore never waits on a
+    // buffer's barrier more than one phase ahead.  Lane l moves 16-byte
+    // chunks l, l + 32, ... of the step's T rows (consecutive lanes:
+    // consecutive chunks of a row).
+    static_assert(C::kFp8 || C::NS == SB * B, "16-bit: one ring stage group per step buffer");
+    constexpr int CH = C::ROW_BYTES / 16;  // 16-byte chunks per row
+    constexpr int PER = T * CH / 32;       // chunks per lane per tensor and step
+    static_assert(T * CH % 32 == 0 && SB <= 32, "whole chunks per lane");
+    constexpr int NW = B < 4 ? B : 4;  // loading warps
+    static_assert(B % NW == 0, "each step buffer has one loading warp");
+    const int w = warp - 4;
+    // block-table entries of a step: lane j < SB holds block u * SB + j
+    auto table_entry = [&](int u) -> int {
+      const int i = u * SB + lane;
+      int phys = 0;
+      if (lane < SB && i < nb) {
+        phys = __ldg(job.table + i);
+        if (phys < 0 || phys >= job.num_blocks) {
+          atomicOr(err, kCheckBadBlock);
+          phys = 0;
+        }
+      }
+      return phys;
+    };
+    int entry = w < NW && w < nsteps ? table_entry(w) : 0;
+#pragma unroll 1
+    for (int u = w; w < NW && u < nsteps; u += NW) {
+      if (u >= B && !wait_all(pvdone0 + 8 * (u % B), ((u - B) / B) & 1)) break;  // step u - B's stages are free
+      const int cb = u % B;
+#pragma unroll
+      for (int k = 0; k < PER; ++k) {
+        const int c = lane + 32 * k;
+        const int row = c / CH, cc = c % CH;  // token u * T + row of the range, 16-byte chunk cc
+        const int j = row / kBS, r = row % kBS;
+        const int phys = __shfl_sync(0xffffffffu, entry, j);
+        const uint32_t off = C::ring(cb * SB + j, r, 16 * cc);
+        const size_t src = ((size_t)phys * kBS + r) * job.row_stride + 16 * cc;
+        // K rows of blocks past the range keep older contents: their scores are masked
+        if (u * SB + j < nb)
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(base + C::OFF_RING_K + off),
+                       "l"(job.k_head + src) : "memory");
+        if (u * T + row < job.kv_valid)
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(base + C::OFF_RING_V + off),
+                       "l"(job.v_head + src) : "memory");
+        else  // P is 0 there, and 0 * garbage could be NaN
+          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(base + C::OFF_RING_V + off), "r"(0u)
+                       : "memory");
+      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      if (u + NW < nsteps) entry = table_entry(u + NW);  // (in flight while the copies land)
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      fence_proxy_async_smem();  // -> visible to the tensor core
+      __syncwarp();
+      if (lane == 0) mbar_arrive(convf0 + 8 * cb);
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // nothing in flight when the CTA exits
   } else if (warp >= 4 && warp < 8) {
-    // ---------------------------------------------------------------- operand staging
-    // fp8: convert each block's K and V rows to f16 (row for row, 128-byte
+    // ---------------------------------------------------------------- fp8 operand staging
+    // Convert each block's K and V rows to f16 (row for row, 128-byte
     // swizzled, the step's SB blocks stacked) and release the ring stage.
-    // 16-bit: the ring is the operand; only V rows past the range's valid
-    // keys are zeroed (P is 0 there, and 0 * garbage could be NaN; the stage
-    // of a block past the range still holds an older block).
+    if constexpr (C::kFp8) {
     const int t = threadIdx.x - 128;
     for (int u = 0; u < nsteps; ++u) {
       const int cb = u % B;
@@ -302,7 +399,7 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
           stop = true;
           break;
         }
-        if constexpr (C::kFp8) {
+        {
           uint8_t* kf = smem + C::OFF_KF + cb * C::F_BYTES;
           uint8_t* vf = smem + C::OFF_VF + cb * C::F_BYTES;
           for (int k = t; k < 2 * kBS * (D / 16); k += 128) {  // (K|V, row, 16 codes) -> 16 halves
@@ -327,14 +424,6 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
             if (lane == 0) mbar_arrive(empty0 + 8 * st);
             if (t == 0) *converted = i + 1;
           }
-        } else {
-          if (valid < kBS) {  // zero V rows valid..15 of this stage, every sub-tile
-            for (int k = t; k < (kBS - valid) * C::SUBTILES * 8; k += 128) {
-              const int r = valid + k / (C::SUBTILES * 8), rest = k % (C::SUBTILES * 8);
-              *reinterpret_cast<uint4*>(smem + C::OFF_RING_V + C::ring(st, r, 16 * rest)) = make_uint4(0u, 0u, 0u, 0u);
-            }
-          }
-          if (t == 0 && i < nb) *converted = i + 1;
         }
       }
       if (stop) break;
@@ -342,8 +431,36 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
       __syncwarp();
       if (lane == 0) mbar_arrive(convf0 + 8 * cb);
     }
+    }
+  } else if (warp == 9 && !C::kFp8) {
+    // ---------------------------------------------------------------- 16-bit: S issue
+    // S = Q K^T for each step once its K and V have landed; the loading
+    // warp refilled the step's stages only after the P V of the step that
+    // last used them (and its S buffer) had completed.  (P V is issued by
+    // warp 8: one thread issues a tcgen05.mma every ~80 cycles at best, so
+    // the two streams of MMAs come from two threads.)
+    if (lane == 0) {
+      constexpr uint32_t idS = umma_idesc_f16(kPrefixRows, T, C::kBf16);
+      const uint32_t qa = base + C::OFF_Q;
+#pragma unroll 1
+      for (int u = 0; u < nsteps; ++u) {
+        const int cb = u % B;
+        if (!wait(convf0 + 8 * cb, (u / B) & 1)) break;
+        tc_fence_after();
+        const uint32_t kb = base + C::OFF_RING_K + cb * SB * (kBS * 128);
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {  // 16-wide slices of D
+          const uint64_t a = umma_desc(qa + (k >> 2) * (kPrefixRows * 128) + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
+          const uint64_t b = umma_desc(kb + (k >> 2) * C::RING_SUB + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
+          umma_f16(tmem + C::S_COL + cb * T, a, b, idS, k > 0);
+        }
+        umma_commit(sfull0 + 8 * cb);
+      }
+      umma_commit(fin);
+      mbar_wait(fin, 0);
+    }
   } else if (warp == 9) {
-    // ---------------------------------------------------------------- MMA issue
+    // ---------------------------------------------------------------- fp8: MMA issue
     if (lane == 0) {
       constexpr uint32_t idS = umma_idesc_f16(kPrefixRows, T, C::kBf16);
       constexpr uint32_t idO = umma_idesc_f16(kPrefixRows, D, C::kBf16, /*b_mn_major=*/true);
@@ -386,10 +503,7 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
             const uint64_t b = umma_desc(va + k * (kBS * 128), VSUB, 1024, kUmmaSwizzle128);
             umma_f16_ts(tmem + C::O_COL, pt + 8 * k, b, idO, (npv > 0 || k > 0) ? 1 : 0);
           }
-          umma_commit(pvdone0 + 8 * cb);
-          if constexpr (!C::kFp8) {  // the step's ring stages are free once these MMAs complete
-            for (int j = 0; j < SB && npv * SB + j < nb; ++j) umma_commit(empty0 + 8 * ((npv * SB + j) % NS));
-          }
+          umma_commit(pvdone0 + 8 * cb);  // (16-bit: the step's ring stages are free once it arrives)
           ++npv;
           progress = true;
         }
@@ -418,33 +532,38 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
       ok = wait_all(sfull0 + 8 * cb, (u / B) & 1);
       if (!ok) break;
       tc_fence_after();
-      float x[T];
-#pragma unroll
-      for (int c0 = 0; c0 < T; c0 += 16) {
-        uint32_t sv[16];
-        tmem_ld16(trow + C::S_COL + cb * T + c0, sv);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) x[c0 + j] = __uint_as_float(sv[j]);
-      }
-      tmem_wait_ld();
+      // The step's T scores, TC at a time in registers: with T > TC a first
+      // pass over the chunks (last to first) takes the maximum, a second
+      // (first to last, the first chunk still in registers) the exponentials.
+      constexpr int TC = T < 32 ? T : 32, NCH = T / TC;
+      static_assert(T % TC == 0, "whole chunks");
       const int valid = min(T, lim - u * T);  // keys of this step the row sees
-      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent max chains
       // Steps before the diagonal, where every row of the warp sees every key
       // and the scale is positive, take the max of the raw scores and fold
       // the scale into the exponent's FMA; the others scale and mask first.
       const bool plain = scale_log2 > 0.f && __all_sync(0xffffffffu, valid >= T);
-      float xs;  // exponent = x * xs - m
-      if (plain) {
+      const float xs = plain ? scale_log2 : 1.f;  // exponent = x * xs - m
+      float x[TC];
+      auto load = [&](int ch) {
 #pragma unroll
-        for (int j = 0; j < T; ++j) mx[j & 3] = fmaxf(mx[j & 3], x[j]);
-        xs = scale_log2;
-      } else {
+        for (int c0 = 0; c0 < TC; c0 += 16) {
+          uint32_t sv[16];
+          tmem_ld16(trow + C::S_COL + cb * T + ch * TC + c0, sv);
 #pragma unroll
-        for (int j = 0; j < T; ++j) {
-          x[j] = j < valid ? x[j] * scale_log2 : -INFINITY;
-          mx[j & 3] = fmaxf(mx[j & 3], x[j]);
+          for (int j = 0; j < 16; ++j) x[c0 + j] = __uint_as_float(sv[j]);
         }
-        xs = 1.f;
+        tmem_wait_ld();
+        if (!plain) {
+#pragma unroll
+          for (int j = 0; j < TC; ++j) x[j] = ch * TC + j < valid ? x[j] * scale_log2 : -INFINITY;
+        }
+      };
+      float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};  // four independent max chains
+#pragma unroll
+      for (int ch = NCH - 1; ch >= 0; --ch) {
+        load(ch);
+#pragma unroll
+        for (int j = 0; j < TC; ++j) mx[j & 3] = fmaxf(mx[j & 3], x[j]);
       }
       const float bm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * xs;
       // lazy rescaling: move the reference max (and rescale l, O) only when
@@ -469,19 +588,24 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
       }
       if (grow) m = bm;
       // P of row r as 16-bit pairs over the first T/2 columns of this S
-      // buffer (its S values are all in registers by now): the A operand of
-      // the step's P V.  The buffer's next S is issued only after that P V.
+      // buffer: chunk ch's P goes to columns ch * TC / 2 .., which held
+      // scores of chunk ch / 2 <= ch, already read.  It is the A operand of
+      // the step's P V; the buffer's next S is issued only after that P V.
       float sm[4] = {0.f, 0.f, 0.f, 0.f};  // four independent sum chains
 #pragma unroll
-      for (int c0 = 0; c0 < T / 2; c0 += 16) {
-        uint32_t pk[16];
+      for (int ch = 0; ch < NCH; ++ch) {
+        if (ch > 0) load(ch);
 #pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float p0 = ex2(fmaf(x[2 * (c0 + q)], xs, -m)), p1 = ex2(fmaf(x[2 * (c0 + q) + 1], xs, -m));
-          sm[q & 3] += p0 + p1;
-          pk[q] = pack2<C::kBf16>(p0, p1);
+        for (int c0 = 0; c0 < TC / 2; c0 += 16) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int q = 0; q < 16; ++q) {
+            const float p0 = ex2(fmaf(x[2 * (c0 + q)], xs, -m)), p1 = ex2(fmaf(x[2 * (c0 + q) + 1], xs, -m));
+            sm[q & 3] += p0 + p1;
+            pk[q] = pack2<C::kBf16>(p0, p1);
+          }
+          tmem_st16(trow + C::S_COL + cb * T + ch * (TC / 2) + c0, pk);
         }
-        tmem_st16(trow + C::S_COL + cb * T + c0, pk);
       }
       l += (sm[0] + sm[1]) + (sm[2] + sm[3]);
       tmem_wait_st();
@@ -613,7 +737,10 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
     }
   };
   const Rows rw{&p, rb, rows, first, hpu, head0, chunk};
-  const StackedJob job{p.block_tables + (size_t)first * p.bt_stride + b0, nb, nb * kBS, kvh, p.num_blocks};
+  const size_t row_stride = (size_t)(p.num_heads / p.group) * C::ROW_BYTES;
+  const StackedJob job{p.block_tables + (size_t)first * p.bt_stride + b0, nb, nb * kBS, kvh, p.num_blocks,
+                       static_cast<const uint8_t*>(p.k_cache) + (size_t)kvh * C::ROW_BYTES,
+                       static_cast<const uint8_t*>(p.v_cache) + (size_t)kvh * C::ROW_BYTES, row_stride};
   stacked_attention<C>(tmK, tmV, job, rw, p.scale_log2, p.v_scale, p.err);
 }
 
