@@ -186,66 +186,58 @@ struct Tuned;
 #ifndef PA_MIN_CTAS_FP8_128
 #define PA_MIN_CTAS_FP8_128 8
 #endif
-// The tensor-core passes (shared prefixes, prefill): ring stages (blocks),
-// blocks per step and step buffers.  16-bit head_dim 64 / 128: 32-key steps
-// with four S buffers (the MMAs run up to three steps ahead of the softmax),
-// which still leave room (tensor and shared memory) for two CTAs per SM, so
-// that two softmax warps share each scheduler; longer steps with one CTA per
-// SM measured slower (the softmax warps, not the tensor core, set the pace).
-#ifndef PA_PX_NS_FP8
-#define PA_PX_NS_FP8 8
+// The tensor-core passes (shared prefixes, prefill): blocks per step and
+// step buffers.  head_dim 64 / 128: 32-key steps with four step buffers (the
+// steps run up to three ahead of the softmax, and four warps load and issue
+// S for them), which still leave room (tensor and shared memory) for two
+// CTAs per SM, so that two softmax warps share each scheduler; 64-key steps
+// with two buffers measured slower (a buffer's refill then sits on the
+// critical path).  head_dim 256: 32-key steps, two buffers (one CTA per SM).
+#ifndef PA_PX_SB
+#define PA_PX_SB 2
 #endif
-#ifndef PA_PX_SB_FP8
-#define PA_PX_SB_FP8 4
-#endif
-#ifndef PA_PF_NS_16B
-#define PA_PF_NS_16B 8
-#endif
-#ifndef PA_PF_SB_16B
-#define PA_PF_SB_16B 2
-#endif
-#ifndef PA_PF_B_16B
-#define PA_PF_B_16B 4
+#ifndef PA_PX_B
+#define PA_PX_B 4
 #endif
 template <> struct Tuned<64, __half, __half> {
   using C = DecodeCfg<64, __half, __half, PA_NS_16B_64, 8>;
   using CS = void;
-  using P = pa::PrefixCfg<64, __half, __half, PA_PF_NS_16B, PA_PF_SB_16B, PA_PF_B_16B>;
+  using P = pa::PrefixCfg<64, __half, __half, PA_PX_SB, PA_PX_B>;
 };
 template <> struct Tuned<128, __half, __half> {
   using C = DecodeCfg<128, __half, __half, PA_NS_16B_128, 8>;
   using CS = DecodeCfg<128, __half, __half, PA_NS_16B_128 - 1, 8>;
-  using P = pa::PrefixCfg<128, __half, __half, PA_PF_NS_16B, PA_PF_SB_16B, PA_PF_B_16B>;
+  using P = pa::PrefixCfg<128, __half, __half, PA_PX_SB, PA_PX_B>;
 };
 template <> struct Tuned<256, __half, __half> {
   using C = DecodeCfg<256, __half, __half, PA_NS_16B_256, 3>;
   using CS = void;
-  using P = pa::PrefixCfg<256, __half, __half, 4, 2>;
+  using P = pa::PrefixCfg<256, __half, __half, 2, 2>;
 };
 template <> struct Tuned<64, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<64, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_64, 8>;
   using CS = void;
-  using P = pa::PrefixCfg<64, __nv_bfloat16, __nv_bfloat16, PA_PF_NS_16B, PA_PF_SB_16B, PA_PF_B_16B>;
+  using P = pa::PrefixCfg<64, __nv_bfloat16, __nv_bfloat16, PA_PX_SB, PA_PX_B>;
 };
 template <> struct Tuned<128, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128, 8>;
   using CS = DecodeCfg<128, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_128 - 1, 8>;
-  using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, PA_PF_NS_16B, PA_PF_SB_16B, PA_PF_B_16B>;
+  using P = pa::PrefixCfg<128, __nv_bfloat16, __nv_bfloat16, PA_PX_SB, PA_PX_B>;
 };
 template <> struct Tuned<256, __nv_bfloat16, __nv_bfloat16> {
   using C = DecodeCfg<256, __nv_bfloat16, __nv_bfloat16, PA_NS_16B_256, 3>;
   using CS = void;
-  using P = pa::PrefixCfg<256, __nv_bfloat16, __nv_bfloat16, 4, 2>;
+  using P = pa::PrefixCfg<256, __nv_bfloat16, __nv_bfloat16, 2, 2>;
 };
 template <> struct Tuned<128, __nv_fp8_e4m3, __half> {
   using C = DecodeCfg<128, __nv_fp8_e4m3, __half, PA_NS_FP8_128, PA_MIN_CTAS_FP8_128>;
   using CS = void;
-  using P = pa::PrefixCfg<128, __nv_fp8_e4m3, __half, PA_PX_NS_FP8, PA_PX_SB_FP8>;
+  using P = pa::PrefixCfg<128, __nv_fp8_e4m3, __half, PA_PX_SB, PA_PX_B>;
 };
 template <> struct Tuned<256, __nv_fp8_e4m3, __half> {
   using C = DecodeCfg<256, __nv_fp8_e4m3, __half, PA_NS_FP8_256, 4>;
   using CS = void;
-  using P = pa::PrefixCfg<256, __nv_fp8_e4m3, __half, 4, 2>;
+  using P = pa::PrefixCfg<256, __nv_fp8_e4m3, __half, 2, 2>;
 };
 
 bool select_kernels(int head_dim, int q_dtype, int kv_dtype, KernelSet* ks) {
@@ -666,7 +658,7 @@ int decode_impl(pa_ctx* ctx, void* out, const void* query, const void* key_cache
     q.row_blocks = row_blocks;
     q.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
     q.v_scale = fp8 ? v_scale : 1.0f;
-    void* qargs[] = {&mk, &mv, &q};
+    void* qargs[] = {&q};
     // grid.y: the attention CTAs, plus one row whose x = 0 CTA checks each group
     const dim3 grid((unsigned)(prefix_chunks > 0 ? prefix_chunks : 1), (unsigned)(kv_units * row_blocks + 1),
                     (unsigned)pre->num_groups);
@@ -793,10 +785,6 @@ PA_API int paged_attention_prefill(pa_ctx* ctx, void* out, const void* query, co
   if (fp8 && !(k_scale > 0.f && v_scale > 0.f && std::isfinite(k_scale) && std::isfinite(v_scale)))
     return fail(ctx, PA_ERR_INVALID_ARG, "fp8 scales must be finite and > 0");
   cudaSetDevice(ctx->device);
-  CUtensorMap mk, mv;
-  int st = tensor_map(ctx, key_cache, &mk);
-  if (st != PA_OK) return st;
-  if ((st = tensor_map(ctx, value_cache, &mv)) != PA_OK) return st;
   pa::PrefillParams p;
   p.out = out;
   p.query = query;
@@ -820,7 +808,7 @@ PA_API int paged_attention_prefill(pa_ctx* ctx, void* out, const void* query, co
   const int tpb = pa::kPrefixRows / hmax;  // query tokens per CTA (fewest: the widest KV unit)
   const dim3 grid((unsigned)((max_query_len + tpb - 1) / tpb), (unsigned)(c.num_kv_heads * p.head_splits),
                   (unsigned)num_seqs);
-  void* args[] = {&mk, &mv, &p};
+  void* args[] = {&p};
   cudaError_t e = cudaLaunchKernel(ctx->ks.prefill, grid, dim3(ctx->ks.prefix_threads), args, ctx->ks.prefix_smem,
                                    reinterpret_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? PA_OK : cuda_fail(ctx, e, "prefill launch");

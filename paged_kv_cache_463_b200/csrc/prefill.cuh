@@ -44,8 +44,7 @@ struct PrefillParams {
 
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
-    paged_prefill_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                         const PrefillParams p) {
+    paged_prefill_kernel(const PrefillParams p) {
   using Q = typename C::Q;
   constexpr int D = C::D;
   const int s = blockIdx.z;
@@ -103,10 +102,10 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
   };
   const Rows rw{&p, rb, tpb, hpu, head0, q_len, qs, len - q_len};
   const size_t row_stride = (size_t)(p.num_heads / p.group) * C::ROW_BYTES;
-  const StackedJob job{p.block_tables + (size_t)s * p.bt_stride, (kv_valid + kBS - 1) / kBS, kv_valid, kvh,
+  const StackedJob job{p.block_tables + (size_t)s * p.bt_stride, (kv_valid + kBS - 1) / kBS, kv_valid,
                        p.num_blocks, static_cast<const uint8_t*>(p.k_cache) + (size_t)kvh * C::ROW_BYTES,
                        static_cast<const uint8_t*>(p.v_cache) + (size_t)kvh * C::ROW_BYTES, row_stride};
-  stacked_attention<C>(tmK, tmV, job, rw, p.scale_log2, p.v_scale, p.err);
+  stacked_attention<C>(job, rw, p.scale_log2, p.v_scale, p.err);
 }
 
 }  // namespace pa

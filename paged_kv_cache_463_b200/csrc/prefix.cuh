@@ -20,7 +20,8 @@
 //   warps 4..7  16-bit caches: copy each step's K and V rows from the cache
 //               into the step's ring stages with 16-byte cp.async (one warp
 //               per step buffer, refilling it as soon as the P V that last
-//               read it completes); the rings, laid out sub-tile-
+//               read it completes) and issue the step's S into its TMEM S
+//               buffer once the rows have landed; the rings, laid out sub-tile-
 //               major so that a step's SB stages hold its tokens' rows
 //               contiguously, are themselves the MMA operands (K K-major, V
 //               MN-major); V rows past the valid keys are written as zeros.
@@ -30,10 +31,9 @@
 //               has written its P (P read from tensor memory as the A
 //               operand).  fp8 caches: TMA producer of the two NS-stage rings
 //               the converting warps read;
-//   warp 9      issues S for a step into one of B TMEM S buffers once its
-//               operands are ready (16-bit caches: and the buffer's previous
-//               P V has completed).  fp8 caches: also P V, both from one
-//               polling loop;
+//   warp 9      fp8 caches: issues S for a step into one of B TMEM S buffers
+//               once its operands are ready, and P V, both from one polling
+//               loop;
 //   warps 0..3  one query row per thread: read the step's S row from TMEM,
 //               online softmax in the log2 domain (lazy: O is rescaled in
 //               TMEM only when a row's maximum grows by more than 2^8), write
@@ -79,40 +79,39 @@ struct PrefixParams {
 
 constexpr int kPrefixRows = 128;  // query rows per CTA (the MMA M)
 
+
 // Shared memory per SM, for capping residency.
 constexpr int kSmemPerSM = 233472;
 
-template <int D_, typename KV_, typename Q_, int NS_, int SB_, int B_ = 2>
+template <int D_, typename KV_, typename Q_, int SB_, int B_>
 struct PrefixCfg {
   static constexpr int D = D_;
   using KV = KV_;
   using Q = Q_;
-  static constexpr int NS = NS_;   // ring stages (blocks)
   static constexpr int SB = SB_;   // blocks per step
   static constexpr int T = SB * kBS;  // tokens per step (the S MMA's N, the P V MMA's K)
-  static constexpr int B = B_;     // step buffers (S and P, and the fp8 operands): how far the MMAs may run ahead
+  static constexpr int B = B_;     // step buffers (S and P in TMEM, K and V in shared memory): how far the steps run ahead
+  static constexpr int NW = B < 4 ? B : 4;  // loading warps: one per step buffer
   static constexpr bool kFp8 = sizeof(KV) == 1;
   static constexpr bool kBf16 = std::is_same<Q, __nv_bfloat16>::value;
-  static constexpr int ROW_BYTES = D * (int)sizeof(KV);
-  static constexpr int SUBTILES = ROW_BYTES / 128;
-  static constexpr int TILE_BYTES = kBS * ROW_BYTES;
-  static constexpr int STAGE_BYTES = 2 * TILE_BYTES;  // K + V of one block
-  // The K and V rings are each [SUBTILES][NS][16 rows x 128 B] (TMA 128-byte
-  // swizzle): the SB consecutive stages of a step hold its tokens' rows of one
-  // sub-tile contiguously, so a 16-bit ring is itself the MMA operand
-  // (K K-major, V MN-major; 8-row atoms 1024 bytes apart).
-  static constexpr int RING_SUB = NS * kBS * 128;      // bytes between a ring's sub-tiles
+  static constexpr int ROW_BYTES = D * (int)sizeof(KV);  // one token's K (or V) row of one KV head in the cache
+  static constexpr int CH = ROW_BYTES / 16;               // its 16-byte chunks
+  // Step buffer layout (both K and V, 16-bit operands, TMA-style 128-byte
+  // swizzle): [D / 64 sub-tiles][T rows x 128 B], so that a sub-tile is a
+  // K-major (K) or MN-major (V) MMA operand with 8-row atoms 1024 bytes apart.
+  static constexpr int BUF_SUB = T * 128;          // bytes between a step buffer's sub-tiles
+  static constexpr int BUF_BYTES = T * D * 2;      // one step buffer of K or V
   static constexpr int Q_BYTES = kPrefixRows * D * 2;  // 128-byte swizzled, D/64 sub-tiles of 128 rows
-  static constexpr int F_BYTES = kFp8 ? T * D * 2 : 0;  // fp8 only: a step's K or V as f16, D/64 sub-tiles of T rows
   static constexpr int OFF_Q = 0;
-  static constexpr int OFF_RING_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_RING_V = OFF_RING_K + NS * TILE_BYTES;
-  static constexpr int OFF_KF = OFF_RING_V + NS * TILE_BYTES;  // [B] (fp8)
-  static constexpr int OFF_VF = OFF_KF + B * F_BYTES;          // [B] (fp8)
-  static constexpr int OFF_BAR = OFF_VF + B * F_BYTES;
-  // full[NS] empty[NS] conv_full[B] s_full[B] p_full[B] pv_done[B] fin
-  static constexpr int NBARS = 2 * NS + 4 * B + 1;
-  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem base, dead flag, blocks converted
+  static constexpr int OFF_K = OFF_Q + Q_BYTES;    // [B] step buffers
+  static constexpr int OFF_V = OFF_K + B * BUF_BYTES;
+  // fp8: each loading warp's raw staging of one step (its K rows, then its V rows, cache layout)
+  static constexpr int RAW_BYTES = kFp8 ? 2 * T * ROW_BYTES : 0;
+  static constexpr int OFF_RAW = OFF_V + B * BUF_BYTES;  // [NW]
+  static constexpr int OFF_BAR = OFF_RAW + NW * RAW_BYTES;
+  // s_full[B] p_full[B] pv_done[B] fin
+  static constexpr int NBARS = 3 * B + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem base, dead flag
   static constexpr int TMEM_COLS = D + B * T <= 128 ? 128 : (D + B * T <= 256 ? 256 : 512);
   // O: D columns; S buffers: T columns each, a step's P over the first T/2 of its buffer
   static constexpr int O_COL = 0, S_COL = D;
@@ -121,26 +120,20 @@ struct PrefixCfg {
   // at least this much shared memory, so that no more than MAX_CTAS CTAs are resident
   static constexpr int MIN_BYTES = kSmemPerSM / (MAX_CTAS + 1) + 1024;
   static constexpr int SMEM_BYTES = LAYOUT_BYTES > MIN_BYTES ? LAYOUT_BYTES : MIN_BYTES;
-  static constexpr int THREADS = 320;
-  // register budget: as many CTAs per SM as tensor and shared memory allow,
-  // up to two (~100 registers a thread: the softmax keeps a step's T scores)
+  static constexpr int THREADS = 288;  // softmax warps 0..3, loading warps 4..7, P V warp 8
+  // register budget: as many CTAs per SM as tensor and shared memory allow, up to two
   static constexpr int SMEM_CTAS = kSmemPerSM / (SMEM_BYTES + 1024);
   static constexpr int FIT_CTAS = MAX_CTAS < SMEM_CTAS ? MAX_CTAS : SMEM_CTAS;
   static constexpr int REG_CTAS = FIT_CTAS < 2 ? FIT_CTAS : 2;
   static_assert(ROW_BYTES % 128 == 0, "rows must be whole 128-byte swizzle spans");
   static_assert(D % 64 == 0, "head_dim must be a multiple of 64");
   static_assert(T % 32 == 0 && T <= 256, "step tokens (P is stored 16 columns at a time)");
-  static_assert(NS % SB == 0, "a step's blocks occupy consecutive ring stages");
+  static_assert(B % NW == 0 && SB <= 32, "each step buffer has one loading warp");
   static_assert(!kFp8 || std::is_same<Q, __half>::value, "fp8 caches pair with fp16 queries");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
   // byte offset of (row, byte-in-row) in a 128-byte-swizzled tile of `rows` rows
   __device__ static uint32_t sw128(int rows, int row, int byte) {
     return (uint32_t)((byte >> 7) * (rows * 128) + row * 128 + (((((byte & 127) >> 4) ^ (row & 7)) << 4) | (byte & 15)));
-  }
-  // byte offset of (row, byte-in-row) of ring stage st, in a K or V ring
-  __device__ static uint32_t ring(int st, int row, int byte) {
-    return (uint32_t)((byte >> 7) * RING_SUB + st * (kBS * 128) + row * 128 +
-                      (((((byte & 127) >> 4) ^ (row & 7)) << 4) | (byte & 15)));
   }
 };
 
@@ -165,53 +158,40 @@ __device__ __forceinline__ int group_prefix_blocks(const PrefixParams& p, int g,
 //   int limit(r)                  keys of the range row r sees (a prefix of it)
 //   void store(r, c0, v[16])      normalised output dims c0..c0+15 (times v_scale)
 //   void store_ml(r, m, l)        the row's max (log2 units) and sum
-// Called by all 320 threads of the CTA; returns after tensor memory is freed.
+// Called by all C::THREADS threads of the CTA; returns after tensor memory is freed.
 struct StackedJob {
   const int32_t* table;  // nb block ids
   int nb;
   int kv_valid;          // tokens 0..kv_valid-1 of the range exist
-  int kvh;
   int num_blocks;        // physical pool size (ids outside it are flagged and replaced by block 0)
-  const uint8_t* k_head;  // 16-bit caches: this KV head's row of token 0 of block 0, K and V
+  const uint8_t* k_head;  // this KV head's row of token 0 of block 0 in the K and V caches
   const uint8_t* v_head;
   size_t row_stride;      // bytes between consecutive token rows of the cache
 };
 
 template <class C, class Rows>
-__device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const CUtensorMap& tmV, const StackedJob& job,
-                                                  const Rows& rows, float scale_log2, float v_scale, int* err) {
-  using Q = typename C::Q;
-  constexpr int D = C::D, NS = C::NS;
+__device__ __forceinline__ void stacked_attention(const StackedJob& job, const Rows& rows, float scale_log2,
+                                                  float v_scale, int* err) {
+  constexpr int D = C::D, B = C::B, SB = C::SB, T = C::T, NW = C::NW, CH = C::CH;
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
   const uint32_t base = smem_u32(smem);
-  const uint32_t bar0 = base + C::OFF_BAR;
-  const uint32_t full0 = bar0, empty0 = bar0 + 8 * NS, convf0 = bar0 + 16 * NS, sfull0 = convf0 + 8 * C::B,
-                 pfull0 = sfull0 + 8 * C::B, pvdone0 = pfull0 + 8 * C::B, fin = pvdone0 + 8 * C::B;
+  const uint32_t sfull0 = base + C::OFF_BAR, pfull0 = sfull0 + 8 * B, pvdone0 = pfull0 + 8 * B, fin = pvdone0 + 8 * B;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* dead = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
-  volatile int* converted = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nb = job.nb;
-  (void)sizeof(Q);
+  const int nsteps = (nb + SB - 1) / SB;
 
   // ---- set-up: barriers, tensor memory, the query tile (128-byte swizzled)
-  constexpr int B = C::B, SB = C::SB, T = C::T;
-  const int nsteps = (nb + SB - 1) / SB;
   if (threadIdx.x == 0) {
-    for (int i = 0; i < NS; ++i) {
-      mbar_init(full0 + 8 * i, 1);
-      mbar_init(empty0 + 8 * i, 4);  // fp8: released by the four converting warps
-    }
     for (int i = 0; i < B; ++i) {
-      mbar_init(convf0 + 8 * i, C::kFp8 ? 4 : 1);  // fp8: the four converting warps; 16-bit: the loading warp
-      mbar_init(sfull0 + 8 * i, 1);  // tcgen05.commit
+      mbar_init(sfull0 + 8 * i, 1);  // tcgen05.commit after the step's S
       mbar_init(pfull0 + 8 * i, 4);  // the four softmax warps
-      mbar_init(pvdone0 + 8 * i, 1);
+      mbar_init(pvdone0 + 8 * i, 1);  // tcgen05.commit after the step's P V
     }
-    mbar_init(fin, C::kFp8 ? 1 : 2);  // the MMA-issuing threads (16-bit: S and P V from two warps)
+    mbar_init(fin, 1 + NW);  // the MMA-issuing threads: the loading warps' (S) and warp 8's (P V)
     *dead = 0;
-    *converted = 0;
     fence_mbar_init();
   }
   if (warp == 0) tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -251,89 +231,30 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
     return __all_sync(0xffffffffu, wait(bar, parity));
   };
 
-  if (warp == 8) {
-    // ---------------------------------------------------------------- TMA producer (fp8)
-    if constexpr (C::kFp8) {
-    int issued = 0, my = 0;
-    if (lane == 0) {
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-    }
-    for (int i = 0; i < nb; ++i) {
-      if ((i & 31) == 0) {  // the next 32 table entries, one per lane
-        my = 0;
-        if (i + lane < nb) {
-          my = __ldg(job.table + i + lane);
-          if (my < 0 || my >= job.num_blocks) {
-            atomicOr(err, kCheckBadBlock);
-            my = 0;
-          }
-        }
-      }
-      const int phys = __shfl_sync(0xffffffffu, my, i & 31);
-      const int st = i % NS;
-      int ok = 1;
-      if (lane == 0) {
-        if (i >= NS) ok = wait(empty0 + 8 * st, ((i / NS) - 1) & 1);
-        if (ok) mbar_arrive_expect_tx(full0 + 8 * st, C::STAGE_BYTES);
-      }
-      // (the whole warp leaves together: the lanes meet again at the next shuffle)
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      if (lane == 0) {
-#pragma unroll
-        for (int sub = 0; sub < C::SUBTILES; ++sub) {
-          const int x = job.kvh * D + sub * (128 / (int)sizeof(typename C::KV));
-          const uint32_t off = sub * C::RING_SUB + st * (kBS * 128);
-          tma_load_2d(base + C::OFF_RING_K + off, &tmK, x, phys * kBS, full0 + 8 * st);
-          tma_load_2d(base + C::OFF_RING_V + off, &tmV, x, phys * kBS, full0 + 8 * st);
-        }
-      }
-      ++issued;
-    }
-    // copies still in flight after a failure: wait for them (bounded) before the CTA exits
-    if (lane == 0)
-      for (int i = *converted; i < issued; ++i) mbar_wait(full0 + 8 * (i % NS), (i / NS) & 1);
-    } else if (lane == 0) {
-      // ---------------------------------------------------------------- 16-bit: P V issue
-      // O += P V for each step once the softmax has written its P (P read
-      // from tensor memory as the A operand, V MN-major from the step's ring
-      // stages); the commit frees the step's S buffer and ring stages.
-      constexpr uint32_t idO = umma_idesc_f16(kPrefixRows, D, C::kBf16, /*b_mn_major=*/true);
-#pragma unroll 1
-      for (int u = 0; u < nsteps; ++u) {
-        const int cb = u % B;
-        if (!wait(pfull0 + 8 * cb, (u / B) & 1)) break;
-        tc_fence_after();
-        const uint32_t pt = tmem + C::S_COL + cb * T;
-        const uint32_t va = base + C::OFF_RING_V + cb * SB * (kBS * 128);
-#pragma unroll
-        for (int k = 0; k < T / 16; ++k) {  // 16-token slices (one block each)
-          const uint64_t b = umma_desc(va + k * (kBS * 128), C::RING_SUB, 1024, kUmmaSwizzle128);
-          umma_f16_ts(tmem + C::O_COL, pt + 8 * k, b, idO, (u > 0 || k > 0) ? 1 : 0);
-        }
-        umma_commit(pvdone0 + 8 * cb);
-      }
-      umma_commit(fin);  // every MMA this thread issued has completed before tensor memory is released
-      mbar_wait(fin, 0);
-    }
-  } else if (warp >= 4 && warp < 8 && !C::kFp8) {
-    // ---------------------------------------------------------------- 16-bit loads
-    // Step u's tokens go to ring stages (u % B) * SB .. + SB - 1, which step
-    // u - B used: its P V must have completed, which also frees S buffer
-    // u % B, so the signal that step u's K and V have landed (`convf`) is
-    // all that S of step u waits for.  Staging warp w < NW loads the steps
-    // u = w mod NW, one at a time (copy, wait for its own copies, then
-    // signal), so that the step buffers refill independently of each other;
-    // every buffer has one loading warp, which therefore never waits on a
-    // buffer's barrier more than one phase ahead.  Lane l moves 16-byte
-    // chunks l, l + 32, ... of the step's T rows (consecutive lanes:
-    // consecutive chunks of a row).
-    static_assert(C::kFp8 || C::NS == SB * B, "16-bit: one ring stage group per step buffer");
-    constexpr int CH = C::ROW_BYTES / 16;  // 16-byte chunks per row
-    constexpr int PER = T * CH / 32;       // chunks per lane per tensor and step
-    static_assert(T * CH % 32 == 0 && SB <= 32, "whole chunks per lane");
-    constexpr int NW = B < 4 ? B : 4;  // loading warps
-    static_assert(B % NW == 0, "each step buffer has one loading warp");
+  if (warp >= 4 && warp < 8) {
+    // ---------------------------------------------------------------- loads, S
+    // Step u (tokens u*T .. u*T+T-1 of the range) uses step buffer cb = u % B
+    // (its K and V operands in shared memory, its S and P in TMEM), which
+    // step u - B used: that step's P V must have completed.  Loading warp
+    // w < NW takes the steps u = w mod NW, one at a time: it fills the
+    // step's K and V operands, waits for its own copies, and its lane 0
+    // issues the step's S (one thread issues a tcgen05.mma only every ~80
+    // cycles, so the steps' S come from NW threads).  The buffers thus
+    // refill independently of each other; every buffer has one loading warp,
+    // which therefore never waits on a barrier more than one phase ahead.
+    // Lane l moves the cache's 16-byte chunks l, l + 32, ... of the step's T
+    // rows (consecutive lanes: consecutive chunks of a row):
+    //   16-bit: straight into the operand (cp.async);
+    //   fp8: into the warp's raw staging slot (cp.async), as soon as the
+    //   warp has converted its previous step, so that the fetch overlaps the
+    //   wait for the step's buffer; then converted to f16 (exact) into the
+    //   operand.
+    // V rows past the valid keys become zeros (P is 0 there, and 0 * garbage
+    // could be NaN); so do the K rows of blocks past the range (masked).
+    constexpr int PER = T * CH / 32;  // chunks per lane per tensor and step
+    static_assert(T * CH % 32 == 0, "whole chunks per lane");
+    constexpr uint32_t idS = umma_idesc_f16(kPrefixRows, T, C::kBf16);
+    const uint32_t qa = base + C::OFF_Q;
     const int w = warp - 4;
     // block-table entries of a step: lane j < SB holds block u * SB + j
     auto table_entry = [&](int u) -> int {
@@ -349,178 +270,141 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
       return phys;
     };
     int entry = w < NW && w < nsteps ? table_entry(w) : 0;
-#pragma unroll 1
-    for (int u = w; w < NW && u < nsteps; u += NW) {
-      if (u >= B && !wait_all(pvdone0 + 8 * (u % B), ((u - B) / B) & 1)) break;  // step u - B's stages are free
-      const int cb = u % B;
+    // fp8: step u's K rows (blocks of the range) and V rows (valid tokens)
+    // into this warp's raw staging slot, cache layout; lane l: chunks l, l + 32, ...
+    auto fetch_raw = [&](int u) {
+      const uint32_t raw = base + C::OFF_RAW + w * C::RAW_BYTES;
 #pragma unroll
-      for (int k = 0; k < PER; ++k) {
-        const int c = lane + 32 * k;
-        const int row = c / CH, cc = c % CH;  // token u * T + row of the range, 16-byte chunk cc
-        const int j = row / kBS, r = row % kBS;
+      for (int kq = 0; kq < 2 * PER; ++kq) {
+        const int which = kq >= PER, c = lane + 32 * (kq - which * PER);
+        const int row = c / CH, cc = c % CH, j = row / kBS, r = row % kBS;
         const int phys = __shfl_sync(0xffffffffu, entry, j);
-        const uint32_t off = C::ring(cb * SB + j, r, 16 * cc);
         const size_t src = ((size_t)phys * kBS + r) * job.row_stride + 16 * cc;
-        // K rows of blocks past the range keep older contents: their scores are masked
-        if (u * SB + j < nb)
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(base + C::OFF_RING_K + off),
-                       "l"(job.k_head + src) : "memory");
-        if (u * T + row < job.kv_valid)
-          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(base + C::OFF_RING_V + off),
-                       "l"(job.v_head + src) : "memory");
-        else  // P is 0 there, and 0 * garbage could be NaN
-          asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(base + C::OFF_RING_V + off), "r"(0u)
-                       : "memory");
+        const bool have = which ? u * T + row < job.kv_valid : u * SB + j < nb;
+        if (have)
+          asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(raw + which * (T * C::ROW_BYTES) +
+                                                                      row * C::ROW_BYTES + 16 * cc),
+                       "l"((which ? job.v_head : job.k_head) + src) : "memory");
       }
       asm volatile("cp.async.commit_group;" ::: "memory");
-      if (u + NW < nsteps) entry = table_entry(u + NW);  // (in flight while the copies land)
-      asm volatile("cp.async.wait_group 0;" ::: "memory");
-      fence_proxy_async_smem();  // -> visible to the tensor core
-      __syncwarp();
-      if (lane == 0) mbar_arrive(convf0 + 8 * cb);
-    }
-    asm volatile("cp.async.wait_all;" ::: "memory");  // nothing in flight when the CTA exits
-  } else if (warp >= 4 && warp < 8) {
-    // ---------------------------------------------------------------- fp8 operand staging
-    // Convert each block's K and V rows to f16 (row for row, 128-byte
-    // swizzled, the step's SB blocks stacked) and release the ring stage.
+    };
     if constexpr (C::kFp8) {
-    const int t = threadIdx.x - 128;
-    for (int u = 0; u < nsteps; ++u) {
-      const int cb = u % B;
-      if (u >= B && !wait_all(pvdone0 + 8 * cb, ((u - B) / B) & 1)) break;  // step u - B's operands are free
-      bool stop = false;
+      if (w < NW && w < nsteps) {
+        fetch_raw(w);
+        if (w + NW < nsteps) entry = table_entry(w + NW);
+      }
+    }
 #pragma unroll 1
-      for (int j = 0; j < SB; ++j) {
-        const int i = u * SB + j;  // block of the range
-        const int st = i % NS;
-        const int valid = min(kBS, max(0, job.kv_valid - i * kBS));  // tokens of this block that exist
-        if (i < nb && !wait_all(full0 + 8 * st, (i / NS) & 1)) {
-          stop = true;
-          break;
+    for (int u = w; w < NW && u < nsteps; u += NW) {
+      const int cb = u % B;
+      if (u >= B && !wait_all(pvdone0 + 8 * cb, ((u - B) / B) & 1)) break;  // step u - B is done with the buffer
+      const uint32_t kbuf = base + C::OFF_K + cb * C::BUF_BYTES, vbuf = base + C::OFF_V + cb * C::BUF_BYTES;
+      if constexpr (!C::kFp8) {
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+          const int c = lane + 32 * k;
+          const int row = c / CH, cc = c % CH;  // token u * T + row of the range, 16-byte chunk cc
+          const int j = row / kBS, r = row % kBS;
+          const int phys = __shfl_sync(0xffffffffu, entry, j);
+          const uint32_t off = C::sw128(T, row, 16 * cc);
+          const size_t src = ((size_t)phys * kBS + r) * job.row_stride + 16 * cc;
+          if (u * SB + j < nb)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(kbuf + off), "l"(job.k_head + src)
+                         : "memory");
+          else
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(kbuf + off), "r"(0u) : "memory");
+          if (u * T + row < job.kv_valid)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(vbuf + off), "l"(job.v_head + src)
+                         : "memory");
+          else
+            asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vbuf + off), "r"(0u) : "memory");
         }
-        {
-          uint8_t* kf = smem + C::OFF_KF + cb * C::F_BYTES;
-          uint8_t* vf = smem + C::OFF_VF + cb * C::F_BYTES;
-          for (int k = t; k < 2 * kBS * (D / 16); k += 128) {  // (K|V, row, 16 codes) -> 16 halves
-            const int which = k / (kBS * (D / 16));
-            const int kk = k - which * (kBS * (D / 16));
-            const int r = kk / (D / 16), cc = kk - r * (D / 16);
-            uint32_t h[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-            if (i < nb && (which == 0 || r < valid)) {
-              const uint4 v = lds128(base + (which ? C::OFF_RING_V : C::OFF_RING_K) + C::ring(st, r, 16 * cc));
-              e4m3x4_to_f16x2x2(v.x, h[0], h[1]);
-              e4m3x4_to_f16x2x2(v.y, h[2], h[3]);
-              e4m3x4_to_f16x2x2(v.z, h[4], h[5]);
-              e4m3x4_to_f16x2x2(v.w, h[6], h[7]);
-            }
-            uint8_t* dst = which ? vf : kf;
-            *reinterpret_cast<uint4*>(dst + C::sw128(T, 16 * j + r, 32 * cc)) = make_uint4(h[0], h[1], h[2], h[3]);
-            *reinterpret_cast<uint4*>(dst + C::sw128(T, 16 * j + r, 32 * cc + 16)) = make_uint4(h[4], h[5], h[6], h[7]);
+        asm volatile("cp.async.commit_group;" ::: "memory");
+        if (u + NW < nsteps) entry = table_entry(u + NW);  // (in flight while the copies land)
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+      } else {
+        // the step's raw rows were fetched into this warp's staging slot ahead of time
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        const uint32_t raw = base + C::OFF_RAW + w * C::RAW_BYTES;
+        // chunks read in batches of up to 16 (independent loads in flight), then converted and stored
+        constexpr int NB = 2 * PER < 16 ? 2 * PER : 16;
+        static_assert((2 * PER) % NB == 0, "whole batches");
+#pragma unroll
+        for (int b0 = 0; b0 < 2 * PER; b0 += NB) {
+          uint4 v[NB];
+#pragma unroll
+          for (int q = 0; q < NB; ++q) {
+            const int kq = b0 + q, which = kq >= PER, c = lane + 32 * (kq - which * PER);
+            const int row = c / CH, cc = c % CH;
+            v[q] = lds128(raw + which * (T * C::ROW_BYTES) + row * C::ROW_BYTES + 16 * cc);
           }
-          if (i < nb) {
-            fence_proxy_async_smem();  // (the ring stage's next writer is TMA)
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty0 + 8 * st);
-            if (t == 0) *converted = i + 1;
+#pragma unroll
+          for (int q = 0; q < NB; ++q) {
+            const int kq = b0 + q, which = kq >= PER, c = lane + 32 * (kq - which * PER);
+            const int row = c / CH, cc = c % CH, j = row / kBS;
+            const bool have = which ? u * T + row < job.kv_valid : u * SB + j < nb;
+            uint32_t h[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+            if (have) {
+              e4m3x4_to_f16x2x2(v[q].x, h[0], h[1]);
+              e4m3x4_to_f16x2x2(v[q].y, h[2], h[3]);
+              e4m3x4_to_f16x2x2(v[q].z, h[4], h[5]);
+              e4m3x4_to_f16x2x2(v[q].w, h[6], h[7]);
+            }
+            const uint32_t dst = which ? vbuf : kbuf;
+            sts128(dst + C::sw128(T, row, 32 * cc), make_uint4(h[0], h[1], h[2], h[3]));
+            sts128(dst + C::sw128(T, row, 32 * cc + 16), make_uint4(h[4], h[5], h[6], h[7]));
           }
         }
       }
-      if (stop) break;
-      fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+      fence_proxy_async_smem();  // this lane's operand writes -> visible to the tensor core
       __syncwarp();
-      if (lane == 0) mbar_arrive(convf0 + 8 * cb);
-    }
-    }
-  } else if (warp == 9 && !C::kFp8) {
-    // ---------------------------------------------------------------- 16-bit: S issue
-    // S = Q K^T for each step once its K and V have landed; the loading
-    // warp refilled the step's stages only after the P V of the step that
-    // last used them (and its S buffer) had completed.  (P V is issued by
-    // warp 8: one thread issues a tcgen05.mma every ~80 cycles at best, so
-    // the two streams of MMAs come from two threads.)
-    if (lane == 0) {
-      constexpr uint32_t idS = umma_idesc_f16(kPrefixRows, T, C::kBf16);
-      const uint32_t qa = base + C::OFF_Q;
-#pragma unroll 1
-      for (int u = 0; u < nsteps; ++u) {
-        const int cb = u % B;
-        if (!wait(convf0 + 8 * cb, (u / B) & 1)) break;
+      if (lane == 0) {  // S = Q K^T of step u into S buffer cb, over 16-wide slices of D
         tc_fence_after();
-        const uint32_t kb = base + C::OFF_RING_K + cb * SB * (kBS * 128);
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {  // 16-wide slices of D
+        for (int k = 0; k < D / 16; ++k) {
           const uint64_t a = umma_desc(qa + (k >> 2) * (kPrefixRows * 128) + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
-          const uint64_t b = umma_desc(kb + (k >> 2) * C::RING_SUB + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
+          const uint64_t b = umma_desc(kbuf + (k >> 2) * C::BUF_SUB + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
           umma_f16(tmem + C::S_COL + cb * T, a, b, idS, k > 0);
         }
         umma_commit(sfull0 + 8 * cb);
       }
-      umma_commit(fin);
-      mbar_wait(fin, 0);
-    }
-  } else if (warp == 9) {
-    // ---------------------------------------------------------------- fp8: MMA issue
-    if (lane == 0) {
-      constexpr uint32_t idS = umma_idesc_f16(kPrefixRows, T, C::kBf16);
-      constexpr uint32_t idO = umma_idesc_f16(kPrefixRows, D, C::kBf16, /*b_mn_major=*/true);
-      const uint32_t qa = base + C::OFF_Q;
-      // Issue S for a step as soon as its operands are staged (at most B
-      // steps ahead of the softmax), and O += P V as soon as the softmax has
-      // written that step's P: both polled without blocking.
-      int ns_ = 0, npv = 0;
-      long long idle_since = clock64();
-      while (npv < nsteps && !*dead) {
-        bool progress = false;
-        if (ns_ < nsteps && ns_ - npv < B && mbar_test_wait(convf0 + 8 * (ns_ % B), (ns_ / B) & 1)) {
-          tc_fence_after();
-          const int cb = ns_ % B;
-          // K operand: the f16 copy (fp8) or the ring stages of the step (16-bit)
-          const uint32_t kb = C::kFp8 ? base + C::OFF_KF + cb * C::F_BYTES
-                                      : base + C::OFF_RING_K + ((ns_ * SB) % NS) * (kBS * 128);
-          constexpr int KSUB = C::kFp8 ? T * 128 : C::RING_SUB;  // bytes between 64-dim sub-tiles
-#pragma unroll
-          for (int k = 0; k < D / 16; ++k) {  // S = Q K^T over 16-wide slices of D
-            const uint64_t a = umma_desc(qa + (k >> 2) * (kPrefixRows * 128) + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
-            const uint64_t b = umma_desc(kb + (k >> 2) * KSUB + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
-            umma_f16(tmem + C::S_COL + cb * T, a, b, idS, k > 0);
-          }
-          umma_commit(sfull0 + 8 * cb);
-          ++ns_;
-          progress = true;
-        }
-        if (npv < ns_ && mbar_test_wait(pfull0 + 8 * (npv % B), (npv / B) & 1)) {
-          tc_fence_after();
-          const int cb = npv % B;
-          const uint32_t pt = tmem + C::S_COL + cb * T;  // P: T/2 columns of 16-bit pairs
-          // V operand, MN-major (dims contiguous in 128-byte rows, one row per
-          // token): the f16 copy (fp8) or the ring stages of the step (16-bit)
-          const uint32_t va = C::kFp8 ? base + C::OFF_VF + cb * C::F_BYTES
-                                      : base + C::OFF_RING_V + ((npv * SB) % NS) * (kBS * 128);
-          constexpr int VSUB = C::kFp8 ? T * 128 : C::RING_SUB;  // bytes between 64-dim sub-tiles
-#pragma unroll
-          for (int k = 0; k < T / 16; ++k) {  // O += P V over 16-token slices (one block each)
-            const uint64_t b = umma_desc(va + k * (kBS * 128), VSUB, 1024, kUmmaSwizzle128);
-            umma_f16_ts(tmem + C::O_COL, pt + 8 * k, b, idO, (npv > 0 || k > 0) ? 1 : 0);
-          }
-          umma_commit(pvdone0 + 8 * cb);  // (16-bit: the step's ring stages are free once it arrives)
-          ++npv;
-          progress = true;
-        }
-        if (progress) {
-          idle_since = clock64();
-        } else if (clock64() - idle_since > kWaitLimitCycles) {
-          atomicOr(err, kCheckWaitTimeout);
-          *dead = 1;
-        } else {
-          __nanosleep(32);  // (leave the issue slots to the softmax warp sharing this scheduler)
+      if constexpr (C::kFp8) {  // this warp's next step: its raw rows land while that step waits for its buffer
+        if (u + NW < nsteps) {
+          fetch_raw(u + NW);
+          if (u + 2 * NW < nsteps) entry = table_entry(u + 2 * NW);
         }
       }
-      // every MMA issued has completed before the CTA releases tensor memory
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // nothing in flight when the CTA exits
+    if (w < NW && lane == 0) {  // every MMA this thread issued has completed before tensor memory is released
       umma_commit(fin);
       mbar_wait(fin, 0);
     }
-  } else {
+  } else if (warp == 8) {
+    // ---------------------------------------------------------------- P V issue
+    // O += P V for each step once the softmax has written its P (P read
+    // from tensor memory as the A operand, V MN-major from the step's
+    // buffer); the commit frees the step buffer.
+    if (lane == 0) {
+      constexpr uint32_t idO = umma_idesc_f16(kPrefixRows, D, C::kBf16, /*b_mn_major=*/true);
+#pragma unroll 1
+      for (int u = 0; u < nsteps; ++u) {
+        const int cb = u % B;
+        if (!wait(pfull0 + 8 * cb, (u / B) & 1)) break;
+        tc_fence_after();
+        const uint32_t pt = tmem + C::S_COL + cb * T;
+        const uint32_t va = base + C::OFF_V + cb * C::BUF_BYTES;
+#pragma unroll
+        for (int k = 0; k < T / 16; ++k) {  // 16-token slices (one block each)
+          const uint64_t b = umma_desc(va + k * (kBS * 128), C::BUF_SUB, 1024, kUmmaSwizzle128);
+          umma_f16_ts(tmem + C::O_COL, pt + 8 * k, b, idO, (u > 0 || k > 0) ? 1 : 0);
+        }
+        umma_commit(pvdone0 + 8 * cb);
+      }
+      umma_commit(fin);  // every MMA this thread issued has completed before tensor memory is released
+      mbar_wait(fin, 0);
+    }
+  } else if (warp < 4) {
     // ---------------------------------------------------------------- softmax (warps 0..3)
     const int r = threadIdx.x;
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
@@ -631,8 +515,8 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
     }
   }
 
-  // ---- tear-down: every tcgen05 operation has completed (the MMA thread
-  // waited for its last commit; loads were waited for); release TMEM
+  // ---- tear-down: every tcgen05 operation has completed (the MMA-issuing
+  // threads waited for their last commits; loads were waited for); release TMEM
   tc_fence_before();
   __syncthreads();
   if (warp == 0) {
@@ -643,8 +527,7 @@ __device__ __forceinline__ void stacked_attention(const CUtensorMap& tmK, const 
 
 template <class C>
 __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
-    paged_prefix_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
-                        const PrefixParams p) {
+    paged_prefix_kernel(const PrefixParams p) {
   using Q = typename C::Q;
   constexpr int D = C::D;
 
@@ -738,10 +621,10 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
   };
   const Rows rw{&p, rb, rows, first, hpu, head0, chunk};
   const size_t row_stride = (size_t)(p.num_heads / p.group) * C::ROW_BYTES;
-  const StackedJob job{p.block_tables + (size_t)first * p.bt_stride + b0, nb, nb * kBS, kvh, p.num_blocks,
+  const StackedJob job{p.block_tables + (size_t)first * p.bt_stride + b0, nb, nb * kBS, p.num_blocks,
                        static_cast<const uint8_t*>(p.k_cache) + (size_t)kvh * C::ROW_BYTES,
                        static_cast<const uint8_t*>(p.v_cache) + (size_t)kvh * C::ROW_BYTES, row_stride};
-  stacked_attention<C>(tmK, tmV, job, rw, p.scale_log2, p.v_scale, p.err);
+  stacked_attention<C>(job, rw, p.scale_log2, p.v_scale, p.err);
 }
 
 }  // namespace pa
