@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(C::THREADS, C::REG_CTAS)
   constexpr int D = C::D;
   const int s = blockIdx.z;
   const int y = blockIdx.y;
-  const int rb = blockIdx.x;
+  const int rb = gridDim.x - 1 - blockIdx.x;  // a sequence's row blocks heaviest (most keys) first
   const int kvh = y / p.head_splits;
   const int hs = y - kvh * p.head_splits;
   const int head0 = kvh * p.group + hs * kNH;

@@ -447,7 +447,7 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
       for (int ch = NCH - 1; ch >= 0; --ch) {
         load(ch);
 #pragma unroll
-        for (int j = 0; j < TC; ++j) mx[j & 3] = fmaxf(mx[j & 3], x[j]);
+        for (int j = 0; j < TC; j += 2) mx[(j >> 1) & 3] = max3f(mx[(j >> 1) & 3], x[j], x[j + 1]);
       }
       const float bm = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * xs;
       // lazy rescaling: move the reference max (and rescale l, O) only when
@@ -475,7 +475,7 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
       // buffer: chunk ch's P goes to columns ch * TC / 2 .., which held
       // scores of chunk ch / 2 <= ch, already read.  It is the A operand of
       // the step's P V; the buffer's next S is issued only after that P V.
-      float sm[4] = {0.f, 0.f, 0.f, 0.f};  // four independent sum chains
+      float2 sm[2] = {{0.f, 0.f}, {0.f, 0.f}};  // four independent sum chains, two per instruction
 #pragma unroll
       for (int ch = 0; ch < NCH; ++ch) {
         if (ch > 0) load(ch);
@@ -483,15 +483,17 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
         for (int c0 = 0; c0 < TC / 2; c0 += 16) {
           uint32_t pk[16];
 #pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const float p0 = ex2(fmaf(x[2 * (c0 + q)], xs, -m)), p1 = ex2(fmaf(x[2 * (c0 + q) + 1], xs, -m));
-            sm[q & 3] += p0 + p1;
-            pk[q] = pack2<C::kBf16>(p0, p1);
+          for (int q = 0; q < 16; ++q) {  // keys 2(c0+q), 2(c0+q)+1: exponents two per instruction
+            const float2 e = fma2(make_float2(x[2 * (c0 + q)], x[2 * (c0 + q) + 1]), make_float2(xs, xs),
+                                  make_float2(-m, -m));
+            const float2 pp = make_float2(ex2(e.x), ex2(e.y));
+            sm[q & 1] = add2(sm[q & 1], pp);
+            pk[q] = pack2<C::kBf16>(pp.x, pp.y);
           }
           tmem_st16(trow + C::S_COL + cb * T + ch * (TC / 2) + c0, pk);
         }
       }
-      l += (sm[0] + sm[1]) + (sm[2] + sm[3]);
+      l += (sm[0].x + sm[1].x) + (sm[0].y + sm[1].y);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
