@@ -109,8 +109,8 @@ struct PrefixCfg {
   static constexpr int RAW_BYTES = kFp8 ? 2 * T * ROW_BYTES : 0;
   static constexpr int OFF_RAW = OFF_V + B * BUF_BYTES;  // [NW]
   static constexpr int OFF_BAR = OFF_RAW + NW * RAW_BYTES;
-  // s_full[B] p_full[B] pv_done[B] fin
-  static constexpr int NBARS = 3 * B + 1;
+  // s_full[B] p_full[B] pv_done[B] fin q_ready
+  static constexpr int NBARS = 3 * B + 2;
   static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;  // tmem base, dead flag
   static constexpr int TMEM_COLS = D + B * T <= 128 ? 128 : (D + B * T <= 256 ? 256 : 512);
   // O: D columns; S buffers: T columns each, a step's P over the first T/2 of its buffer
@@ -176,14 +176,17 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
   extern __shared__ uint8_t smem_dyn[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~uintptr_t(1023));
   const uint32_t base = smem_u32(smem);
-  const uint32_t sfull0 = base + C::OFF_BAR, pfull0 = sfull0 + 8 * B, pvdone0 = pfull0 + 8 * B, fin = pvdone0 + 8 * B;
+  const uint32_t sfull0 = base + C::OFF_BAR, pfull0 = sfull0 + 8 * B, pvdone0 = pfull0 + 8 * B, fin = pvdone0 + 8 * B,
+                 qready = fin + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* dead = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nb = job.nb;
   const int nsteps = (nb + SB - 1) / SB;
 
-  // ---- set-up: barriers, tensor memory, the query tile (128-byte swizzled)
+  // ---- set-up: barriers, tensor memory, the query tile (128-byte swizzled):
+  // its copies are in flight while the loading warps start on the first
+  // steps' K and V; only the first S waits for it
   if (threadIdx.x == 0) {
     for (int i = 0; i < B; ++i) {
       mbar_init(sfull0 + 8 * i, 1);  // tcgen05.commit after the step's S
@@ -191,6 +194,7 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
       mbar_init(pvdone0 + 8 * i, 1);  // tcgen05.commit after the step's P V
     }
     mbar_init(fin, 1 + NW);  // the MMA-issuing threads: the loading warps' (S) and warp 8's (P V)
+    mbar_init(qready, 4);    // the query tile has landed (the four softmax warps' rows)
     *dead = 0;
     fence_mbar_init();
   }
@@ -206,13 +210,18 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
       else
         asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(dst), "r"(0u) : "memory");
     }
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-    fence_proxy_async_smem();
+    asm volatile("cp.async.commit_group;" ::: "memory");
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  if (warp < 4) {  // (barrier initialisation is visible to every thread by now)
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    fence_proxy_async_smem();  // this thread's query row -> visible to the tensor core
+    __syncwarp();
+    if (lane == 0) mbar_arrive(qready);
+  }
 
   // A failed (timed-out) wait marks the CTA dead: every role then stops at
   // its next wait that does not complete at once.
@@ -270,6 +279,7 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
       return phys;
     };
     int entry = w < NW && w < nsteps ? table_entry(w) : 0;
+    bool q_landed = false;
     // fp8: step u's K rows (blocks of the range) and V rows (valid tokens)
     // into this warp's raw staging slot, cache layout; lane l: chunks l, l + 32, ...
     auto fetch_raw = [&](int u) {
@@ -358,6 +368,10 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
       }
       fence_proxy_async_smem();  // this lane's operand writes -> visible to the tensor core
       __syncwarp();
+      if (!q_landed) {  // the query tile, once
+        if (!wait_all(qready, 0)) break;
+        q_landed = true;
+      }
       if (lane == 0) {  // S = Q K^T of step u into S buffer cb, over 16-wide slices of D
         tc_fence_after();
 #pragma unroll
@@ -503,15 +517,20 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
     if (ok) {
       tc_fence_after();
       const float inv = l > 0.f ? v_scale / l : 0.f;
+      constexpr int OB = D < 64 ? D : 64;  // O columns read per wait
 #pragma unroll 1
-      for (int c0 = 0; c0 < D; c0 += 16) {
-        uint32_t o[16];
-        tmem_ld16(trow + C::O_COL + c0, o);
-        tmem_wait_ld();
-        float v[16];
+      for (int c0 = 0; c0 < D; c0 += OB) {
+        uint32_t o[OB / 16][16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(o[j]) * inv;
-        rows.store(r, c0, v);
+        for (int k = 0; k < OB / 16; ++k) tmem_ld16(trow + C::O_COL + c0 + 16 * k, o[k]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < OB / 16; ++k) {
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(o[k][j]) * inv;
+          rows.store(r, c0 + 16 * k, v);
+        }
       }
       rows.store_ml(r, m, l);
     }
