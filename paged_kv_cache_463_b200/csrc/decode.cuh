@@ -526,17 +526,30 @@ __device__ __forceinline__ HandOut decode_hand_out(const DecodeParams& p, int* p
   bool bad = false;
   long long sum_len = 0;
   int min_len = 0x7fffffff, max_len = 0;
-  for (int b = 0; b < S; b += 32) {
-    const int s = b + lane;
-    if (s < S) {
-      const int raw = p.seq_lens[s];
-      int len = clamp_len(raw, p);
-      bad |= raw != len;
-      if (p.seq_skip) len = max(0, len - p.seq_skip[s] * kBS);  // the private suffix
-      lens[s] = len;
-      sum_len += len;
-      min_len = min(min_len, len);
-      max_len = max(max_len, len);
+  // The lengths (and suffix offsets) of up to 256 sequences are loaded
+  // before any is stored to shared memory: loads queued behind each chunk's
+  // stores would cost one memory round trip per 32 sequences.
+  constexpr int HB = 8;
+  for (int b0 = 0; b0 < S; b0 += 32 * HB) {
+    int raw[HB], skip[HB];
+#pragma unroll
+    for (int k = 0; k < HB; ++k) {
+      const int s = b0 + 32 * k + lane;
+      raw[k] = s < S ? __ldg(p.seq_lens + s) : 0;
+      skip[k] = (p.seq_skip && s < S) ? __ldg(p.seq_skip + s) : 0;
+    }
+#pragma unroll
+    for (int k = 0; k < HB; ++k) {
+      const int s = b0 + 32 * k + lane;
+      if (s < S) {
+        int len = clamp_len(raw[k], p);
+        bad |= raw[k] != len;
+        if (p.seq_skip) len = max(0, len - skip[k] * kBS);  // the private suffix
+        lens[s] = len;
+        sum_len += len;
+        min_len = min(min_len, len);
+        max_len = max(max_len, len);
+      }
     }
   }
 #pragma unroll
@@ -551,28 +564,41 @@ __device__ __forceinline__ HandOut decode_hand_out(const DecodeParams& p, int* p
     if (!sk) pb = uniform_partition_blocks(p, sum_len, max_len, gridDim.x);
   }
   __syncwarp();
+  // exclusive prefix of the per-sequence counts: 8 chunks of 32 scanned side
+  // by side (independent shuffle chains), then chained by their totals
   int carry = 0;
-  for (int b = 0; b < S; b += 32) {
-    const int s = b + lane;
-    int n = 0;
-    if (s < S) {
-      const int len = lens[s];
-      const int nblk = (len + kBS - 1) / kBS;
-      if (sk) {
-        n = nblk;
-      } else {
-        bad |= (nblk + pb - 1) / pb > p.max_parts;
-        n = max(1, num_partitions(len, pb, p)) * p.kv_units;
+  for (int b0 = 0; b0 < S; b0 += 32 * HB) {
+    int x[HB];
+#pragma unroll
+    for (int k = 0; k < HB; ++k) {
+      const int s = b0 + 32 * k + lane;
+      int n = 0;
+      if (s < S) {
+        const int len = lens[s];
+        const int nblk = (len + kBS - 1) / kBS;
+        if (sk) {
+          n = nblk;
+        } else {
+          bad |= (nblk + pb - 1) / pb > p.max_parts;
+          n = max(1, num_partitions(len, pb, p)) * p.kv_units;
+        }
       }
+      x[k] = n;
     }
-    int x = n;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const int y = __shfl_up_sync(0xffffffffu, x, off);
-      if (lane >= off) x += y;
+#pragma unroll
+      for (int k = 0; k < HB; ++k) {
+        const int y = __shfl_up_sync(0xffffffffu, x[k], off);
+        if (lane >= off) x[k] += y;
+      }
     }
-    if (s < S) prefix[s + 1] = carry + x;
-    carry += __shfl_sync(0xffffffffu, x, 31);
+#pragma unroll
+    for (int k = 0; k < HB; ++k) {
+      const int s = b0 + 32 * k + lane;
+      if (s < S) prefix[s + 1] = carry + x[k];
+      carry += __shfl_sync(0xffffffffu, x[k], 31);
+    }
   }
   if (lane == 0) prefix[0] = 0;
   if (blockIdx.x == 0 && __any_sync(0xffffffffu, bad) && lane == 0) atomicOr(p.err, kCheckSeqTooLong);
