@@ -82,6 +82,7 @@ struct DecodeParams {
   int q_slot_bytes; // min(group, 8) * head_dim * 2: one item's query rows
   int merge_hpc;    // merge kernel: query heads per CTA
   int merge_slices; // merge kernel: partition slices per head
+  int merge_hpt;    // merge kernel: heads per thread (2 only with one slice)
   float scale_log2;  // softmax scale * log2(e) (* k_scale for fp8)
   float v_scale;     // 1, or the fp8 value scale
   // shared-prefix decode (all null / 0 otherwise): the prefix pass covered the
@@ -1098,6 +1099,56 @@ __global__ void __launch_bounds__(256, 4) paged_decode_merge_kernel(const Decode
   };
   const int c = threadIdx.x % CH;
   const int rest = threadIdx.x / CH;
+  // fold a summary (m, w, a4), w = sum l 2^(m_q - m) and a4 = sum l 2^(m_q - m) o_q, into (M, W, acc)
+  auto fold = [](float& M, float& W, float4& acc, float m, float w, const float4& a4) {
+    if (!(w > 0.f)) return;
+    const float mn = fmaxf(M, m);
+    const float a = ex2(M - mn), b = ex2(m - mn);
+    acc.x = fmaf(b, a4.x, acc.x * a);
+    acc.y = fmaf(b, a4.y, acc.y * a);
+    acc.z = fmaf(b, a4.z, acc.z * a);
+    acc.w = fmaf(b, a4.w, acc.w * a);
+    W = fmaf(W, a, w * b);
+    M = mn;
+  };
+  auto write = [&](int h, const float4& acc, float W) {
+    const float inv = W > 0.f ? 1.f / W : 0.f;  // no weighted partial: a zero row
+    Q* dst = reinterpret_cast<Q*>(p.out) + ((size_t)s * p.num_heads + h) * D + 4 * c;
+    *reinterpret_cast<uint2*>(dst) = make_uint2(pack2<BF16>(acc.x * inv, acc.y * inv), pack2<BF16>(acc.z * inv, acc.w * inv));
+  };
+  if (p.merge_hpt == 2) {
+    // one slice, two heads per thread (rest and rest + hpass of the CTA's
+    // heads): both heads' partial loads in flight together, two partials of
+    // each per batch
+    const int hpass = (int)blockDim.x / CH;
+    const int ha = h0 + rest, hb = h0 + rest + hpass;
+    const bool aa = rest < hpc && ha < p.num_heads, ab = rest + hpass < hpc && hb < p.num_heads;
+    float Ma = -INFINITY, Wa = 0.f, Mb = -INFINITY, Wb = 0.f;
+    float4 acca = make_float4(0.f, 0.f, 0.f, 0.f), accb = acca;
+    for (int q0 = 0; q0 < nt; q0 += 2) {
+      float2 mlq[4];
+      float4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {  // u: (head b?, partial q0 + (u & 1))
+        const int q = q0 + (u & 1);
+        const bool isb = u >> 1;
+        const bool ok = q < nt && (isb ? ab : aa);
+        const int hh = isb ? hb : ha;
+        mlq[u] = ok ? *reinterpret_cast<const float2*>(ml_of(hh, q)) : make_float2(-INFINITY, 0.f);
+        v[u] = ok ? *reinterpret_cast<const float4*>(o_of(hh, q) + 4 * c) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {  // a partial (o, m, l) is the summary (m, l, l o)
+        const float l = mlq[u].y;
+        const float4 a4 = make_float4(l * v[u].x, l * v[u].y, l * v[u].z, l * v[u].w);
+        if (u >> 1) fold(Mb, Wb, accb, mlq[u].x, l, a4);
+        else fold(Ma, Wa, acca, mlq[u].x, l, a4);
+      }
+    }
+    if (aa) write(ha, acca, Wa);
+    if (ab) write(hb, accb, Wb);
+    return;
+  }
   const int slice = rest % slices, hl = rest / slices;
   const int h = h0 + hl;
   const bool active = hl < hpc && h < p.num_heads;
@@ -1144,11 +1195,7 @@ __global__ void __launch_bounds__(256, 4) paged_decode_merge_kernel(const Decode
       }
     }
   }
-  if (slice == 0 && active) {
-    const float inv = W > 0.f ? 1.f / W : 0.f;  // no weighted partial: a zero row
-    Q* dst = reinterpret_cast<Q*>(p.out) + ((size_t)s * p.num_heads + h) * D + 4 * c;
-    *reinterpret_cast<uint2*>(dst) = make_uint2(pack2<BF16>(acc.x * inv, acc.y * inv), pack2<BF16>(acc.z * inv, acc.w * inv));
-  }
+  if (slice == 0 && active) write(h, acc, W);
 }
 
 }  // namespace pa

@@ -124,7 +124,7 @@ cudaError_t pin_all_carveouts(const KernelSet& ks) {
 // wait (griddepcontrol.wait) for the decode grid before reading partials.
 // Merge CTA shape: more partitions -> more partition slices per head, fewer
 // heads per CTA (256 threads = heads x slices x head_dim/4 chunks).
-void merge_shape(int head_dim, int parts, int num_heads, int* hpc, int* slices) {
+void merge_shape(int head_dim, int parts, int num_heads, int* hpc, int* slices, int* hpt) {
   const int ch = head_dim / 4;
   int sl = 1;
   while (sl < 8 && sl * 16 <= parts) sl *= 2;  // <= 15 partitions: 1 slice, ... , >= 128: 8
@@ -133,8 +133,12 @@ void merge_shape(int head_dim, int parts, int num_heads, int* hpc, int* slices) 
   if (h > pa::kNH) h = pa::kNH;
   if (h > num_heads) h = num_heads;
   if (h < 1) h = 1;
-  *hpc = h;
+  // one slice and many heads: two heads per thread (half the CTAs: a large
+  // batch's merge in one wave instead of two)
+  const int t = (sl == 1 && h == 256 / ch && num_heads >= 2 * h) ? 2 : 1;
+  *hpc = h * t;
   *slices = sl;
+  *hpt = t;
 }
 
 cudaError_t launch_merge(const KernelSet& ks, const pa::DecodeParams& p, cudaStream_t s) {
@@ -726,7 +730,7 @@ int decode_impl(pa_ctx* ctx, void* out, const void* query, const void* key_cache
     ctx->test_wait_limit = 0;
   }
 
-  merge_shape(c.head_dim, parts + prefix_chunks, c.num_heads, &p.merge_hpc, &p.merge_slices);
+  merge_shape(c.head_dim, parts + prefix_chunks, c.num_heads, &p.merge_hpc, &p.merge_slices, &p.merge_hpt);
   void* args[] = {&mk, &mv, &p};
   cudaError_t e = cudaLaunchKernel(ctx->ks.decode, dim3(ctx->grid), dim3(ctx->ks.threads), args,
                                    ctx->ks.smem(q_slot_bytes(c.num_heads, c.num_kv_heads, c.head_dim), c.max_num_seqs), s);
@@ -1052,7 +1056,7 @@ PA_API int paged_attention_decode_noalloc(void* out, const void* query, const vo
   p.scale_log2 = (float)((double)scale * 1.4426950408889634 * (fp8 ? (double)k_scale : 1.0));
   p.v_scale = fp8 ? v_scale : 1.0f;
 
-  merge_shape(head_dim, parts, num_heads, &p.merge_hpc, &p.merge_slices);
+  merge_shape(head_dim, parts, num_heads, &p.merge_hpc, &p.merge_slices, &p.merge_hpt);
   void* args[] = {&mk, &mv, &p};
   if (cudaLaunchKernel(ks.decode, dim3(num_sms * per_sm), dim3(ks.threads), args, smem, s) != cudaSuccess)
     return PA_ERR_CUDA;
