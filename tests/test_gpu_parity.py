@@ -108,6 +108,23 @@ def test_step_parity_small(name):
     assert_out_close(out, ref, tol, spec.q_dtype, name)
 
 
+@pytest.mark.parametrize("lens", [(1, 300), (160, 160)], ids=["streamk-ragged", "tickets-uniform"])
+def test_step_parity_many_sequences(lens):
+    """More than 256 sequences (the decode kernel's work hand-out reads the
+    lengths 256 at a time): 600 short sequences, ragged (stream-K) and
+    uniform (tickets), every output element against the oracle."""
+    spec = wl.scaled(wl.SPEC_BY_NAME["gqa-70b-like"], num_seqs=600, num_heads=8, num_kv_heads=2, head_dim=64,
+                     seq_len_min=lens[0], seq_len_max=lens[1], pool_blocks=None)
+    w = wl.make_workload(spec, DEV)
+    pa = _ctx(spec, w.num_blocks, w.block_tables.shape[1])
+    kh, vh = raw(w.key_cache), raw(w.value_cache)
+    out = _run_step(pa, w, w.key_cache, w.value_cache)
+    ref, kh2, vh2 = _oracle_full(w, kh, vh)
+    np.testing.assert_array_equal(raw(w.key_cache), kh2)
+    assert_out_close(out, ref, TOL[spec.q_dtype], spec.q_dtype, f"600 seqs {lens}")
+    pa.close()
+
+
 def _sample_pairs(S, H, rng, nseq=6, nh=4):
     seqs = sorted(set([0, S - 1] + rng.choice(S, size=min(S, nseq), replace=False).tolist()))
     heads = sorted(set([0, H - 1] + rng.choice(H, size=min(H, nh), replace=False).tolist()))

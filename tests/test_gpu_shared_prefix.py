@@ -119,6 +119,20 @@ def test_long_prefix_many_rows(q_dtype, kv_dtype, partition):
     assert_out_close(out, _oracle(w, kh, vh), _tol(sp), q_dtype, f"partition={partition}")
 
 
+@pytest.mark.parametrize("q_dtype,kv_dtype", [("f16", "f16"), ("f16", "fp8_e4m3")])
+def test_many_sequences(q_dtype, kv_dtype):
+    """520 sequences in 10 groups (the decode kernel's work hand-out reads the
+    lengths and suffix offsets 256 sequences at a time; the merge folds two
+    heads per thread): every output element against the oracle."""
+    sp = _spec(q_dtype, kv_dtype, 128, 4, 64, num_seqs=520, groups=10, suffix=(0, 100))
+    w = wl.make_workload(sp, DEV)
+    kc, vc, kh, vh = _caches(w)
+    pa = _ctx(sp, w.num_blocks, w.block_tables.shape[1])
+    out, bits = _shared(pa, w, kc, vc)
+    assert bits == 0
+    assert_out_close(out, _oracle(w, kh, vh), _tol(sp), q_dtype, f"520 seqs {q_dtype}/{kv_dtype}")
+
+
 def test_ungrouped_sequences_and_zero_prefix():
     """Sequences before the first group and after the last share nothing, and
     a group may declare a zero-length prefix: all are decoded in full."""
