@@ -11,29 +11,24 @@
 // combines the two sets of (o, m, l) partials by log-sum-exp.
 //
 // With all members' query heads of one KV head stacked, attention over the
-// prefix is a dense contraction: for a step of T tokens (SB blocks),
+// prefix is a dense contraction: for a step of T = 32 tokens (SB = 2 blocks),
 // S[128 rows x T] = Q K^T, then O[128 x D] += P V.  Both run on the
-// 5th-generation tensor cores (tcgen05.mma, issued by one thread,
-// accumulators in tensor memory), one CTA per (group, KV unit, 128 query
-// rows, chunk of 32 prefix blocks).  The core, `stacked_attention`, is shared
-// with the multi-query (prefill) kernel; its roles:
-//   warps 4..7  16-bit caches: copy each step's K and V rows from the cache
-//               into the step's ring stages with 16-byte cp.async (one warp
-//               per step buffer, refilling it as soon as the P V that last
-//               read it completes) and issue the step's S into its TMEM S
-//               buffer once the rows have landed; the rings, laid out sub-tile-
-//               major so that a step's SB stages hold its tokens' rows
-//               contiguously, are themselves the MMA operands (K K-major, V
-//               MN-major); V rows past the valid keys are written as zeros.
-//               fp8 caches: convert each block's K and V rows to f16 once,
-//               into per-step operand buffers;
-//   warp 8      16-bit caches: issues O += P V for a step once the softmax
-//               has written its P (P read from tensor memory as the A
-//               operand).  fp8 caches: TMA producer of the two NS-stage rings
-//               the converting warps read;
-//   warp 9      fp8 caches: issues S for a step into one of B TMEM S buffers
-//               once its operands are ready, and P V, both from one polling
-//               loop;
+// 5th-generation tensor cores (tcgen05.mma, accumulators in tensor memory),
+// one CTA per (group, KV unit, 128 query rows, chunk of 32 prefix blocks).
+// The core, `stacked_attention`, is shared with the multi-query (prefill)
+// kernel.  It keeps B step buffers (a step's K and V operands in shared
+// memory, 128-byte swizzled, K K-major and V MN-major; its S, then P, in
+// tensor memory); its roles:
+//   warps 4..7  one loading warp per step buffer: wait for the P V that last
+//               read the buffer, fill the step's K and V operands from the
+//               cache (16-bit: 16-byte cp.async straight into the operand;
+//               fp8: from the warp's raw staging slot, fetched with cp.async
+//               while it waited, converted to f16), write zero V rows past
+//               the valid keys, and issue the step's S (lane 0; a thread
+//               issues a tcgen05.mma only every ~80 cycles, so the steps' S
+//               come from four threads);
+//   warp 8      issues O += P V for a step once the softmax has written its
+//               P (P read from tensor memory as the A operand);
 //   warps 0..3  one query row per thread: read the step's S row from TMEM,
 //               online softmax in the log2 domain (lazy: O is rescaled in
 //               TMEM only when a row's maximum grows by more than 2^8), write
@@ -96,7 +91,7 @@ struct PrefixCfg {
   static constexpr bool kBf16 = std::is_same<Q, __nv_bfloat16>::value;
   static constexpr int ROW_BYTES = D * (int)sizeof(KV);  // one token's K (or V) row of one KV head in the cache
   static constexpr int CH = ROW_BYTES / 16;               // its 16-byte chunks
-  // Step buffer layout (both K and V, 16-bit operands, TMA-style 128-byte
+  // Step buffer layout (both K and V, 16-bit operands, 128-byte
   // swizzle): [D / 64 sub-tiles][T rows x 128 B], so that a sub-tile is a
   // K-major (K) or MN-major (V) MMA operand with 8-row atoms 1024 bytes apart.
   static constexpr int BUF_SUB = T * 128;          // bytes between a step buffer's sub-tiles
