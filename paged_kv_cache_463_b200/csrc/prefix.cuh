@@ -418,6 +418,7 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
     const int r = threadIdx.x;
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);  // this warp's TMEM lanes
     const int lim = min(rows.limit(r), job.kv_valid);  // keys this row sees, from the range start
+    const int wlim = __reduce_min_sync(0xffffffffu, lim);  // the warp's fewest
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int u = 0; u < nsteps && ok; ++u) {
@@ -434,16 +435,23 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
       // Steps before the diagonal, where every row of the warp sees every key
       // and the scale is positive, take the max of the raw scores and fold
       // the scale into the exponent's FMA; the others scale and mask first.
-      const bool plain = scale_log2 > 0.f && __all_sync(0xffffffffu, valid >= T);
+      const bool plain = scale_log2 > 0.f && wlim >= (u + 1) * T;  // (every row of the warp sees every key)
       const float xs = plain ? scale_log2 : 1.f;  // exponent = x * xs - m
       float x[TC];
       auto load = [&](int ch) {
+        if constexpr (TC == 32) {
+          uint32_t sv[32];
+          tmem_ld32(trow + C::S_COL + cb * T + ch * TC, sv);
 #pragma unroll
-        for (int c0 = 0; c0 < TC; c0 += 16) {
-          uint32_t sv[16];
-          tmem_ld16(trow + C::S_COL + cb * T + ch * TC + c0, sv);
+          for (int j = 0; j < 32; ++j) x[j] = __uint_as_float(sv[j]);
+        } else {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) x[c0 + j] = __uint_as_float(sv[j]);
+          for (int c0 = 0; c0 < TC; c0 += 16) {
+            uint32_t sv[16];
+            tmem_ld16(trow + C::S_COL + cb * T + ch * TC + c0, sv);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) x[c0 + j] = __uint_as_float(sv[j]);
+          }
         }
         tmem_wait_ld();
         if (!plain) {
