@@ -305,12 +305,30 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
       if (u >= B && !wait_all(pvdone0 + 8 * cb, ((u - B) / B) & 1)) break;  // step u - B is done with the buffer
       const uint32_t kbuf = base + C::OFF_K + cb * C::BUF_BYTES, vbuf = base + C::OFF_V + cb * C::BUF_BYTES;
       if constexpr (!C::kFp8) {
+        int ph[SB];  // the step's block ids (one shuffle per block)
+#pragma unroll
+        for (int j = 0; j < SB; ++j) ph[j] = __shfl_sync(0xffffffffu, entry, j);
+        if ((u + 1) * SB <= nb && (u + 1) * T <= job.kv_valid) {
+          // interior step: every block and every row exists
+#pragma unroll
+          for (int k = 0; k < PER; ++k) {
+            const int c = lane + 32 * k;
+            const int row = c / CH, cc = c % CH;
+            const int j = row / kBS, r = row % kBS;
+            const uint32_t off = C::sw128(T, row, 16 * cc);
+            const size_t src = ((size_t)ph[j] * kBS + r) * job.row_stride + 16 * cc;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(kbuf + off), "l"(job.k_head + src)
+                         : "memory");
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(vbuf + off), "l"(job.v_head + src)
+                         : "memory");
+          }
+        } else {
 #pragma unroll
         for (int k = 0; k < PER; ++k) {
           const int c = lane + 32 * k;
           const int row = c / CH, cc = c % CH;  // token u * T + row of the range, 16-byte chunk cc
           const int j = row / kBS, r = row % kBS;
-          const int phys = __shfl_sync(0xffffffffu, entry, j);
+          const int phys = ph[j];
           const uint32_t off = C::sw128(T, row, 16 * cc);
           const size_t src = ((size_t)phys * kBS + r) * job.row_stride + 16 * cc;
           if (u * SB + j < nb)
@@ -323,6 +341,7 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
                          : "memory");
           else
             asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(vbuf + off), "r"(0u) : "memory");
+        }
         }
         asm volatile("cp.async.commit_group;" ::: "memory");
         if (u + NW < nsteps) entry = table_entry(u + NW);  // (in flight while the copies land)
