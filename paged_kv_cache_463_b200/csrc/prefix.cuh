@@ -274,6 +274,20 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
       return phys;
     };
     int entry = w < NW && w < nsteps ? table_entry(w) : 0;
+    // 16-bit interior steps: lane l's chunks k = 0..PER-1 are row lrow + RPK k
+    // of the step, 16-byte chunk lcc of the row (RPK = 32 / CH rows per k, so
+    // chunk k lies in block (RPK k) / 16 whatever the lane); the cache offset
+    // within a block and the shared-memory offset are per-lane constants plus
+    // compile-time terms, the swizzle term cycling with period 8 / RPK
+    constexpr int RPK = 32 / CH;
+    static_assert(C::kFp8 || (32 % CH == 0 && 8 % RPK == 0), "whole rows per chunk index");
+    constexpr int NXT = 8 / RPK;
+    const int lrow = lane / CH, lcc = lane % CH;
+    const uint32_t lsrc = (uint32_t)lrow * (uint32_t)job.row_stride + 16u * lcc;
+    const uint32_t lbase = (uint32_t)((lcc >> 3) * (T * 128) + lrow * 128);
+    uint32_t xt[NXT];
+#pragma unroll
+    for (int i = 0; i < NXT; ++i) xt[i] = (uint32_t)(((lcc & 7) ^ ((lrow + RPK * i) & 7)) << 4);
     bool q_landed = false;
     // fp8: step u's K rows (blocks of the range) and V rows (valid tokens)
     // into this warp's raw staging slot, cache layout; lane l: chunks l, l + 32, ...
@@ -310,16 +324,22 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
         for (int j = 0; j < SB; ++j) ph[j] = __shfl_sync(0xffffffffu, entry, j);
         if ((u + 1) * SB <= nb && (u + 1) * T <= job.kv_valid) {
           // interior step: every block and every row exists
+          const uint8_t* kb[SB];
+          const uint8_t* vb[SB];
+#pragma unroll
+          for (int j = 0; j < SB; ++j) {
+            const size_t b = (size_t)ph[j] * kBS * job.row_stride + lsrc;
+            kb[j] = job.k_head + b;
+            vb[j] = job.v_head + b;
+          }
 #pragma unroll
           for (int k = 0; k < PER; ++k) {
-            const int c = lane + 32 * k;
-            const int row = c / CH, cc = c % CH;
-            const int j = row / kBS, r = row % kBS;
-            const uint32_t off = C::sw128(T, row, 16 * cc);
-            const size_t src = ((size_t)ph[j] * kBS + r) * job.row_stride + 16 * cc;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(kbuf + off), "l"(job.k_head + src)
+            const int j = (RPK * k) / kBS, ro = (RPK * k) % kBS;  // block, row offset beyond lrow (compile-time)
+            const uint32_t so = (uint32_t)ro * (uint32_t)job.row_stride;
+            const uint32_t off = lbase + RPK * k * 128 + xt[k % NXT];
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(kbuf + off), "l"(kb[j] + so)
                          : "memory");
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(vbuf + off), "l"(job.v_head + src)
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(vbuf + off), "l"(vb[j] + so)
                          : "memory");
           }
         } else {
