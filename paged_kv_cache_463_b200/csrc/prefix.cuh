@@ -408,10 +408,12 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
       }
       if (lane == 0) {  // S = Q K^T of step u into S buffer cb, over 16-wide slices of D
         tc_fence_after();
+        // a slice's descriptor is the operand's with its byte offset / 16 added to the start-address field
+        const uint64_t a0 = umma_desc(qa, 16, 1024, kUmmaSwizzle128), b0 = umma_desc(kbuf, 16, 1024, kUmmaSwizzle128);
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint64_t a = umma_desc(qa + (k >> 2) * (kPrefixRows * 128) + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
-          const uint64_t b = umma_desc(kbuf + (k >> 2) * C::BUF_SUB + (k & 3) * 32, 16, 1024, kUmmaSwizzle128);
+          const uint64_t a = a0 + (uint64_t)((((k >> 2) * (kPrefixRows * 128) + (k & 3) * 32)) >> 4);
+          const uint64_t b = b0 + (uint64_t)((((k >> 2) * C::BUF_SUB + (k & 3) * 32)) >> 4);
           umma_f16(tmem + C::S_COL + cb * T, a, b, idS, k > 0);
         }
         umma_commit(sfull0 + 8 * cb);
@@ -442,9 +444,10 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
         tc_fence_after();
         const uint32_t pt = tmem + C::S_COL + cb * T;
         const uint32_t va = base + C::OFF_V + cb * C::BUF_BYTES;
+        const uint64_t v0 = umma_desc(va, C::BUF_SUB, 1024, kUmmaSwizzle128);
 #pragma unroll
         for (int k = 0; k < T / 16; ++k) {  // 16-token slices (one block each)
-          const uint64_t b = umma_desc(va + k * (kBS * 128), C::BUF_SUB, 1024, kUmmaSwizzle128);
+          const uint64_t b = v0 + (uint64_t)((k * (kBS * 128)) >> 4);
           umma_f16_ts(tmem + C::O_COL, pt + 8 * k, b, idO, (u > 0 || k > 0) ? 1 : 0);
         }
         umma_commit(pvdone0 + 8 * cb);
