@@ -293,13 +293,17 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
     // into this warp's raw staging slot, cache layout; lane l: chunks l, l + 32, ...
     auto fetch_raw = [&](int u) {
       const uint32_t raw = base + C::OFF_RAW + w * C::RAW_BYTES;
+      int ph[SB];  // the step's block ids (one shuffle per block)
+#pragma unroll
+      for (int j = 0; j < SB; ++j) ph[j] = __shfl_sync(0xffffffffu, entry, j);
+      const bool interior = (u + 1) * SB <= nb && (u + 1) * T <= job.kv_valid;  // every block and row present
 #pragma unroll
       for (int kq = 0; kq < 2 * PER; ++kq) {
         const int which = kq >= PER, c = lane + 32 * (kq - which * PER);
         const int row = c / CH, cc = c % CH, j = row / kBS, r = row % kBS;
-        const int phys = __shfl_sync(0xffffffffu, entry, j);
+        const int phys = ph[j];
         const size_t src = ((size_t)phys * kBS + r) * job.row_stride + 16 * cc;
-        const bool have = which ? u * T + row < job.kv_valid : u * SB + j < nb;
+        const bool have = interior || (which ? u * T + row < job.kv_valid : u * SB + j < nb);
         if (have)
           asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(raw + which * (T * C::ROW_BYTES) +
                                                                       row * C::ROW_BYTES + 16 * cc),
@@ -373,6 +377,7 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
         // chunks read in batches of up to 16 (independent loads in flight), then converted and stored
         constexpr int NB = 2 * PER < 16 ? 2 * PER : 16;
         static_assert((2 * PER) % NB == 0, "whole batches");
+        const bool interior = (u + 1) * SB <= nb && (u + 1) * T <= job.kv_valid;  // every block and row present
 #pragma unroll
         for (int b0 = 0; b0 < 2 * PER; b0 += NB) {
           uint4 v[NB];
@@ -386,7 +391,7 @@ __device__ __forceinline__ void stacked_attention(const StackedJob& job, const R
           for (int q = 0; q < NB; ++q) {
             const int kq = b0 + q, which = kq >= PER, c = lane + 32 * (kq - which * PER);
             const int row = c / CH, cc = c % CH, j = row / kBS;
-            const bool have = which ? u * T + row < job.kv_valid : u * SB + j < nb;
+            const bool have = interior || (which ? u * T + row < job.kv_valid : u * SB + j < nb);
             uint32_t h[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
             if (have) {
               e4m3x4_to_f16x2x2(v[q].x, h[0], h[1]);
